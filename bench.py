@@ -1,0 +1,419 @@
+"""Benchmark of the partitioned-attention step with selective state reuse.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: the plan, the
+partial attention of the fresh pairs and the log-sum-exp merge (with the
+cache refreshed in place), through the library's C ABI.  The default
+workload is the frame-tile sparse attention over a 29-frame 720p latent
+(8 frames x 3600 tokens, B=1, H=24, d=96).  Metric: effective attention
+TFLOP/s, counting only the freshly computed (query partition, KV partition)
+blocks: 4 * d * B * H * sum over fresh pairs of L_i * L_j.
+
+Several GPUs run independent replicas (one process per GPU under torchrun);
+the path has no exchange between GPUs.  --impl reference times the fp64 CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import configs, inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = configs.FRAME_TILE.name
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ counting
+def pair_mask(w):
+    """Active pairs of the workload, from the library's host logic."""
+    import sparse_state_reuse_b200 as dt
+    g = dt.Geometry(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask())
+    return np.array(dt.ditango_slot_table(g)) >= 0
+
+
+def effective_flops(w, fresh_mask):
+    po = np.array(w.part_off())
+    L = np.diff(po)
+    return float(4.0 * w.d * w.BH * (np.outer(L, L) * fresh_mask).sum())
+
+
+def merge_bytes(w, A, fresh_mask, out_bytes_per_elem=2, writeback=False):
+    """Algorithmic HBM bytes of the merge: every active state read once
+    ((d+1) fp32 per row), the output written once (d elements + fp32 lse),
+    plus the write-back of fresh states when they are copied."""
+    po = np.array(w.part_off())
+    L = np.diff(po)
+    rows_states = (A.sum(axis=1) * L).sum() * w.BH
+    b = rows_states * (w.d + 1) * 4 + w.BH * w.N * (w.d * out_bytes_per_elem + 4)
+    if writeback:
+        b += (fresh_mask.sum(axis=1) * L).sum() * w.BH * (w.d + 1) * 4
+    return float(b)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def kernel_source_hash(name):
+    src = os.path.join(ROOT, "sparse_state_reuse_b200", "csrc", name)
+    h = hashlib.sha256()
+    for f in (src, os.path.join(ROOT, "sparse_state_reuse_b200", "csrc", "common.cuh")):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel_file, {}).get(workload)
+    if not e or e.get("source_hash") != kernel_source_hash(kernel_file):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import sparse_state_reuse_b200 as dt
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def up(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+
+    hq, hk, hv = (up(inputs.full(w, t)) for t in "qkv")
+    Q, K, V = (x.to(dev) for x in (hq, hk, hv))
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask(),
+                                 device=dev)
+    if w.reuses:
+        Kp = up(inputs.full(w, "k", prev=True)).to(dev)
+        Vp = up(inputs.full(w, "v", prev=True)).to(dev)
+        pa.plan_step(anchor=True)
+        pa.partial(Q, Kp, Vp)          # anchor step: the cache of the previous denoising step
+        torch.cuda.synchronize()
+        del Kp, Vp
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device=dev)
+    out_lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    kw = dict(band_k=w.band_k, budget=w.budget, anchor=w.anchor)
+
+    # one step to learn the plan (the fresh set is the same every step here)
+    with torch.cuda.stream(stream):
+        pa.step(Q, K, V, out, out_lse, stream=stream, **kw)
+    stream.synchronize()
+    plan = pa.plan.cpu().numpy().reshape(w.P, w.P)
+    A = plan != 0
+    fresh = plan == 1
+    flops = effective_flops(w, fresh)
+    mbytes = merge_bytes(w, A, fresh)
+    launches_per_step = (1 if w.anchor else 2) + 1 + 1
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    n_ev = args.steps
+    e_part0, e_part1 = [ev() for _ in range(n_ev)], [ev() for _ in range(n_ev)]
+    e_merge1 = [ev() for _ in range(n_ev)]
+    e_start, e_end = ev(), ev()
+
+    def one_step(t=None):
+        with torch.cuda.stream(stream):
+            pa.plan_step(w.band_k, w.budget, w.anchor, stream=stream)
+            if t is not None:
+                e_part0[t].record(stream)
+            pa.partial(Q, K, V, stream=stream)
+            if t is not None:
+                e_part1[t].record(stream)
+            pa.merge(out, out_lse, stream=stream)
+            if t is not None:
+                e_merge1[t].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    stream.synchronize()
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = ClockSampler(local_rank)
+    clk.start()
+    time.sleep(0.3)
+    e_start.record(stream)
+    for t in range(args.steps):
+        one_step(t)
+    e_end.record(stream)
+    stream.synchronize()
+    clocks = clk.stop()
+    torch.cuda.synchronize()
+    ms = e_start.elapsed_time(e_end)
+    part_ms = float(np.mean([e_part0[t].elapsed_time(e_part1[t]) for t in range(n_ev)]))
+    merge_ms = float(np.mean([e_part1[t].elapsed_time(e_merge1[t]) for t in range(n_ev)]))
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+        dist.barrier()
+    status = int(pa.status.item())
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+
+    # end to end through the public API: pinned host inputs in, result out
+    hq_p, hk_p, hv_p = (x.pin_memory() for x in (hq, hk, hv))
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_lse = torch.empty(out_lse.shape, dtype=out_lse.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            Q.copy_(hq_p, non_blocking=True)
+            K.copy_(hk_p, non_blocking=True)
+            V.copy_(hv_p, non_blocking=True)
+            pa.step(Q, K, V, out, out_lse, stream=stream, **kw)
+            h_out.copy_(out, non_blocking=True)
+            h_lse.copy_(out_lse, non_blocking=True)
+
+    e2e_step()
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    a, b = ev(), ev()
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    stream.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
+
+    ms_step = ms / args.steps
+    peaks, peak_src = load_peaks()
+    tflops_part = flops / (part_ms * 1e-3) / 1e12
+    peak_t = float(peaks.get("bf16_tflops_sustained" if args.steps * ms_step > 2000 else "bf16_tflops"))
+    merge_gbs = mbytes / (merge_ms * 1e-3) / 1e9
+    traffic = recorded_traffic("attn_partial.cu", w.name)
+    res = {
+        "metric": "effective attention TFLOP/s (fresh blocks only) at 1 B200; tokens/s",
+        "value": round(world * flops / (ms_step * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s",
+        "tokens_per_s": round(world * w.B * w.N / (ms_step * 1e-3), 1),
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, shaped like the pages' workloads)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "P": w.P,
+                   "frames": w.F, "fresh_pairs": int(fresh.sum()), "active_pairs": int(A.sum()),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (Q/K/V %.0f MB, states %.0f MB)" % (
+                       h2d / 1e6, pa.state_O.numel() * 4 / 1e6)},
+        "roofline": {"bound": "tensor", "kernel": "attn_partial", "achieved": round(tflops_part, 2),
+                     "peak": peak_t, "unit": "TFLOP/s", "frac": round(tflops_part / peak_t, 4),
+                     "peak_source": peak_src, "traffic": traffic,
+                     "kernel_ms": round(part_ms, 4),
+                     "algorithmic_flops_per_launch": flops},
+        "merge_roofline": {"bound": "hbm", "achieved": round(merge_gbs, 1),
+                           "peak": float(peaks.get("hbm_gbs")), "unit": "GB/s",
+                           "frac": round(merge_gbs / float(peaks.get("hbm_gbs")), 4),
+                           "kernel_ms": round(merge_ms, 4),
+                           "algorithmic_bytes_per_launch": mbytes,
+                           "traffic": recorded_traffic("merge.cu", w.name)},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    return res
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(w, rng_seed, rows_per_sample, deadline_s):
+    """Time the fp64 oracle on seeded (b, h, partition, row-block) samples of
+    the workload until deadline_s of CPU work; returns (flops, seconds, desc)."""
+    from oracle import masks as OM, step as OS
+    from oracle.plan import PLAN_FRESH
+    A = OM.pair_mask(w.part_off(), w.frame_off(), w.frame_mask())
+    plan = np.where(A, PLAN_FRESH, 0).astype(np.int8)  # the fresh work of the step
+    rng = np.random.default_rng(rng_seed)
+    po = w.part_off()
+    flops, secs, n = 0.0, 0.0, 0
+    while secs < deadline_s:
+        bh = int(rng.integers(w.BH))
+        b, h = divmod(bh, w.H)
+        i = int(rng.integers(w.P))
+        lo, hi = po[i], po[i + 1]
+        r0 = int(rng.integers(lo, max(lo + 1, hi - rows_per_sample)))
+        rows = np.arange(r0, min(hi, r0 + rows_per_sample))
+        q = inputs.slab_f64(w, "q", b, h)
+        k = inputs.slab_f64(w, "k", b, h)
+        v = inputs.slab_f64(w, "v", b, h)
+        t0 = time.perf_counter()
+        OS.step_rows(q, k, v, k, v, plan, po, i, rows, w.frame_off(), w.frame_mask())
+        secs += time.perf_counter() - t0
+        keys = sum(po[j + 1] - po[j] for j in range(w.P) if A[i, j])
+        flops += 4.0 * w.d * rows.size * keys
+        n += 1
+    return flops, secs, f"{n} samples of {rows_per_sample} query rows x all active KV partitions, one (b,h) each"
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([x.get("num_threads", 1) for x in info] or [1])
+    except Exception:
+        return cpu_cores()
+
+
+def run_reference(args, w):
+    per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, 7, 128, per_step / 4)
+    tot_f, tot_s, desc = 0.0, 0.0, ""
+    for s in range(args.steps):
+        f, sec, desc = oracle_sample(w, 1000 + s, 128, per_step)
+        tot_f += f
+        tot_s += sec
+    val = tot_f / tot_s / 1e12
+    return {
+        "impl": "reference",
+        "metric": "effective attention TFLOP/s (fresh blocks only) at 1 B200; tokens/s",
+        "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 values)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "P": w.P},
+        "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(configs.BY_NAME))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = configs.BY_NAME[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, w, rank, world, local_rank)
+        if rank == 0 and world == 1:
+            f, s, desc = oracle_sample(w, 5, 128, args.cpu_baseline_seconds)
+            res["cpu_baseline"] = {"value": round(f / s / 1e12, 6), "unit": "TFLOP/s",
+                                   "cores": blas_threads(), "kind": "oracle", "sample": desc}
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

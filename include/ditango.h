@@ -1,0 +1,206 @@
+/*
+ * ditango.h -- C ABI of the partitioned-attention hot path with selective
+ * attention-state reuse, for NVIDIA B200 (sm_100a).
+ *
+ * What it computes (sources by page title and section):
+ *  - "DiTango: Cost-Effective Parallel Diffusion Generation with Selective
+ *    Attention State Reuse", technical summary:
+ *      Metodologia: the token sequence is split into P context partitions and
+ *        attention is computed per (query partition i, KV partition j) pair;
+ *        near partitions contribute most (spatial locality).
+ *      1. Anchor-Guided Selection Planner: per pair, recompute ("fresh") or
+ *        reuse the previous denoising step's attention state, guided by the
+ *        partition's importance w; anchor steps recompute everything.
+ *      2. State-Centric Parallel Runtime, "Composizione dello Stato": an
+ *        attention state is (output, log-sum-exp); states are cached instead
+ *        of raw K/V and compose associatively and commutatively.
+ *  - "Efficient-vDiT: Efficient Video Diffusion Transformers With Attention
+ *    Tile", abstract: a frame-tile sparse mask whose cost grows linearly
+ *    with the number of frames.
+ *
+ * Conventions shared by every entry point
+ *  - Every buffer is allocated by the caller.  "dev" marks device pointers,
+ *    "host" host pointers.  The library keeps no pointer after a call
+ *    returns and allocates no device memory.
+ *  - Every device-side call is asynchronous on `stream` (a cudaStream_t;
+ *    NULL is the legacy default stream) and never synchronises the host.
+ *  - Arguments are validated before anything is launched: a bad argument
+ *    returns DITANGO_ERR_INVALID, a valid but unsupported shape returns
+ *    DITANGO_ERR_UNSUPPORTED, a failed launch returns DITANGO_ERR_CUDA.
+ *    Device-side failures (a pipeline wait that exceeded its time limit) are
+ *    written as a status code into `dev_status` where a call takes one.
+ *  - Token order is frame-major; partitions are contiguous token ranges.
+ *  - State layout ("state buffer"): O is float32 [n_idx][B*H][Lmax][d] and
+ *    lse is float32 [n_idx][B*H][Lmax], where Lmax = max partition length
+ *    (ditango_state_rows) and the leading index is either the slot of an
+ *    active pair (row-major rank of the active pairs, see ditango_slot_table)
+ *    or the position of a pair in the fresh list.  Row r of pair (i, j)
+ *    holds query token part_off[i] + r; rows r >= L_i are never written.
+ *    O is normalised (sum_k softmax_k v_k) and lse is the natural
+ *    log-sum-exp of the scaled logits.
+ *  - Plan codes: 0 skip (masked pair), 1 fresh, 2 reuse.
+ */
+#ifndef DITANGO_H
+#define DITANGO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DITANGO_OK = 0,
+  DITANGO_ERR_INVALID = 1,      /* bad argument (null, negative, inconsistent) */
+  DITANGO_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels handle */
+  DITANGO_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  DITANGO_ERR_TIMEOUT = 4       /* device: a pipeline wait exceeded its limit */
+} ditango_status;
+
+enum { DITANGO_PLAN_SKIP = 0, DITANGO_PLAN_FRESH = 1, DITANGO_PLAN_REUSE = 2 };
+
+typedef void *ditango_stream; /* cudaStream_t */
+
+/* Geometry of one attention call; host struct, read during the call only.
+ *   B, H     batch and heads; N tokens; d head dim in {64, 96, 128}.
+ *   P        partitions, 1 <= P <= 64; part_off host int32 [P+1],
+ *            part_off[0] = 0 < part_off[1] < ... < part_off[P] = N.
+ *   F        frames of the frame-tile mask, 0 = no mask (all pairs active);
+ *            else 1 <= F <= 64, frame_off host int32 [F+1] (same rules as
+ *            part_off) and frame_mask host uint8 [F*F], row = query frame,
+ *            nonzero = the query frame may attend the key frame.  Every
+ *            partition must lie inside one frame (else UNSUPPORTED): the mask
+ *            is then exact at pair granularity.
+ *   q/k/v_strides  element strides of the (b, h, n) dimensions of the bf16
+ *            Q, K, V tensors; the d dimension is contiguous.  Strides times 2
+ *            bytes must be multiples of 16 and the base pointers 16-byte
+ *            aligned (TMA). */
+typedef struct {
+  int32_t B, H, N, d;
+  int32_t P, F;
+  const int32_t *part_off;
+  const int32_t *frame_off;
+  const uint8_t *frame_mask;
+  int64_t q_strides[3];
+  int64_t k_strides[3];
+  int64_t v_strides[3];
+} ditango_geom;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int32_t ditango_version(void);
+
+/* Static string for a status code. */
+const char *ditango_status_string(int32_t status);
+
+/* Validate a geometry without launching anything. */
+ditango_status ditango_check_geom(const ditango_geom *g);
+
+/* Number of active pairs (= slots): pairs (i, j) whose tokens the frame mask
+ * lets attend each other (all P*P when F = 0).  Returns -1 on a bad geometry. */
+int64_t ditango_num_active(const ditango_geom *g);
+
+/* Lmax, rows per (index, b*h) block of a state buffer. -1 on a bad geometry. */
+int64_t ditango_state_rows(const ditango_geom *g);
+
+/* Host helper: slot_out host int32 [P*P] receives the slot of each pair,
+ * -1 for masked pairs (row-major rank of the active pairs). */
+ditango_status ditango_slot_table(const ditango_geom *g, int32_t *slot_out);
+
+/* Bytes of device scratch ditango_plan needs. */
+size_t ditango_plan_workspace_size(const ditango_geom *g);
+
+/* Plan: per pair, fresh or reuse (DiTango, 1. Anchor-Guided Selection
+ * Planner; spatial locality from Metodologia).
+ *   cache_lse    dev float32 state-buffer lse indexed by slot (the previous
+ *                step's cached states); may be NULL when anchor != 0.
+ *   cache_valid  dev uint8 [slots] (nonzero = slot holds a state) or NULL
+ *                (all valid).  An invalid slot is forced fresh and holds no
+ *                mass.
+ *   band_k       pairs with |i - j| <= band_k are always fresh.
+ *   budget       fraction of active pairs to recompute: the fresh count is
+ *                max(|band|, floor(budget * active + 1e-9)); the pairs added
+ *                beyond the band are those of largest mass w, ties to the
+ *                lower linear index i*P + j.
+ *   anchor       nonzero: every active pair fresh (an anchor step).
+ * w[i][j] = mean over (b, h, rows r of partition i) of
+ *           exp(lse_ij[r]) / sum_{j' active, valid} exp(lse_ij'[r]),
+ * computed in float32 with a fixed reduction order (deterministic).
+ * Outputs (dev): plan int8 [P*P]; fresh_list int32 [slots] = linear indices
+ * i*P + j of the fresh pairs in row-major order; counts int32 [2] = {fresh,
+ * reuse}; score_out float32 [P*P] (w, 0 for masked pairs) or NULL.
+ * workspace: dev, >= ditango_plan_workspace_size bytes. */
+ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
+                            const uint8_t *cache_valid, int32_t band_k, double budget,
+                            int32_t anchor, int8_t *plan, int32_t *fresh_list,
+                            int32_t *counts, float *score_out, void *workspace,
+                            size_t workspace_bytes, ditango_stream stream);
+
+/* Partial attention states of the fresh pairs (tcgen05 tensor cores, TMA).
+ * For each fresh pair (i, j) = fresh_list[f], f < counts[0] (read on the
+ * device), and each (b, h): S = Q_i K_j^T * scale, O = softmax(S) V_j
+ * (normalised), lse = logsumexp(S) -- the state of DiTango's
+ * "Composizione dello Stato".  bf16 inputs, fp32 accumulation and softmax;
+ * the probabilities are rounded to bf16 for the P V product.
+ *   Q, K, V      dev bf16 (uint16 bit patterns) with the geometry's strides.
+ *   scale        logit scale; 0 means 1/sqrt(d).
+ *   out_O/out_lse  dev state buffer; index = f (out_by_slot = 0) or the
+ *                pair's slot (out_by_slot = 1, e.g. writing the cache in
+ *                place).  Must hold counts[0] (resp. all slots) indices.
+ *   out_valid    dev uint8 [slots] or NULL; with out_by_slot = 1 the written
+ *                slots are set to 1.
+ *   dev_status   dev int32 or NULL; set to DITANGO_ERR_TIMEOUT if a pipeline
+ *                wait exceeded the limit (the kernel then stops cleanly).
+ */
+ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q,
+                                    const uint16_t *K, const uint16_t *V,
+                                    const int32_t *fresh_list, const int32_t *counts,
+                                    float scale, float *out_O, float *out_lse,
+                                    int32_t out_by_slot, uint8_t *out_valid,
+                                    int32_t *dev_status, ditango_stream stream);
+
+/* Merge: the final output of every token is the log-sum-exp composition of
+ * the states of its partition's active pairs (DiTango, "Composizione dello
+ * Stato"): L = log sum_j exp(lse_j), O = sum_j exp(lse_j - L) O_j, with
+ * fresh states read from part_O/part_lse (indexed by fresh-list position)
+ * and reused ones from cache_O/cache_lse (indexed by slot).  part_O = NULL
+ * means the fresh states were already written into the cache slots
+ * (ditango_attn_partial with out_by_slot = 1).
+ *   plan          dev int8 [P*P] from ditango_plan.
+ *   writeback     nonzero: also copy each fresh state into its cache slot
+ *                 and mark cache_valid (ignored when part_O is NULL).
+ *   out           dev [B, H, N, d] (element strides out_strides for b, h, n;
+ *                 NULL = contiguous), bf16 bits (out_is_fp32 = 0) or float32.
+ *   out_lse       dev float32 [B, H, N] or NULL.
+ * A token whose partition has no active pair gets O = 0, lse = -inf. */
+ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan,
+                             const float *part_O, const float *part_lse,
+                             float *cache_O, float *cache_lse, uint8_t *cache_valid,
+                             int32_t writeback, void *out, int32_t out_is_fp32,
+                             const int64_t *out_strides, float *out_lse,
+                             ditango_stream stream);
+
+/* Cache update: copy the fresh states (indexed by fresh position) into their
+ * cache slots and mark them valid -- the write half of an anchor step
+ * (DiTango, "Anchor Steps": everything is recomputed and the cache
+ * refreshed). */
+ditango_status ditango_cache_update(const ditango_geom *g, const int8_t *plan,
+                                    const float *part_O, const float *part_lse,
+                                    float *cache_O, float *cache_lse,
+                                    uint8_t *cache_valid, ditango_stream stream);
+
+/* Time limit, in nanoseconds, of every wait inside the kernels (default
+ * 1e9).  Process-wide; read at each launch. */
+void ditango_set_wait_limit_ns(int64_t ns);
+
+/* Failure-detection self-test: launches one block that waits on a barrier
+ * nothing will complete, with a limit of limit_ns; the kernel returns and
+ * writes DITANGO_ERR_TIMEOUT into dev_status (dev int32).  Exercises the
+ * same bounded wait the pipeline kernels use. */
+ditango_status ditango_selftest_bounded_wait(int64_t limit_ns, int32_t *dev_status,
+                                             ditango_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DITANGO_H */

@@ -17,7 +17,8 @@ Readings of what the pages leave open (the plainest ones that fit the rest):
     the band is fresh even above the budget; the budget fills with the
     highest-w active pairs outside the band;
   * equal w: the lower linear index i * P + j is taken first;
-  * a pair whose cache slot was never written is fresh regardless of budget;
+  * a pair whose cache slot was never written is fresh regardless of budget
+    and holds no mass;
   * one plan per (i, j), shared by every batch entry and head;
   * the ranking decision is taken on w rounded to float32 (the precision the
     CUDA path holds w in).
@@ -31,16 +32,19 @@ import numpy as np
 PLAN_SKIP, PLAN_FRESH, PLAN_REUSE = 0, 1, 2
 
 
-def mass_scores(cache_lse, A, part_off):
+def mass_scores(cache_lse, A, part_off, valid=None):
     """w [P, P] (fp64) from cached log-sum-exps.
 
     cache_lse: [slots, BH, Lmax] array indexed by slot (row-major rank of the
     active pair); row r of pair (i, j) is cache_lse[slot(i,j), :, r] for
-    r < L_i.  Inactive pairs get w = 0.
+    r < L_i.  Inactive pairs get w = 0.  valid: optional bool [slots]; a slot
+    that was never written holds no state and therefore no mass.
     """
     A = np.asarray(A, dtype=bool)
     P = A.shape[0]
     lse_all = np.asarray(cache_lse)
+    if valid is not None:
+        lse_all = np.where(np.asarray(valid, dtype=bool)[:, None, None], lse_all, -np.inf)
     w = np.zeros((P, P), dtype=np.float64)
     slot = 0
     for i in range(P):

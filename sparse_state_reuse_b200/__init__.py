@@ -1,0 +1,92 @@
+"""B200 partitioned attention with selective attention-state reuse.
+
+The token sequence is split into P context partitions; for every (query
+partition, KV partition) pair the plan either recomputes the attention state
+(output, log-sum-exp) or reuses the one cached at the previous denoising
+step, and the states of each query partition are composed by an exact
+log-sum-exp merge (DiTango: "Cost-Effective Parallel Diffusion Generation
+with Selective Attention State Reuse").  An optional frame-tile mask keeps
+only some frame tiles (Efficient-vDiT: "Efficient Video Diffusion
+Transformers With Attention Tile").
+
+All compute runs in libditango.so (CUDA, sm_100a) through its C ABI
+(include/ditango.h); this package only marshals arguments.  PyTorch is used
+for device memory and streams.
+"""
+from __future__ import annotations
+
+from ._abi import (  # noqa: F401
+    DitangoError, Geometry, PLAN_FRESH, PLAN_REUSE, PLAN_SKIP, LIB_PATH, EXPORTED,
+    ditango_version, ditango_check_geom, ditango_num_active, ditango_state_rows,
+    ditango_slot_table, ditango_plan_workspace_size, ditango_plan, ditango_attn_partial,
+    ditango_merge, ditango_cache_update, ditango_set_wait_limit_ns,
+    ditango_selftest_bounded_wait, status_string,
+)
+
+
+class PartitionedAttention:
+    """Device buffers for one geometry and the three-call step.
+
+    The state buffer (O float32 [slots, B*H, Lmax, d], lse float32
+    [slots, B*H, Lmax]) is the attention-state cache: a step writes its fresh
+    states into their slots and the merge reads every active pair from it, so
+    after a step the cache holds this step's fresh states and the reused ones.
+    """
+
+    def __init__(self, B, H, N, d, part_off, frame_off=None, frame_mask=None,
+                 device="cuda", strides=None):
+        import torch
+        self.B, self.H, self.N, self.d = B, H, N, d
+        self.part_off = list(part_off)
+        self.frame_off = None if frame_off is None else list(frame_off)
+        self.frame_mask = frame_mask
+        self.device = torch.device(device)
+        self.geom = self._geometry(strides)
+        self.P = self.geom.P
+        self.n_slots = ditango_num_active(self.geom)
+        self.Lmax = ditango_state_rows(self.geom)
+        BH = B * H
+        dev = self.device
+        self.state_O = torch.empty((self.n_slots, BH, self.Lmax, d), dtype=torch.float32, device=dev)
+        self.state_lse = torch.empty((self.n_slots, BH, self.Lmax), dtype=torch.float32, device=dev)
+        self.valid = torch.zeros(self.n_slots, dtype=torch.uint8, device=dev)
+        self.plan = torch.zeros(self.P * self.P, dtype=torch.int8, device=dev)
+        self.fresh_list = torch.zeros(max(self.n_slots, 1), dtype=torch.int32, device=dev)
+        self.counts = torch.zeros(2, dtype=torch.int32, device=dev)
+        self.score = torch.zeros(self.P * self.P, dtype=torch.float32, device=dev)
+        self.ws_bytes = ditango_plan_workspace_size(self.geom)
+        self.workspace = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def _geometry(self, strides):
+        s = strides or (None, None, None)
+        return Geometry(self.B, self.H, self.N, self.d, self.part_off, self.frame_off,
+                        self.frame_mask, q_strides=s[0], k_strides=s[1], v_strides=s[2])
+
+    def _bind(self, Q, K, V):
+        want = tuple(tuple(t.stride()[:3]) for t in (Q, K, V))
+        have = (tuple(self.geom.g.q_strides), tuple(self.geom.g.k_strides), tuple(self.geom.g.v_strides))
+        if want != have:
+            self.geom = self._geometry(want)
+
+    def plan_step(self, band_k=0, budget=1.0, anchor=False, stream=None):
+        ditango_plan(self.geom, None if anchor else self.state_lse, self.valid, band_k, budget,
+                     anchor, self.plan, self.fresh_list, self.counts, self.score, self.workspace,
+                     self.ws_bytes, stream)
+
+    def partial(self, Q, K, V, scale=0.0, stream=None):
+        self._bind(Q, K, V)
+        ditango_attn_partial(self.geom, Q, K, V, self.fresh_list, self.counts, scale,
+                             self.state_O, self.state_lse, 1, self.valid, self.status, stream)
+
+    def merge(self, out, out_lse=None, stream=None):
+        import torch
+        ditango_merge(self.geom, self.plan, None, None, self.state_O, self.state_lse, self.valid, 0,
+                      out, out.dtype == torch.float32, tuple(out.stride()[:3]), out_lse, stream)
+
+    def step(self, Q, K, V, out, out_lse=None, band_k=0, budget=1.0, anchor=False, scale=0.0,
+             stream=None):
+        """plan -> partial attention of the fresh pairs -> merge, on one stream."""
+        self.plan_step(band_k, budget, anchor, stream)
+        self.partial(Q, K, V, scale, stream)
+        self.merge(out, out_lse, stream)

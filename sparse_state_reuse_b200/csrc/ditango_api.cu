@@ -1,0 +1,309 @@
+// Host side of the C ABI declared in include/ditango.h: argument checks,
+// the kernels' geometry, TMA tensor maps and launches.  No device memory is
+// allocated here.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace ditango {
+cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const CUtensorMap &tk,
+                                const CUtensorMap &tv, const int *fresh_list, const int *counts,
+                                float scale, float *out_O, float *out_lse, int out_by_slot,
+                                unsigned char *out_valid, int *dev_status, long long wait_limit_ns,
+                                int num_sms, cudaStream_t stream);
+size_t plan_workspace_bytes(const DevGeom &g);
+cudaError_t launch_plan(const DevGeom &g, const float *cache_lse, const unsigned char *cache_valid,
+                        int band_k, int target, int anchor, signed char *plan_out, int *fresh_list,
+                        int *counts, float *score_out, void *workspace, cudaStream_t stream);
+cudaError_t launch_merge(const DevGeom &g, const signed char *plan, const float *part_O,
+                         const float *part_lse, float *cache_O, float *cache_lse,
+                         unsigned char *cache_valid, int writeback, void *out, int out_is_fp32,
+                         long long osb, long long osh, long long osn, float *out_lse,
+                         cudaStream_t stream);
+cudaError_t launch_cache_update(const DevGeom &g, const signed char *plan, const float *part_O,
+                                const float *part_lse, float *cache_O, float *cache_lse,
+                                unsigned char *cache_valid, int num_sms, cudaStream_t stream);
+cudaError_t launch_bounded_wait_selftest(long long limit_ns, int *dev_status,
+                                         cudaStream_t stream);
+}  // namespace ditango
+
+using namespace ditango;
+
+namespace {
+
+long long g_wait_limit_ns = 1000000000LL;
+
+// Build the kernels' geometry; returns DITANGO_OK or the reason it cannot.
+ditango_status make_geom(const ditango_geom *in, DevGeom *out) {
+  if (!in) return DITANGO_ERR_INVALID;
+  if (in->B < 1 || in->H < 1 || in->N < 1 || in->P < 1 || in->d < 1) return DITANGO_ERR_INVALID;
+  if (in->P > kMaxP) return DITANGO_ERR_UNSUPPORTED;
+  if (!(in->d == 64 || in->d == 96 || in->d == 128)) return DITANGO_ERR_UNSUPPORTED;
+  if ((long long)in->B * in->H > 65535) return DITANGO_ERR_UNSUPPORTED;  // grid.z of the merge
+  if (!in->part_off) return DITANGO_ERR_INVALID;
+  if (in->part_off[0] != 0 || in->part_off[in->P] != in->N) return DITANGO_ERR_INVALID;
+  for (int p = 0; p < in->P; ++p)
+    if (in->part_off[p + 1] <= in->part_off[p]) return DITANGO_ERR_INVALID;
+  if (in->F < 0 || in->F > kMaxP) return in->F < 0 ? DITANGO_ERR_INVALID : DITANGO_ERR_UNSUPPORTED;
+  int part_frame[kMaxP];
+  if (in->F > 0) {
+    if (!in->frame_off || !in->frame_mask) return DITANGO_ERR_INVALID;
+    if (in->frame_off[0] != 0 || in->frame_off[in->F] != in->N) return DITANGO_ERR_INVALID;
+    for (int f = 0; f < in->F; ++f)
+      if (in->frame_off[f + 1] <= in->frame_off[f]) return DITANGO_ERR_INVALID;
+    // every partition inside one frame: the frame mask is then exact per pair
+    for (int p = 0; p < in->P; ++p) {
+      int f = 0;
+      while (in->frame_off[f + 1] <= in->part_off[p]) ++f;
+      if (in->part_off[p + 1] > in->frame_off[f + 1]) return DITANGO_ERR_UNSUPPORTED;
+      part_frame[p] = f;
+    }
+  }
+  DevGeom g;
+  std::memset(&g, 0, sizeof(g));
+  g.B = in->B;
+  g.H = in->H;
+  g.N = in->N;
+  g.d = in->d;
+  g.P = in->P;
+  g.BH = in->B * in->H;
+  int lmax = 0;
+  for (int p = 0; p <= in->P; ++p) g.part_off[p] = in->part_off[p];
+  for (int p = 0; p < in->P; ++p) {
+    int L = in->part_off[p + 1] - in->part_off[p];
+    if (L > lmax) lmax = L;
+  }
+  g.Lmax = lmax;
+  int slot = 0;
+  for (int i = 0; i < in->P; ++i) {
+    g.row_start[i] = slot;
+    unsigned long long m = 0;
+    for (int j = 0; j < in->P; ++j) {
+      bool act = true;
+      if (in->F > 0) act = in->frame_mask[part_frame[i] * in->F + part_frame[j]] != 0;
+      if (act) {
+        m |= 1ull << j;
+        ++slot;
+      }
+    }
+    g.row_mask[i] = m;
+  }
+  g.row_start[in->P] = slot;
+  g.n_active = slot;
+  *out = g;
+  return DITANGO_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool strides_ok(const int64_t s[3]) {
+  for (int k = 0; k < 3; ++k)
+    if (s[k] <= 0 || ((s[k] * 2) % 16) != 0 || s[k] * 2 >= (1LL << 40)) return false;
+  return true;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 4-D map over a bf16 [B, H, N, d] tensor (d contiguous), box 64 x 128 rows,
+// 128-byte swizzle; columns past d and rows past N read as zero.
+bool make_qkv_map(CUtensorMap *m, const void *base, const DevGeom &g, const int64_t s[3]) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)g.d, (cuuint64_t)g.N, (cuuint64_t)g.H, (cuuint64_t)g.B};
+  cuuint64_t strides[3] = {(cuuint64_t)(s[2] * 2), (cuuint64_t)(s[1] * 2), (cuuint64_t)(s[0] * 2)};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms_current() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n;
+}
+
+ditango_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return DITANGO_OK;
+  (void)cudaGetLastError();
+  return DITANGO_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t ditango_version(void) { return 10000; }
+
+const char *ditango_status_string(int32_t s) {
+  switch (s) {
+    case DITANGO_OK: return "ok";
+    case DITANGO_ERR_INVALID: return "invalid argument";
+    case DITANGO_ERR_UNSUPPORTED: return "unsupported shape";
+    case DITANGO_ERR_CUDA: return "CUDA error";
+    case DITANGO_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+ditango_status ditango_check_geom(const ditango_geom *g) {
+  DevGeom dg;
+  return make_geom(g, &dg);
+}
+
+int64_t ditango_num_active(const ditango_geom *g) {
+  DevGeom dg;
+  if (make_geom(g, &dg) != DITANGO_OK) return -1;
+  return dg.n_active;
+}
+
+int64_t ditango_state_rows(const ditango_geom *g) {
+  DevGeom dg;
+  if (make_geom(g, &dg) != DITANGO_OK) return -1;
+  return dg.Lmax;
+}
+
+ditango_status ditango_slot_table(const ditango_geom *g, int32_t *slot_out) {
+  DevGeom dg;
+  ditango_status st = make_geom(g, &dg);
+  if (st != DITANGO_OK) return st;
+  if (!slot_out) return DITANGO_ERR_INVALID;
+  for (int i = 0; i < dg.P; ++i)
+    for (int j = 0; j < dg.P; ++j)
+      slot_out[i * dg.P + j] = ((dg.row_mask[i] >> j) & 1ull) ? slot_of(dg, i, j) : -1;
+  return DITANGO_OK;
+}
+
+size_t ditango_plan_workspace_size(const ditango_geom *g) {
+  DevGeom dg;
+  if (make_geom(g, &dg) != DITANGO_OK) return 0;
+  return plan_workspace_bytes(dg);
+}
+
+ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
+                            const uint8_t *cache_valid, int32_t band_k, double budget,
+                            int32_t anchor, int8_t *plan, int32_t *fresh_list, int32_t *counts,
+                            float *score_out, void *workspace, size_t workspace_bytes,
+                            ditango_stream stream) {
+  DevGeom dg;
+  ditango_status st = make_geom(g, &dg);
+  if (st != DITANGO_OK) return st;
+  if (!plan || !fresh_list || !counts) return DITANGO_ERR_INVALID;
+  if (!anchor) {
+    if (!cache_lse || band_k < 0 || !(budget >= 0.0 && budget <= 1.0)) return DITANGO_ERR_INVALID;
+    if (!workspace || workspace_bytes < plan_workspace_bytes(dg)) return DITANGO_ERR_INVALID;
+  }
+  int n_band = 0;
+  for (int i = 0; i < dg.P; ++i)
+    for (int j = 0; j < dg.P; ++j)
+      if (((dg.row_mask[i] >> j) & 1ull) && std::abs(i - j) <= band_k) ++n_band;
+  int target = (int)std::floor(budget * (double)dg.n_active + 1e-9);
+  if (target < n_band) target = n_band;
+  if (target > dg.n_active) target = dg.n_active;
+  dg.n_band = n_band;
+  return cuda_status(launch_plan(dg, cache_lse, cache_valid, band_k, target, anchor ? 1 : 0,
+                                 reinterpret_cast<signed char *>(plan), fresh_list, counts,
+                                 score_out, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q, const uint16_t *K,
+                                    const uint16_t *V, const int32_t *fresh_list,
+                                    const int32_t *counts, float scale, float *out_O,
+                                    float *out_lse, int32_t out_by_slot, uint8_t *out_valid,
+                                    int32_t *dev_status, ditango_stream stream) {
+  DevGeom dg;
+  ditango_status st = make_geom(g, &dg);
+  if (st != DITANGO_OK) return st;
+  if (!Q || !K || !V || !fresh_list || !counts || !out_O || !out_lse) return DITANGO_ERR_INVALID;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out_O))
+    return DITANGO_ERR_INVALID;
+  if (!strides_ok(g->q_strides) || !strides_ok(g->k_strides) || !strides_ok(g->v_strides))
+    return DITANGO_ERR_INVALID;
+  if (!(scale >= 0.f) || !std::isfinite(scale)) return DITANGO_ERR_INVALID;
+  if (scale == 0.f) scale = 1.f / std::sqrt((float)dg.d);
+  CUtensorMap tq, tk, tv;
+  if (!make_qkv_map(&tq, Q, dg, g->q_strides) || !make_qkv_map(&tk, K, dg, g->k_strides) ||
+      !make_qkv_map(&tv, V, dg, g->v_strides))
+    return DITANGO_ERR_CUDA;
+  return cuda_status(launch_attn_partial(dg, tq, tk, tv, fresh_list, counts, scale, out_O, out_lse,
+                                         out_by_slot ? 1 : 0, out_valid, dev_status,
+                                         g_wait_limit_ns, num_sms_current(),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan, const float *part_O,
+                             const float *part_lse, float *cache_O, float *cache_lse,
+                             uint8_t *cache_valid, int32_t writeback, void *out,
+                             int32_t out_is_fp32, const int64_t *out_strides, float *out_lse,
+                             ditango_stream stream) {
+  DevGeom dg;
+  ditango_status st = make_geom(g, &dg);
+  if (st != DITANGO_OK) return st;
+  if (!plan || !out) return DITANGO_ERR_INVALID;
+  if ((part_O == nullptr) != (part_lse == nullptr)) return DITANGO_ERR_INVALID;
+  if ((cache_O == nullptr) != (cache_lse == nullptr)) return DITANGO_ERR_INVALID;
+  if (part_O == nullptr && cache_O == nullptr) return DITANGO_ERR_INVALID;
+  if (writeback && part_O && !cache_O) return DITANGO_ERR_INVALID;
+  long long osb = (long long)dg.H * dg.N * dg.d, osh = (long long)dg.N * dg.d, osn = dg.d;
+  if (out_strides) {
+    osb = out_strides[0];
+    osh = out_strides[1];
+    osn = out_strides[2];
+    if (osb <= 0 || osh <= 0 || osn <= 0) return DITANGO_ERR_INVALID;
+  }
+  const int esz = out_is_fp32 ? 4 : 2;
+  if ((osb * esz) % 16 || (osh * esz) % 16 || (osn * esz) % 16 ||
+      (reinterpret_cast<uintptr_t>(out) % (out_is_fp32 ? 16 : 8)))
+    return DITANGO_ERR_INVALID;
+  return cuda_status(launch_merge(dg, reinterpret_cast<const signed char *>(plan), part_O,
+                                  part_lse, cache_O, cache_lse, cache_valid,
+                                  (writeback && part_O) ? 1 : 0, out, out_is_fp32 ? 1 : 0, osb,
+                                  osh, osn, out_lse, static_cast<cudaStream_t>(stream)));
+}
+
+ditango_status ditango_cache_update(const ditango_geom *g, const int8_t *plan,
+                                    const float *part_O, const float *part_lse, float *cache_O,
+                                    float *cache_lse, uint8_t *cache_valid,
+                                    ditango_stream stream) {
+  DevGeom dg;
+  ditango_status st = make_geom(g, &dg);
+  if (st != DITANGO_OK) return st;
+  if (!plan || !part_O || !part_lse || !cache_O || !cache_lse) return DITANGO_ERR_INVALID;
+  return cuda_status(launch_cache_update(dg, reinterpret_cast<const signed char *>(plan), part_O,
+                                         part_lse, cache_O, cache_lse, cache_valid,
+                                         num_sms_current(), static_cast<cudaStream_t>(stream)));
+}
+
+void ditango_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns = ns > 0 ? ns : 1; }
+
+ditango_status ditango_selftest_bounded_wait(int64_t limit_ns, int32_t *dev_status,
+                                             ditango_stream stream) {
+  if (!dev_status || limit_ns <= 0) return DITANGO_ERR_INVALID;
+  return cuda_status(
+      launch_bounded_wait_selftest(limit_ns, dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

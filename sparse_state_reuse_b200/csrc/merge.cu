@@ -1,0 +1,252 @@
+// Log-sum-exp merge of attention states and the cache write-back.
+//
+// DiTango, "Riepilogo Tecnico" -> Metodologia -> 2. State-Centric Parallel
+// Runtime, "Composizione dello Stato": the output of a query row is the
+// composition of the states of all active pairs of its partition,
+//   L = M + log sum_j exp(lse_j - M),  O = sum_j exp(lse_j - L) O_j,
+// fresh states coming from this step's partial buffer and reused ones from
+// the cache.  "Anchor Steps": the states computed fresh refresh the cache.
+//
+// The merge is HBM bound: one warp per token row, d/4 lanes each holding a
+// float4 of d; the loads of up to 8 states are issued before they are
+// consumed so that enough bytes are in flight.  The per-block table of
+// source pointers (fresh -> partial buffer at its fresh-list position,
+// reuse -> cache slot) is built once per (b*h, partition) in shared memory.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace ditango {
+namespace merge {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kRowsPerBlock = 128;
+constexpr int kUnroll = 8;
+
+struct Src {
+  const float *O;    // [Lmax][d] block of this (index, b*h)
+  const float *lse;  // [Lmax]
+  float *wbO;        // cache block to write back into, or null
+  float *wblse;
+};
+
+__device__ __forceinline__ void store_out(void *out, int is_fp32, size_t off, float4 v) {
+  if (is_fp32) {
+    *reinterpret_cast<float4 *>(static_cast<float *>(out) + off) = v;
+  } else {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t *>(&a);
+    u.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(out) + off) = u;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+merge_kernel(DevGeom g, const signed char *__restrict__ plan, const float *__restrict__ part_O,
+             const float *__restrict__ part_lse, float *cache_O, float *cache_lse,
+             unsigned char *cache_valid, int writeback, void *out, int out_is_fp32, long long osb,
+             long long osh, long long osn, float *__restrict__ out_lse) {
+  constexpr int G = D / 4;  // lanes carrying one row
+  const int i = blockIdx.y;
+  const int bh = blockIdx.z;
+  const int Li = g.part_off[i + 1] - g.part_off[i];
+  const int r0 = blockIdx.x * kRowsPerBlock;
+  if (r0 >= Li) return;
+  const int P = g.P;
+  __shared__ Src src[kMaxP];
+  __shared__ int s_nact, s_fresh_before;
+  __shared__ int warp_cnt[kWarps];
+
+  // fresh pairs before row i (row-major), for fresh-list positions
+  int cnt = 0;
+  for (int p = threadIdx.x; p < i * P; p += kThreads) cnt += (plan[p] == DITANGO_PLAN_FRESH);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if ((threadIdx.x & 31) == 0) warp_cnt[threadIdx.x >> 5] = cnt;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int fb = 0;
+    for (int w = 0; w < kWarps; ++w) fb += warp_cnt[w];
+    s_fresh_before = fb;
+    const size_t blk = (size_t)g.BH * g.Lmax;
+    int a = 0;
+    const int slot0 = g.row_start[i];
+    int fpos = fb;
+    for (int j = 0; j < P; ++j) {
+      if (!((g.row_mask[i] >> j) & 1ull)) continue;
+      const int code = plan[i * P + j];
+      const int slot = slot0 + __popcll(g.row_mask[i] & ((j == 0) ? 0ull : (~0ull >> (64 - j))));
+      Src s;
+      s.wbO = nullptr;
+      s.wblse = nullptr;
+      if (code == DITANGO_PLAN_FRESH) {
+        if (part_O != nullptr) {
+          s.O = part_O + ((size_t)fpos * blk + (size_t)bh * g.Lmax) * D;
+          s.lse = part_lse + (size_t)fpos * blk + (size_t)bh * g.Lmax;
+          if (writeback) {
+            s.wbO = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * D;
+            s.wblse = cache_lse + (size_t)slot * blk + (size_t)bh * g.Lmax;
+            if (cache_valid && bh == 0 && blockIdx.x == 0) cache_valid[slot] = 1;
+          }
+        } else {
+          s.O = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * D;
+          s.lse = cache_lse + (size_t)slot * blk + (size_t)bh * g.Lmax;
+        }
+        ++fpos;
+      } else if (code == DITANGO_PLAN_REUSE) {
+        s.O = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * D;
+        s.lse = cache_lse + (size_t)slot * blk + (size_t)bh * g.Lmax;
+      } else {
+        continue;  // active pair the plan skipped: contributes nothing
+      }
+      src[a++] = s;
+    }
+    s_nact = a;
+  }
+  __syncthreads();
+  const int nact = s_nact;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = bh / g.H, h = bh - (bh / g.H) * g.H;
+  const int rend = (r0 + kRowsPerBlock < Li) ? r0 + kRowsPerBlock : Li;
+
+  for (int r = r0 + warp; r < rend; r += kWarps) {
+    // weights: lane a holds state a (and a + 32)
+    float l0 = -INFINITY, l1 = -INFINITY;
+    if (lane < nact) l0 = __ldg(src[lane].lse + r);
+    if (lane + 32 < nact) l1 = __ldg(src[lane + 32].lse + r);
+    float M = fmaxf(l0, l1);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const bool dead = !(M > -INFINITY);
+    const float Ms = dead ? 0.f : M;
+    float e0 = expf(l0 - Ms), e1 = expf(l1 - Ms);
+    float S = e0 + e1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+    const float invS = dead ? 0.f : 1.f / S;
+    const float w0 = e0 * invS, w1 = e1 * invS;
+    const float L = dead ? -INFINITY : Ms + logf(S);
+
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const bool act = lane < G;
+    for (int a0 = 0; a0 < nact; a0 += kUnroll) {
+      float4 v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int a = a0 + u;
+        if (act && a < nact)
+          v[u] = __ldg(reinterpret_cast<const float4 *>(src[a].O + (size_t)r * D) + lane);
+        else
+          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int a = a0 + u;
+        const float wa = __shfl_sync(0xffffffffu, (a < 32) ? w0 : w1, a & 31);
+        if (a < nact) {
+          acc.x = fmaf(wa, v[u].x, acc.x);
+          acc.y = fmaf(wa, v[u].y, acc.y);
+          acc.z = fmaf(wa, v[u].z, acc.z);
+          acc.w = fmaf(wa, v[u].w, acc.w);
+          if (act && src[a].wbO) reinterpret_cast<float4 *>(src[a].wbO + (size_t)r * D)[lane] = v[u];
+        }
+      }
+    }
+    // write back the lse of fresh states
+    if (lane < nact && src[lane].wblse) src[lane].wblse[r] = l0;
+    if (lane + 32 < nact && src[lane + 32].wblse) src[lane + 32].wblse[r] = l1;
+    const int n = g.part_off[i] + r;
+    if (act) store_out(out, out_is_fp32, (size_t)b * osb + (size_t)h * osh + (size_t)n * osn + lane * 4, acc);
+    if (out_lse && lane == 0) out_lse[((size_t)b * g.H + h) * g.N + n] = L;
+  }
+}
+
+// Copy the fresh states (fresh-list positions) into their cache slots.
+// blockIdx.y = slot; the block finds its pair, and if the plan marks it fresh
+// counts the fresh pairs before it (row-major) to find its fresh position.
+__global__ void __launch_bounds__(256)
+cache_update_kernel(DevGeom g, const signed char *__restrict__ plan,
+                    const float *__restrict__ part_O, const float *__restrict__ part_lse,
+                    float *cache_O, float *cache_lse, unsigned char *cache_valid, int D) {
+  const int slot = blockIdx.y;
+  int i = 0;
+  while (i + 1 < g.P && g.row_start[i + 1] <= slot) ++i;
+  int rank = slot - g.row_start[i];
+  unsigned long long m = g.row_mask[i];
+  for (int t = 0; t < rank; ++t) m &= m - 1;
+  const int j = __ffsll((long long)m) - 1;
+  const int pair = i * g.P + j;
+  if (plan[pair] != DITANGO_PLAN_FRESH) return;
+  __shared__ int warp_cnt[8];
+  __shared__ int s_fpos;
+  int cnt = 0;
+  for (int p = threadIdx.x; p < pair; p += blockDim.x) cnt += (plan[p] == DITANGO_PLAN_FRESH);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if ((threadIdx.x & 31) == 0) warp_cnt[threadIdx.x >> 5] = cnt;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int c = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) c += warp_cnt[w];
+    s_fpos = c;
+  }
+  __syncthreads();
+  const int f = s_fpos;
+  const size_t blk = (size_t)g.BH * g.Lmax;
+  const float4 *s = reinterpret_cast<const float4 *>(part_O + (size_t)f * blk * D);
+  float4 *d = reinterpret_cast<float4 *>(cache_O + (size_t)slot * blk * D);
+  const size_t n4 = blk * D / 4;
+  for (size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x; t < n4;
+       t += (size_t)gridDim.x * blockDim.x)
+    d[t] = __ldg(s + t);
+  const float *sl = part_lse + (size_t)f * blk;
+  float *dl = cache_lse + (size_t)slot * blk;
+  for (size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x; t < blk;
+       t += (size_t)gridDim.x * blockDim.x)
+    dl[t] = __ldg(sl + t);
+  if (cache_valid && blockIdx.x == 0 && threadIdx.x == 0) cache_valid[slot] = 1;
+}
+
+}  // namespace merge
+
+cudaError_t launch_merge(const DevGeom &g, const signed char *plan, const float *part_O,
+                         const float *part_lse, float *cache_O, float *cache_lse,
+                         unsigned char *cache_valid, int writeback, void *out, int out_is_fp32,
+                         long long osb, long long osh, long long osn, float *out_lse,
+                         cudaStream_t stream) {
+  dim3 grid((g.Lmax + merge::kRowsPerBlock - 1) / merge::kRowsPerBlock, g.P, g.BH);
+  switch (g.d) {
+#define DITANGO_MERGE(DD)                                                                        \
+  case DD:                                                                                       \
+    merge::merge_kernel<DD><<<grid, merge::kThreads, 0, stream>>>(                               \
+        g, plan, part_O, part_lse, cache_O, cache_lse, cache_valid, writeback, out, out_is_fp32, \
+        osb, osh, osn, out_lse);                                                                 \
+    return cudaGetLastError();
+    DITANGO_MERGE(64)
+    DITANGO_MERGE(96)
+    DITANGO_MERGE(128)
+#undef DITANGO_MERGE
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_cache_update(const DevGeom &g, const signed char *plan, const float *part_O, const float *part_lse, float *cache_O,
+                                float *cache_lse, unsigned char *cache_valid, int num_sms,
+                                cudaStream_t stream) {
+  if (g.n_active == 0) return cudaSuccess;
+  const size_t n4 = (size_t)g.BH * g.Lmax * g.d / 4;
+  int bx = (int)((n4 + 255) / 256);
+  const int cap = (num_sms * 8 + g.n_active - 1) / g.n_active;
+  if (bx > cap) bx = cap < 1 ? 1 : cap;
+  dim3 grid(bx, g.n_active);
+  merge::cache_update_kernel<<<grid, 256, 0, stream>>>(g, plan, part_O, part_lse, cache_O,
+                                                        cache_lse, cache_valid, g.d);
+  return cudaGetLastError();
+}
+
+}  // namespace ditango

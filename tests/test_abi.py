@@ -1,0 +1,90 @@
+"""The C ABI library loads without a GPU, exports every declared entry point,
+and its host-side logic (argument checks, active pairs, slot numbering)
+agrees with the oracle.  No compute call is made here."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import sparse_state_reuse_b200 as dt
+from oracle import masks
+from workloads import configs
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "ditango.h")
+
+
+def declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ditango_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    import ctypes
+    lib = ctypes.CDLL(dt.LIB_PATH)
+    names = declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(dt.EXPORTED)
+
+
+def test_version_and_status_strings():
+    assert dt.ditango_version() >= 10000
+    assert dt.status_string(0) == "ok"
+    assert "timed out" in dt.status_string(4)
+
+
+@pytest.mark.parametrize("w", configs.ALL, ids=lambda w: w.name)
+def test_active_pairs_and_slots_match_oracle(w):
+    g = dt.Geometry(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask())
+    A = masks.pair_mask(w.part_off(), w.frame_off(), w.frame_mask())
+    assert dt.ditango_check_geom(g) == 0
+    assert dt.ditango_num_active(g) == int(A.sum())
+    assert dt.ditango_state_rows(g) == w.Lp
+    assert (np.array(dt.ditango_slot_table(g)) == masks.slot_table(A)).all()
+
+
+def test_ragged_partitions_within_frames():
+    po = [0, 100, 130, 300, 555, 1000]
+    fo = [0, 300, 1000]
+    fm = [[1, 0], [1, 1]]
+    g = dt.Geometry(2, 3, 1000, 64, po, fo, fm)
+    A = masks.pair_mask(po, fo, fm)
+    assert dt.ditango_num_active(g) == int(A.sum())
+    assert (np.array(dt.ditango_slot_table(g)) == masks.slot_table(A)).all()
+    assert dt.ditango_state_rows(g) == 445
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(part_off=[0, 10, 10, 64]), 1),          # empty partition
+    (dict(part_off=[0, 32, 63]), 1),              # does not end at N
+    (dict(d=80), 2),                              # head dim without a kernel
+    (dict(part_off=list(range(0, 65 * 2, 2))[:66] + [130]), 2),  # P > 64
+    (dict(frame_off=[0, 40, 64], frame_mask=[[1, 1], [1, 1]]), 2),  # partition straddles frames
+    (dict(B=0), 1),
+])
+def test_geometry_validation(kw, status):
+    args = dict(B=1, H=2, N=64, d=64, part_off=[0, 32, 64], frame_off=None, frame_mask=None)
+    args.update(kw)
+    if args["part_off"][-1] != args["N"] and status == 2 and len(args["part_off"]) > 65:
+        args["N"] = args["part_off"][-1]
+    g = dt.Geometry(**args)
+    assert dt.ditango_check_geom(g) == status
+
+
+def test_calls_reject_bad_arguments_before_launching():
+    g = dt.Geometry(1, 2, 64, 64, [0, 32, 64])
+    with pytest.raises(dt.DitangoError) as e:
+        dt.ditango_plan(g, None, None, 1, 0.5, 0, None, None, None, stream=0)
+    assert e.value.status == 1
+    with pytest.raises(dt.DitangoError):
+        dt.ditango_plan(g, 16, None, 1, 1.5, 0, 16, 16, 16, None, 16, 10**6, stream=0)  # budget > 1
+    with pytest.raises(dt.DitangoError):
+        dt.ditango_attn_partial(g, 16, 16, 8, 16, 16, 0.0, 16, 16, stream=0)  # misaligned V
+    with pytest.raises(dt.DitangoError):
+        dt.ditango_merge(g, 16, None, None, None, None, None, 0, 16, 1, stream=0)  # no sources
+    with pytest.raises(dt.DitangoError):
+        dt.ditango_selftest_bounded_wait(0, 16, stream=0)
+    assert dt.ditango_plan_workspace_size(g) > 0

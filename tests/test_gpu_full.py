@@ -1,0 +1,120 @@
+"""Full-size workloads on the GPU, in the launch configuration the benchmark
+times, checked against the oracle on sampled rows (head/tail rows of the
+first, a middle and the last partition, including ragged tile tails), plus
+the plan kernel at full size on a seeded synthetic cache."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import sparse_state_reuse_b200 as dt
+from oracle import masks as OM
+from oracle.plan import PLAN_FRESH, PLAN_REUSE, mass_scores, select, budget_target
+from workloads import configs, inputs
+
+import gpu_common as G
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+
+def sample_rows(w, i, n=24):
+    lo, hi = w.part_off()[i], w.part_off()[i + 1]
+    L = hi - lo
+    picks = list(range(0, min(n, L))) + list(range(max(L - n, 0), L))
+    mid = L // 2
+    picks += list(range(mid - 4, mid + 4)) + [min(127, L - 1), min(128, L - 1), min(255, L - 1), min(256, L - 1)]
+    return lo + np.unique(np.clip(picks, 0, L - 1))
+
+
+def run_workload(w, out_dtype=torch.float32):
+    Q, K, V = G.upload(w)
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask())
+    if w.reuses:
+        Kp, Vp = G.upload_prev(w)
+        pa.plan_step(anchor=True)
+        pa.partial(Q, Kp, Vp)
+        del Kp, Vp
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=out_dtype, device="cuda")
+    out_lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
+    pa.step(Q, K, V, out, out_lse, band_k=w.band_k, budget=w.budget, anchor=w.anchor)
+    torch.cuda.synchronize()
+    assert pa.status.item() == 0
+    return pa, out, out_lse
+
+
+@pytest.mark.parametrize("w", [configs.FRAME_TILE, configs.DITANGO_REUSE, configs.LONG_VIDEO,
+                               configs.DENSE], ids=lambda w: w.name)
+def test_full_size_sampled_rows(w):
+    pa, out, out_lse = run_workload(w)
+    plan = pa.plan.cpu().numpy().reshape(w.P, w.P)
+    G.check_plan_valid(w, plan)
+    counts = pa.counts.cpu().numpy()
+    assert counts[0] == int((plan == PLAN_FRESH).sum())
+    bhs = sorted({0, w.BH - 1, w.BH // 2})
+    parts = sorted({0, w.P // 2, w.P - 1})
+    for bh in bhs:
+        b, h = divmod(bh, w.H)
+        for i in parts:
+            rows = sample_rows(w, i)
+            Oo, lo, _ = G.oracle_rows(w, plan, b, h, i, rows)
+            rt = torch.as_tensor(rows, device="cuda")
+            G.assert_close(out[b, h].index_select(0, rt).cpu().numpy(), Oo, f"{w.name} out bh{bh} p{i}")
+            G.assert_close(out_lse[b, h].index_select(0, rt).cpu().numpy(), lo, f"{w.name} lse bh{bh} p{i}")
+    if w.anchor and w.F == 0:
+        # all fresh, unmasked: the merged output is unpartitioned attention
+        from oracle.attention import dense_attention
+        q, k, v, _, _ = G.slabs(w, 0, 0, with_prev=False)
+        rows = sample_rows(w, w.P - 1)
+        Od, ld = dense_attention(q[rows], k, v)
+        G.assert_close(out[0, 0].index_select(0, torch.as_tensor(rows, device="cuda")).cpu().numpy(), Od,
+                       "dense equality")
+
+
+@pytest.mark.parametrize("w,invalid", [(configs.DITANGO_REUSE, ()), (configs.LONG_VIDEO, ()),
+                                       (configs.DITANGO_REUSE, (5, 77, 300))],
+                         ids=["reuse_p32", "long_video", "reuse_p32_invalid_slots"])
+def test_plan_full_size_synthetic_cache(w, invalid):
+    g = dt.Geometry(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask())
+    A = OM.pair_mask(w.part_off(), w.frame_off(), w.frame_mask())
+    pairs = OM.slot_pairs(A)
+    lse = inputs.synthetic_cache_lse(w, len(pairs), pairs, seed=w.seed + 500)
+    valid = np.ones(len(pairs), dtype=np.uint8)
+    valid[list(invalid)] = 0
+    lse_d = torch.from_numpy(lse).cuda()
+    valid_d = torch.from_numpy(valid).cuda()
+    plan = torch.zeros(w.P * w.P, dtype=torch.int8, device="cuda")
+    fresh = torch.zeros(len(pairs), dtype=torch.int32, device="cuda")
+    counts = torch.zeros(2, dtype=torch.int32, device="cuda")
+    score = torch.zeros(w.P * w.P, dtype=torch.float32, device="cuda")
+    nws = dt.ditango_plan_workspace_size(g)
+    ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+    dt.ditango_plan(g, lse_d, valid_d, w.band_k, w.budget, 0, plan, fresh, counts, score, ws, nws)
+    torch.cuda.synchronize()
+    w_o = mass_scores(lse, A, w.part_off(), valid=valid.astype(bool))
+    valid_pp = np.zeros((w.P, w.P), dtype=bool)
+    valid_pp[A] = valid.astype(bool)
+    valid_pp[~A] = True
+    plan_o, fl_o = select(w_o, A, w.band_k, w.budget, valid=valid_pp)
+    got_w = score.cpu().numpy().reshape(w.P, w.P)
+    np.testing.assert_allclose(got_w, w_o, rtol=1e-5, atol=1e-9)
+    got = plan.cpu().numpy().reshape(w.P, w.P)
+    # ties within fp32 resolution may legitimately go either way: locate them
+    cand = A & (plan_o != 0)
+    diff = got != plan_o
+    if diff.any():
+        sel = (plan_o == PLAN_FRESH) & cand
+        ii, jj = np.indices((w.P, w.P))
+        band = A & (np.abs(ii - jj) <= w.band_k)
+        extra = sel & ~band & valid_pp
+        cut = w_o[extra].min()
+        for i, j in zip(*np.nonzero(diff)):
+            assert abs(w_o[i, j] - cut) <= 1e-5 * cut, (i, j, w_o[i, j], cut)
+    else:
+        assert (fresh.cpu().numpy()[:counts[0].item()] == fl_o).all()
+    for s in invalid:
+        i, j = pairs[s]
+        assert got[i, j] == PLAN_FRESH
+    assert counts.cpu().numpy()[0] == int((got == PLAN_FRESH).sum())

@@ -1,0 +1,226 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small cases are compared element by element (every row of every pair,
+ragged partitions and tails included); the full-size workloads are run in
+the launch configuration the benchmark times and compared on sampled rows.
+Plans are compared exactly; floating point against fp64 within max-abs 2e-2
+and mean-abs 2e-3.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import sparse_state_reuse_b200 as dt
+from sparse_state_reuse_b200 import _abi
+from oracle import attention as OA
+from oracle import masks as OM
+from oracle.plan import PLAN_FRESH, PLAN_REUSE, mass_scores, select
+from oracle import step as OS
+from workloads import configs, inputs
+
+import gpu_common as G
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+
+def geom_of(w, part_off=None):
+    return dt.Geometry(w.B, w.H, w.N, w.d, part_off or w.part_off(), w.frame_off(), w.frame_mask())
+
+
+def all_pairs_partial(geom, Q, K, V, n, Lmax, d, BH):
+    P = geom.P
+    plan = torch.zeros(P * P, dtype=torch.int8, device="cuda")
+    fresh = torch.full((max(n, 1),), -1, dtype=torch.int32, device="cuda")
+    counts = torch.zeros(2, dtype=torch.int32, device="cuda")
+    dt.ditango_plan(geom, None, None, 0, 1.0, True, plan, fresh, counts)
+    O = torch.full((n, BH, Lmax, d), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.full((n, BH, Lmax), float("nan"), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dt.ditango_attn_partial(geom, Q, K, V, fresh, counts, 0.0, O, lse, 0, None, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    return plan.cpu().numpy(), fresh.cpu().numpy(), counts.cpu().numpy(), O.cpu().numpy(), lse.cpu().numpy()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dt.ditango_selftest_bounded_wait(2_000_000, st)
+    torch.cuda.synchronize()
+    assert st.item() == _abi.ERR_TIMEOUT
+    x = torch.arange(8, device="cuda", dtype=torch.float32)
+    assert float(x.sum()) == 28.0
+
+
+@pytest.mark.parametrize("d,part_off,frames", [
+    (64, None, None),                                  # the tiny workload's geometry
+    (64, [0, 100, 130, 300, 555, 1000], None),         # ragged: short and multi-tile partitions
+    (96, [0, 100, 130, 300, 555, 1000], None),
+    (128, [0, 100, 130, 300, 555, 1000], None),
+    (96, [0, 130, 300, 555, 1000], ([0, 300, 1000], [[1, 0], [1, 1]])),  # frame mask
+    (128, [0, 257, 512, 640, 1024], None),             # 256-row unit boundaries +-1
+])
+def test_partial_states_every_row(d, part_off, frames):
+    if part_off is None:
+        w = configs.TINY
+        part_off = w.part_off()
+    else:
+        w = configs.scaled(configs.TINY, N=part_off[-1], d=d, B=2, H=3, P=1, seed=77 + d,
+                           name=f"ragged_{d}")
+    fo, fm = (frames if frames else (None, None))
+    geom = dt.Geometry(w.B, w.H, w.N, w.d, part_off, fo, fm)
+    A = OM.pair_mask(part_off, fo, fm)
+    n, Lmax = int(A.sum()), max(np.diff(part_off))
+    Q, K, V = G.upload(w)
+    plan, fresh, counts, O, lse = all_pairs_partial(geom, Q, K, V, n, Lmax, w.d, w.BH)
+    P = len(part_off) - 1
+    assert counts.tolist() == [n, 0]
+    assert (fresh[:n] == np.nonzero(A.ravel())[0]).all()
+    assert (plan.reshape(P, P) == np.where(A, 1, 0)).all()
+    for bh in range(w.BH):
+        b, h = divmod(bh, w.H)
+        q, k, v, _, _ = G.slabs(w, b, h, with_prev=False)
+        for f, p in enumerate(fresh[:n]):
+            i, j = divmod(int(p), P)
+            rows = np.arange(part_off[i], part_off[i + 1])
+            Oo, lo = OS.pair_state(q[rows], rows, k, v, part_off, j, fo, fm)
+            G.assert_close(O[f, bh, :rows.size], Oo, f"O pair {(i, j)} bh {bh}")
+            G.assert_close(lse[f, bh, :rows.size], lo, f"lse pair {(i, j)} bh {bh}")
+
+
+def oracle_cache_lse(w):
+    po = w.part_off()
+    A = OM.pair_mask(po, w.frame_off(), w.frame_mask())
+    per = []
+    for bh in range(w.BH):
+        b, h = divmod(bh, w.H)
+        per.append(OS.cache_lse_for_slab(inputs.slab_f64(w, "q", b, h),
+                                         inputs.slab_f64(w, "k", b, h, prev=True),
+                                         inputs.slab_f64(w, "v", b, h, prev=True), A, po,
+                                         w.frame_off(), w.frame_mask()))
+    return np.stack(per, axis=1), A
+
+
+def build_cache(pa, Q, Kp, Vp):
+    pa.plan_step(anchor=True)
+    pa.partial(Q, Kp, Vp)
+
+
+def test_tiny_reuse_step_plan_and_output():
+    w = configs.TINY
+    Q, K, V = G.upload(w)
+    Kp, Vp = G.upload_prev(w)
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    build_cache(pa, Q, Kp, Vp)
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    out_lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
+    pa.step(Q, K, V, out, out_lse, band_k=w.band_k, budget=w.budget)
+    torch.cuda.synchronize()
+    assert pa.status.item() == 0
+    lse_o, A = oracle_cache_lse(w)
+    w_o = mass_scores(lse_o, A, w.part_off())
+    plan_o, fl_o = select(w_o, A, w.band_k, w.budget)
+    gpu_plan = pa.plan.cpu().numpy().reshape(w.P, w.P)
+    assert (gpu_plan == plan_o).all(), (gpu_plan, plan_o)
+    counts = pa.counts.cpu().numpy()
+    assert counts.tolist() == [12, 4]
+    assert (pa.fresh_list.cpu().numpy()[:12] == fl_o).all()
+    score = pa.score.cpu().numpy().reshape(w.P, w.P)
+    np.testing.assert_allclose(score, w_o, rtol=1e-4, atol=1e-7)
+    o = out.cpu().numpy()
+    ol = out_lse.cpu().numpy()
+    for bh in range(w.BH):
+        b, h = divmod(bh, w.H)
+        for i in range(w.P):
+            rows = np.arange(w.part_off()[i], w.part_off()[i + 1])
+            Oo, lo, _ = G.oracle_rows(w, plan_o, b, h, i, rows)
+            G.assert_close(o[b, h, rows], Oo, f"out bh {bh} part {i}")
+            G.assert_close(ol[b, h, rows], lo, f"out lse bh {bh} part {i}")
+
+
+def test_tiny_compact_partials_merge_writeback_and_cache_update_agree():
+    """Three routes to the same step must give bit-identical states and outputs:
+    in-place partials, compact partials + merge write-back, compact partials +
+    cache update + merge from the cache."""
+    w = configs.TINY
+    Q, K, V = G.upload(w)
+    Kp, Vp = G.upload_prev(w)
+    ref = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    build_cache(ref, Q, Kp, Vp)
+    cache0_O, cache0_l = ref.state_O.clone(), ref.state_lse.clone()
+    out_ref = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    ref.step(Q, K, V, out_ref, band_k=w.band_k, budget=w.budget)
+    g = ref.geom
+    nf = 12
+    part_O = torch.empty((nf, w.BH, w.Lp, w.d), dtype=torch.float32, device="cuda")
+    part_l = torch.empty((nf, w.BH, w.Lp), dtype=torch.float32, device="cuda")
+    for route in ("writeback", "cache_update"):
+        cO, cl = cache0_O.clone(), cache0_l.clone()
+        valid = torch.ones(ref.n_slots, dtype=torch.uint8, device="cuda")
+        plan = torch.zeros(w.P * w.P, dtype=torch.int8, device="cuda")
+        fresh = torch.zeros(ref.n_slots, dtype=torch.int32, device="cuda")
+        counts = torch.zeros(2, dtype=torch.int32, device="cuda")
+        ws = torch.empty(ref.ws_bytes, dtype=torch.uint8, device="cuda")
+        dt.ditango_plan(g, cl, valid, w.band_k, w.budget, 0, plan, fresh, counts, None, ws, ref.ws_bytes)
+        dt.ditango_attn_partial(g, Q, K, V, fresh, counts, 0.0, part_O, part_l, 0, None, None)
+        out = torch.empty_like(out_ref)
+        if route == "writeback":
+            dt.ditango_merge(g, plan, part_O, part_l, cO, cl, valid, 1, out, 1)
+        else:
+            dt.ditango_cache_update(g, plan, part_O, part_l, cO, cl, valid)
+            dt.ditango_merge(g, plan, None, None, cO, cl, valid, 0, out, 1)
+        torch.cuda.synchronize()
+        assert torch.equal(plan, ref.plan)
+        assert torch.equal(out, out_ref), route
+        L = w.Lp
+        assert torch.equal(cO[:, :, :L], ref.state_O[:, :, :L]), route
+        assert torch.equal(cl[:, :, :L], ref.state_lse[:, :, :L]), route
+
+
+def test_zero_drift_reuse_is_bitwise_fresh():
+    w = configs.TINY
+    Q, K, V = G.upload(w)
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    build_cache(pa, Q, K, V)                 # cache from the current K/V
+    out_r = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    pa.step(Q, K, V, out_r, band_k=w.band_k, budget=w.budget)
+    assert (pa.plan.cpu().numpy() == PLAN_REUSE).sum() == 4
+    out_f = torch.empty_like(out_r)
+    pa.step(Q, K, V, out_f, anchor=True)
+    torch.cuda.synchronize()
+    assert torch.equal(out_r, out_f)
+
+
+def test_bf16_output_and_strided_output():
+    w = configs.TINY
+    Q, K, V = G.upload(w)
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    o32 = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    pa.step(Q, K, V, o32, anchor=True)
+    o16 = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device="cuda")
+    pa.merge(o16)
+    obnhd = torch.empty((w.B, w.N, w.H, w.d), dtype=torch.float32, device="cuda")
+    pa.merge(obnhd.permute(0, 2, 1, 3))
+    torch.cuda.synchronize()
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+    assert torch.equal(obnhd.permute(0, 2, 1, 3), o32)
+
+
+def test_strided_qkv_inputs():
+    """Q/K/V as views of one [B, N, 3, H, d] tensor (head-interleaved layout)."""
+    w = configs.TINY
+    Q, K, V = G.upload(w)
+    qkv = torch.empty((w.B, w.N, 3, w.H, w.d), dtype=torch.bfloat16, device="cuda")
+    for t, x in enumerate((Q, K, V)):
+        qkv[:, :, t] = x.permute(0, 2, 1, 3)
+    Qs, Ks, Vs = (qkv[:, :, t].permute(0, 2, 1, 3) for t in range(3))
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    o1 = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    pa.step(Q, K, V, o1, anchor=True)
+    o2 = torch.empty_like(o1)
+    pa.step(Qs, Ks, Vs, o2, anchor=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)

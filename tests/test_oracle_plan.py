@@ -125,6 +125,10 @@ def test_mass_closed_forms():
     lse3 = lse.copy()
     lse3[masks.slot_table(A)[2, 0]] += math.log(7.0)  # 7x the mass of each other pair
     np.testing.assert_allclose(mass_scores(lse3, A, po)[2, 0], 0.7, atol=1e-12)
+    valid = np.ones(P * P, dtype=bool)
+    valid[masks.slot_table(A)[1, 3]] = False        # a never-written slot: no mass
+    w4 = mass_scores(lse, A, po, valid=valid)
+    np.testing.assert_allclose(w4, w, atol=1e-15)
 
 
 def _brute_force_plan(w, A, band_k, budget):
