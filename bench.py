@@ -91,6 +91,23 @@ def recorded_traffic(kernel_file, workload):
     return e.get("dram_bytes_per_launch")
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(x, device, dist=None):
+    """Max of a per-rank float over all ranks (the slowest replica sets the
+    time); identity on one process."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world, flops_per_replica, ms_per_step):
+    """Whole-job effective TFLOP/s: every replica does the same step."""
+    return world * flops_per_replica / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -216,10 +233,8 @@ def run_ours(args, w, rank, world, local_rank):
     ms = e_start.elapsed_time(e_end)
     part_ms = float(np.mean([e_part0[t].elapsed_time(e_part1[t]) for t in range(n_ev)]))
     merge_ms = float(np.mean([e_part1[t].elapsed_time(e_merge1[t]) for t in range(n_ev)]))
+    ms = max_over_ranks(ms, dev, dist)
     if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
         dist.barrier()
     status = int(pa.status.item())
     if status != 0:
@@ -251,10 +266,7 @@ def run_ours(args, w, rank, world, local_rank):
     b.record(stream)
     stream.synchronize()
     e2e_ms = a.elapsed_time(b) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev, dist)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
     d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
 
@@ -266,7 +278,7 @@ def run_ours(args, w, rank, world, local_rank):
     traffic = recorded_traffic("attn_partial.cu", w.name)
     res = {
         "metric": "effective attention TFLOP/s (fresh blocks only) at 1 B200; tokens/s",
-        "value": round(world * flops / (ms_step * 1e-3) / 1e12, 3),
+        "value": round(aggregate_tflops(world, flops, ms_step), 3),
         "unit": "TFLOP/s",
         "tokens_per_s": round(world * w.B * w.N / (ms_step * 1e-3), 1),
         "n_gpus": world,
@@ -294,7 +306,7 @@ def run_ours(args, w, rank, world, local_rank):
                            "kernel_ms": round(merge_ms, 4),
                            "algorithmic_bytes_per_launch": mbytes,
                            "traffic": recorded_traffic("merge.cu", w.name)},
-        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        "e2e": {"value": round(aggregate_tflops(world, flops, e2e_ms), 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
