@@ -189,6 +189,28 @@ ditango_status ditango_cache_update(const ditango_geom *g, const int8_t *plan,
                                     float *cache_O, float *cache_lse,
                                     uint8_t *cache_valid, ditango_stream stream);
 
+/* Allocation-free variant of ditango_plan (no counterpart in the papers: it
+ * exists for callers, not for the method).  For callers that cannot allocate
+ * device memory -- code running inside an arena it does not own, a serving
+ * process whose allocator is frozen after start-up, or a host that must not
+ * call cudaMalloc between steps -- and so cannot provide ditango_plan's
+ * workspace.  Same arguments, meaning and results as ditango_plan without
+ * workspace/workspace_bytes; the scratch is a fixed 4 MiB device array inside
+ * the library (held by every GPU that loads the library until the process
+ * exits).  Returns DITANGO_ERR_UNSUPPORTED when ditango_plan_workspace_size
+ * exceeds 4 MiB (anchor plans need no scratch and are never rejected).
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * The first call on a device looks up the array's device address (one
+ * cudaGetSymbolAddress with that device current); make that first call
+ * before any stream capture.  Every call shares the one array per device and
+ * overwrites all of the scratch it reads, so nothing carries over between
+ * calls; but calls that overlap on the GPU (other streams, concurrent graph
+ * branches) race on it -- order them. */
+ditango_status ditango_plan_noalloc(const ditango_geom *g, const float *cache_lse,
+                                    const uint8_t *cache_valid, int32_t band_k, double budget,
+                                    int32_t anchor, int8_t *plan, int32_t *fresh_list,
+                                    int32_t *counts, float *score_out, ditango_stream stream);
+
 /* Time limit, in nanoseconds, of every wait inside the kernels (default
  * 1e9).  Process-wide; read at each launch. */
 void ditango_set_wait_limit_ns(int64_t ns);

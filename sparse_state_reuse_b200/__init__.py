@@ -20,7 +20,7 @@ from ._abi import (  # noqa: F401
     ditango_version, ditango_check_geom, ditango_num_active, ditango_state_rows,
     ditango_slot_table, ditango_plan_workspace_size, ditango_plan, ditango_attn_partial,
     ditango_merge, ditango_cache_update, ditango_set_wait_limit_ns,
-    ditango_selftest_bounded_wait, status_string,
+    ditango_selftest_bounded_wait, ditango_plan_noalloc, status_string,
 )
 
 

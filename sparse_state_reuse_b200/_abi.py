@@ -62,6 +62,8 @@ _SIGS = {
                                        _P, _P]),
     "ditango_merge": (C.c_int, [_G, _P, _P, _P, _P, _P, _P, C.c_int32, _P, C.c_int32, _P, _P, _P]),
     "ditango_cache_update": (C.c_int, [_G, _P, _P, _P, _P, _P, _P, _P]),
+    "ditango_plan_noalloc": (C.c_int, [_G, _P, _P, C.c_int32, C.c_double, C.c_int32, _P, _P, _P,
+                                       _P, _P]),
     "ditango_set_wait_limit_ns": (None, [C.c_int64]),
     "ditango_selftest_bounded_wait": (C.c_int, [C.c_int64, _P, _P]),
 }
@@ -207,3 +209,11 @@ def ditango_set_wait_limit_ns(ns: int) -> None:
 def ditango_selftest_bounded_wait(limit_ns, dev_status, stream=None):
     _check("ditango_selftest_bounded_wait", _lib.ditango_selftest_bounded_wait(
         int(limit_ns), _ptr(dev_status), _stream(stream)))
+
+
+def ditango_plan_noalloc(geom, cache_lse, cache_valid, band_k, budget, anchor, plan, fresh_list,
+                         counts, score_out=None, stream=None):
+    """ditango_plan with the library's own fixed scratch (allocates nothing)."""
+    _check("ditango_plan_noalloc", _lib.ditango_plan_noalloc(
+        geom.ref, _ptr(cache_lse), _ptr(cache_valid), int(band_k), float(budget), int(bool(anchor)),
+        _ptr(plan), _ptr(fresh_list), _ptr(counts), _ptr(score_out), _stream(stream)))

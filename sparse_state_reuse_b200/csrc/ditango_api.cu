@@ -307,3 +307,64 @@ ditango_status ditango_selftest_bounded_wait(int64_t limit_ns, int32_t *dev_stat
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free plan.
+//
+// Some callers cannot allocate device memory at all: code that runs inside a
+// memory arena owned by someone else, a serving process whose allocator is
+// frozen after start-up, or a host that must never call cudaMalloc between
+// denoising steps.  They still pass their own inputs and outputs, but the
+// plan's scratch (the per-chunk mass sums) lives here, in a fixed device
+// array of this library of kNoAllocPlanScratchBytes.  Every GPU that loads
+// the library holds that array until the process exits.
+namespace {
+constexpr size_t kNoAllocPlanScratchBytes = size_t(4) << 20;  // 4 MiB
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_scratch[kNoAllocMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_plan_scratch[kNoAllocPlanScratchBytes];
+
+extern "C" ditango_status ditango_plan_noalloc(const ditango_geom *g, const float *cache_lse,
+                                               const uint8_t *cache_valid, int32_t band_k,
+                                               double budget, int32_t anchor, int8_t *plan,
+                                               int32_t *fresh_list, int32_t *counts,
+                                               float *score_out, ditango_stream stream) {
+  DevGeom dg;
+  ditango_status st = make_geom(g, &dg);
+  if (st != DITANGO_OK) return st;
+  if (!plan || !fresh_list || !counts) return DITANGO_ERR_INVALID;
+  if (!anchor) {
+    if (!cache_lse || band_k < 0 || !(budget >= 0.0 && budget <= 1.0)) return DITANGO_ERR_INVALID;
+    if (plan_workspace_bytes(dg) > kNoAllocPlanScratchBytes) return DITANGO_ERR_UNSUPPORTED;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaErrorInvalidDevice);
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return DITANGO_ERR_UNSUPPORTED;
+  void *scratch = nullptr;
+  {
+    // once per device, with that device current: the host-side name of the
+    // array is not a device address; ask the runtime for the real one.
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_scratch[dev]) {
+      void *p = nullptr;
+      cudaError_t e = cudaGetSymbolAddress(&p, g_plan_scratch);
+      if (e != cudaSuccess || p == nullptr) return cuda_status(e == cudaSuccess ? cudaErrorUnknown : e);
+      g_noalloc_scratch[dev] = p;
+    }
+    scratch = g_noalloc_scratch[dev];
+  }
+  int n_band = 0;
+  for (int i = 0; i < dg.P; ++i)
+    for (int j = 0; j < dg.P; ++j)
+      if (((dg.row_mask[i] >> j) & 1ull) && std::abs(i - j) <= band_k) ++n_band;
+  int target = (int)std::floor(budget * (double)dg.n_active + 1e-9);
+  if (target < n_band) target = n_band;
+  if (target > dg.n_active) target = dg.n_active;
+  dg.n_band = n_band;
+  return cuda_status(launch_plan(dg, cache_lse, cache_valid, band_k, target, anchor ? 1 : 0,
+                                 reinterpret_cast<signed char *>(plan), fresh_list, counts,
+                                 score_out, scratch, static_cast<cudaStream_t>(stream)));
+}
