@@ -7,11 +7,17 @@
 // the state O = softmax(Q K^T * scale) V (normalised) and
 // lse = log sum exp(Q K^T * scale), by an online softmax over 128-key tiles.
 //
-// CTA organisation (one CTA per SM, persistent over work units):
+// CTA organisation (one CTA per SM, persistent over work units, 384 threads):
 //   warps 0-3  softmax warpgroup 0: rows   0..127 of the unit (Q tile 0)
 //   warps 4-7  softmax warpgroup 1: rows 128..255 of the unit (Q tile 1)
 //   warp  8    TMA producer (Q tiles, then a 2-stage K ring and V ring)
 //   warp  9    TMEM owner and MMA issuer (one thread)
+//   warps 10-11 idle
+// Registers are rebalanced with setmaxnreg: the softmax warpgroups, which
+// hold a whole 128-column S row per thread, get kSoftmaxRegs; warpgroup 2
+// drops to kControlRegs.  2 * 128 * 216 + 128 * 72 = 384 * 168, the
+// registers the CTA is launched with; the launcher refuses to launch a build
+// whose register count differs (an unbalanced split would block forever).
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [384,384+d).
 // The bf16 probabilities P_k overwrite the first 64 columns of S_k and feed
 // the P V product straight from TMEM.  The two Q tiles ping-pong: while one
@@ -26,7 +32,12 @@ namespace attn {
 
 constexpr int BM = 128;            // query rows per tile
 constexpr int BN = 128;            // keys per tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;   // 65536 / 384, rounded down to a multiple of 8
+constexpr int kSoftmaxRegs = 216;
+constexpr int kControlRegs = 72;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kThreads * kLaunchRegs,
+              "register split must equal the launch budget");
 constexpr int kStages = 2;         // K ring and V ring depth
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -38,7 +49,9 @@ struct Cfg {
   static constexpr int OFF_Q = 0;                    // Q0, Q1
   static constexpr int OFF_K = 2 * TILE;
   static constexpr int OFF_V = OFF_K + kStages * TILE;
-  static constexpr int OFF_BAR = OFF_V + kStages * TILE;
+  static constexpr int OFF_EPI = OFF_V + kStages * TILE;     // 8 warps x 32 rows x 128 B
+  static constexpr int EPI_BYTES = 8 * 32 * 128;
+  static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
   static constexpr int BAR_BYTES = 256;
   static constexpr int USED = OFF_BAR + BAR_BYTES;
   // >= 116 KB keeps one CTA per SM (each CTA allocates all 512 TMEM columns).
@@ -58,44 +71,121 @@ struct Params {
   long long wait_limit_ns;
 };
 
-struct Unit {
+// A work item: up to 256 query rows of partition i for one (b, h).  The item
+// visits every fresh pair (i, j) of row i in fresh-list order, so its Q tiles
+// are loaded once and reused for all of them.
+struct Item {
   bool live;
-  int f, i, j, bh, b, h;
-  int q0;          // first query token of the unit
+  int i, bh, b, h;
+  int q0;          // first query token of the item
   int rloc0;       // row of q0 inside partition i
   int rows0, rows1;
-  int k0, Lk, T;   // first key token, keys, key tiles
+  int f0, f1;      // fresh-list range of row i
 };
 
-__device__ __forceinline__ Unit decode(const Params &p, int u, int nqt2) {
-  Unit w;
+struct PairRange {
+  int f, j;
+  int k0, Lk, T;   // first key token, keys, key tiles of partition j
+};
+
+__device__ __forceinline__ Item decode_item(const Params &p, const int *row_fresh, int it, int nqt2) {
+  Item w;
   const DevGeom &g = p.g;
-  int qt2 = u % nqt2;
-  int rest = u / nqt2;
+  const int qt2 = it % nqt2;
+  const int rest = it / nqt2;
   w.bh = rest % g.BH;
-  w.f = rest / g.BH;
-  int pair = __ldg(p.fresh_list + w.f);
-  w.i = pair / g.P;
-  w.j = pair - w.i * g.P;
+  w.i = rest / g.BH;
   w.b = w.bh / g.H;
   w.h = w.bh - w.b * g.H;
   w.rloc0 = qt2 * 2 * BM;
   w.q0 = g.part_off[w.i] + w.rloc0;
-  int rem = g.part_off[w.i + 1] - w.q0;
+  const int rem = g.part_off[w.i + 1] - w.q0;
   w.rows0 = rem < BM ? rem : BM;
-  int r1 = rem - BM;
+  const int r1 = rem - BM;
   w.rows1 = r1 <= 0 ? 0 : (r1 < BM ? r1 : BM);
-  w.k0 = g.part_off[w.j];
-  w.Lk = g.part_off[w.j + 1] - w.k0;
-  w.T = (w.Lk + BN - 1) / BN;
-  w.live = (w.rows0 > 0) && (w.Lk > 0);
+  w.f0 = row_fresh[w.i];
+  w.f1 = row_fresh[w.i + 1];
+  w.live = (w.rows0 > 0) && (w.f1 > w.f0);
   return w;
+}
+
+__device__ __forceinline__ PairRange pair_at(const Params &p, int f) {
+  PairRange q;
+  const int pair = __ldg(p.fresh_list + f);
+  q.f = f;
+  q.j = pair % p.g.P;
+  q.k0 = p.g.part_off[q.j];
+  q.Lk = p.g.part_off[q.j + 1] - q.k0;
+  q.T = (q.Lk + BN - 1) / BN;
+  return q;
 }
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA/ALU pipes, to take part of the exponentials off the
+// special-function unit.  Range reduction to the nearest integer with the
+// 1.5 * 2^23 rounding constant (x = n + f, f in [-1/2, 1/2]); 2^f by a
+// degree-3 polynomial fitted here for minimum relative error on [-1/2, 1/2]
+// (max relative error 1.0e-4, far below the bf16 rounding P gets next);
+// 2^n by adding n to the exponent field.  Inputs below -126 give ~0.
+constexpr float kExpC1 = 0.6932829022f;
+constexpr float kExpC2 = 0.2422106713f;
+constexpr float kExpC3 = 0.0550087579f;
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float kRound = 12582912.0f;  // 1.5 * 2^23
+  const float t = x + kRound;        // t = 1.5 * 2^23 + round(x), exactly
+  const float n = t - kRound;
+  const float f = x - n;
+  const float p = fmaf(fmaf(fmaf(kExpC3, f, kExpC2), f, kExpC1), f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Of every 16 probabilities of a row, this many use exp2_poly, the rest the
+// ex2 instruction.  Measured on B200: moving exponentials off the special
+// function unit does not pay at the current pipeline depth, so 0 by default.
+#ifndef DITANGO_EMU_D64
+#define DITANGO_EMU_D64 0
+#endif
+#ifndef DITANGO_EMU_D96
+#define DITANGO_EMU_D96 0
+#endif
+#ifndef DITANGO_EMU_D128
+#define DITANGO_EMU_D128 0
+#endif
+template <int D>
+__host__ __device__ constexpr int emu_per16() {
+  return D == 64 ? DITANGO_EMU_D64 : (D == 96 ? DITANGO_EMU_D96 : DITANGO_EMU_D128);
+}
+
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic: one instruction, two lanes).
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unf2(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -129,6 +219,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   auto o_full = [&](int k) { return bar + 112 + 8 * k; };
   auto o_empty = [&](int k) { return bar + 128 + 8 * k; };
   const uint32_t drain = bar + 144;
+
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + 192);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_BAR + 200);
 
@@ -137,7 +228,19 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   WaitCtl ctl{abort_flag, p.dev_status, p.wait_limit_ns};
 
   const int nqt2 = (p.g.Lmax + 2 * BM - 1) / (2 * BM);
-  const int n_units = __ldg(p.counts) * p.g.BH * nqt2;
+  const int n_items = p.g.P * p.g.BH * nqt2;
+  // fresh-list range of every query partition (the list is row-major)
+  __shared__ int row_fresh[kMaxP + 1];
+  if (threadIdx.x <= p.g.P) row_fresh[threadIdx.x] = 0;
+  __syncthreads();
+  {
+    const int n_fresh = __ldg(p.counts);
+    for (int f = threadIdx.x; f < n_fresh; f += blockDim.x)
+      atomicAdd(&row_fresh[__ldg(p.fresh_list + f) / p.g.P + 1], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int i = 1; i <= p.g.P; ++i) row_fresh[i] += row_fresh[i - 1];
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -150,11 +253,12 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(s_full(k), 1);
-      mbar_init(p_full(k), 128);
+      mbar_init(p_full(k), 4);    // one arrival per softmax warp
       mbar_init(o_full(k), 1);
-      mbar_init(o_empty(k), 128);
+      mbar_init(o_empty(k), 4);
     }
     mbar_init(drain, 1);
+
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -172,16 +276,19 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp >= 8) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
+   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t kc = 0, vc = 0, uc = 0;
       // last armed phase per full barrier (for a clean stop on abort)
-      int q_armed = -1, k_armed[kStages], v_armed[kStages];
-      for (int s = 0; s < kStages; ++s) k_armed[s] = v_armed[s] = -1;
+      // bit 2s: stage s armed at least once; bit 2s+1: parity of its last arming
+      int q_armed = -1;
+      uint32_t k_armed = 0, v_armed = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        Unit w = decode(p, u, nqt2);
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const Item w = decode_item(p, row_fresh, it, nqt2);
         if (!w.live) continue;
         if (!(ok = wait_bounded(q_empty, (uc & 1) ^ 1, ctl))) break;
         const uint32_t qbytes = C::TILE * (w.rows1 > 0 ? 2 : 1);
@@ -192,22 +299,25 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (w.rows1 > 0)
           for (int c = 0; c < C::NCH; ++c)
             tma_load_4d(sQ + C::TILE + c * C::CHUNK, &tmQ, q_full, c * 64, w.q0 + BM, w.h, w.b);
-        for (int t = 0; t < w.T && ok; ++t) {
-          const int row = w.k0 + t * BN;
-          int s = kc % kStages;
-          if (!(ok = wait_bounded(k_empty(s), ((kc / kStages) & 1) ^ 1, ctl))) break;
-          mbar_arrive_expect_tx(k_full(s), C::TILE);
-          k_armed[s] = (kc / kStages) & 1;
-          for (int c = 0; c < C::NCH; ++c)
-            tma_load_4d(sK + s * C::TILE + c * C::CHUNK, &tmK, k_full(s), c * 64, row, w.h, w.b);
-          ++kc;
-          s = vc % kStages;
-          if (!(ok = wait_bounded(v_empty(s), ((vc / kStages) & 1) ^ 1, ctl))) break;
-          mbar_arrive_expect_tx(v_full(s), C::TILE);
-          v_armed[s] = (vc / kStages) & 1;
-          for (int c = 0; c < C::NCH; ++c)
-            tma_load_4d(sV + s * C::TILE + c * C::CHUNK, &tmV, v_full(s), c * 64, row, w.h, w.b);
-          ++vc;
+        for (int f = w.f0; f < w.f1 && ok; ++f) {
+          const PairRange pr = pair_at(p, f);
+          for (int t = 0; t < pr.T && ok; ++t) {
+            const int row = pr.k0 + t * BN;
+            int s = kc % kStages;
+            if (!(ok = wait_bounded(k_empty(s), ((kc / kStages) & 1) ^ 1, ctl))) break;
+            mbar_arrive_expect_tx(k_full(s), C::TILE);
+            k_armed = (k_armed & ~(3u << (2 * s))) | ((1u | (((kc / kStages) & 1u) << 1)) << (2 * s));
+            for (int c = 0; c < C::NCH; ++c)
+              tma_load_4d(sK + s * C::TILE + c * C::CHUNK, &tmK, k_full(s), c * 64, row, w.h, w.b);
+            ++kc;
+            s = vc % kStages;
+            if (!(ok = wait_bounded(v_empty(s), ((vc / kStages) & 1) ^ 1, ctl))) break;
+            mbar_arrive_expect_tx(v_full(s), C::TILE);
+            v_armed = (v_armed & ~(3u << (2 * s))) | ((1u | (((vc / kStages) & 1u) << 1)) << (2 * s));
+            for (int c = 0; c < C::NCH; ++c)
+              tma_load_4d(sV + s * C::TILE + c * C::CHUNK, &tmV, v_full(s), c * 64, row, w.h, w.b);
+            ++vc;
+          }
         }
         ++uc;
       }
@@ -217,9 +327,10 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         volatile int never = 0;
         drain_ctl.abort_flag = &never;
         if (q_armed >= 0) wait_bounded(q_full, (uint32_t)q_armed, drain_ctl);
+#pragma unroll
         for (int s = 0; s < kStages; ++s) {
-          if (k_armed[s] >= 0) wait_bounded(k_full(s), (uint32_t)k_armed[s], drain_ctl);
-          if (v_armed[s] >= 0) wait_bounded(v_full(s), (uint32_t)v_armed[s], drain_ctl);
+          if ((k_armed >> (2 * s)) & 1u) wait_bounded(k_full(s), (k_armed >> (2 * s + 1)) & 1u, drain_ctl);
+          if ((v_armed >> (2 * s)) & 1u) wait_bounded(v_full(s), (v_armed >> (2 * s + 1)) & 1u, drain_ctl);
         }
       }
     }
@@ -231,86 +342,100 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       uint32_t kc = 0, vc = 0, uc = 0;
       uint32_t pc[2] = {0, 0}, oc[2] = {0, 0};
       bool ok = true;
+      // Descriptors are built once; a k-step only adds a compile-time offset
+      // to the start-address field (all addresses stay below 256 KB, so the
+      // 14-bit field never carries).
+      const uint64_t dQ0 = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dQ1 = smem_desc_sw128(sQ + C::TILE, 16, 1024);
+      const uint64_t dK0 = smem_desc_sw128(sK, 16, 1024);
+      const uint64_t dK1 = smem_desc_sw128(sK + C::TILE, 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(sV, C::CHUNK, 1024);
+      const uint64_t dV1 = smem_desc_sw128(sV + C::TILE, C::CHUNK, 1024);
+      static_assert(kStages == 2, "descriptor selection assumes two stages");
       auto qk = [&](int k, int ks) {
         // S_k = Q_k K^T : K-major A and B, 16 columns of d per instruction
-        const uint32_t qa = sQ + k * C::TILE;
-        const uint32_t kb = sK + ks * C::TILE;
+        const uint64_t a0 = k ? dQ1 : dQ0;
+        const uint64_t b0 = ks ? dK1 : dK0;
+        const uint32_t d_tmem = tmem + k * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + k * 128, smem_desc_sw128(qa + off, 16, 1024),
-                 smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0);
+          const uint64_t off = (uint64_t)(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
+          mma_ss(d_tmem, a0 + off, b0 + off, idesc_qk, kk > 0);
         }
       };
       auto pv = [&](int k, int vs, bool acc) {
         // O_k (+)= P_k V : P from TMEM (K-major), V MN-major (d contiguous)
-        const uint32_t vb = sV + vs * C::TILE;
+        const uint64_t b0 = vs ? dV1 : dV0;
+        const uint32_t d_tmem = tmem + 256 + k * 128;
+        const uint32_t a_tmem = tmem + k * 128;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          mma_ts(tmem + 256 + k * 128, tmem + k * 128 + kk * 8,
-                 smem_desc_sw128(vb + kk * 2048, C::CHUNK, 1024), idesc_pv, (acc || kk > 0));
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(d_tmem, a_tmem + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv, (acc || kk > 0));
       };
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        Unit w = decode(p, u, nqt2);
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const Item w = decode_item(p, row_fresh, it, nqt2);
         if (!w.live) continue;
         const bool has1 = w.rows1 > 0;
         if (!(ok = wait_bounded(q_full, uc & 1, ctl))) break;
-        int ks = kc % kStages;
-        if (!(ok = wait_bounded(k_full(ks), (kc / kStages) & 1, ctl))) break;
-        tc_fence_after();
-        qk(0, ks);
-        tc_commit(s_full(0));
-        if (has1) {
-          qk(1, ks);
-          tc_commit(s_full(1));
-        }
-        tc_commit(k_empty(ks));
-        ++kc;
-        if (w.T == 1) tc_commit(q_empty);
-        for (int t = 0; t < w.T && ok; ++t) {
-          const int vs = vc % kStages;
-          if (!(ok = wait_bounded(v_full(vs), (vc / kStages) & 1, ctl))) break;
-          const bool more = (t + 1 < w.T);
-          // ---- Q tile 0
-          if (!(ok = wait_bounded(p_full(0), pc[0] & 1, ctl))) break;
-          ++pc[0];
-          if (t == 0) {
-            if (!(ok = wait_bounded(o_empty(0), (oc[0] & 1) ^ 1, ctl))) break;
-            ++oc[0];
-          }
+        for (int f = w.f0; f < w.f1 && ok; ++f) {
+          const PairRange pr = pair_at(p, f);
+          const bool last_pair = (f + 1 == w.f1);
+          int ks = kc % kStages;
+          if (!(ok = wait_bounded(k_full(ks), (kc / kStages) & 1, ctl))) break;
           tc_fence_after();
-          pv(0, vs, t > 0);
-          if (!more) tc_commit(o_full(0));
-          int ks2 = kc % kStages;
-          if (more) {
-            if (!(ok = wait_bounded(k_full(ks2), (kc / kStages) & 1, ctl))) break;
-            tc_fence_after();
-            qk(0, ks2);
-            tc_commit(s_full(0));
-          }
-          // ---- Q tile 1
+          qk(0, ks);
+          tc_commit(s_full(0));
           if (has1) {
-            if (!(ok = wait_bounded(p_full(1), pc[1] & 1, ctl))) break;
-            ++pc[1];
+            qk(1, ks);
+            tc_commit(s_full(1));
+          }
+          tc_commit(k_empty(ks));
+          ++kc;
+          if (pr.T == 1 && last_pair) tc_commit(q_empty);
+          for (int t = 0; t < pr.T && ok; ++t) {
+            const int vs = vc % kStages;
+            if (!(ok = wait_bounded(v_full(vs), (vc / kStages) & 1, ctl))) break;
+            const bool more = (t + 1 < pr.T);
+            // ---- Q tile 0
+            if (!(ok = wait_bounded(p_full(0), pc[0] & 1, ctl))) break;
+            ++pc[0];
             if (t == 0) {
-              if (!(ok = wait_bounded(o_empty(1), (oc[1] & 1) ^ 1, ctl))) break;
-              ++oc[1];
+              if (!(ok = wait_bounded(o_empty(0), (oc[0] & 1) ^ 1, ctl))) break;
+              ++oc[0];
             }
             tc_fence_after();
-            pv(1, vs, t > 0);
-            if (!more) tc_commit(o_full(1));
+            pv(0, vs, t > 0);
+            if (!more) tc_commit(o_full(0));
+            const int ks2 = kc % kStages;
             if (more) {
-              qk(1, ks2);
-              tc_commit(s_full(1));
+              if (!(ok = wait_bounded(k_full(ks2), (kc / kStages) & 1, ctl))) break;
+              tc_fence_after();
+              qk(0, ks2);
+              tc_commit(s_full(0));
             }
-          }
-          tc_commit(v_empty(vs));
-          ++vc;
-          if (more) {
-            tc_commit(k_empty(ks2));
-            ++kc;
-            if (t + 2 == w.T) tc_commit(q_empty);
+            // ---- Q tile 1
+            if (has1) {
+              if (!(ok = wait_bounded(p_full(1), pc[1] & 1, ctl))) break;
+              ++pc[1];
+              if (t == 0) {
+                if (!(ok = wait_bounded(o_empty(1), (oc[1] & 1) ^ 1, ctl))) break;
+                ++oc[1];
+              }
+              tc_fence_after();
+              pv(1, vs, t > 0);
+              if (!more) tc_commit(o_full(1));
+              if (more) {
+                qk(1, ks2);
+                tc_commit(s_full(1));
+              }
+            }
+            tc_commit(v_empty(vs));
+            ++vc;
+            if (more) {
+              tc_commit(k_empty(ks2));
+              ++kc;
+              if (t + 2 == pr.T && last_pair) tc_commit(q_empty);
+            }
           }
         }
         ++uc;
@@ -322,8 +447,20 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       drain_ctl.abort_flag = &never;
       wait_bounded(drain, 0, drain_ctl);
     }
+   }
+    // end of the control warpgroup: warp 9 frees TMEM once every warp is done
+    if (warp == 9) {
+      named_bar_sync(1, kThreads);
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    } else {
+      tc_fence_before();
+      named_bar_arrive(1, kThreads);
+    }
+    return;
   } else {
     // ------------------------------------------------------------ softmax
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     const int k = warp >> 2;                 // Q tile of this warpgroup
     const int r = threadIdx.x & 127;         // row within the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -332,37 +469,41 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const float sl2 = p.scale_log2;
     uint32_t sc = 0, ofc = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      Unit w = decode(p, u, nqt2);
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const Item w = decode_item(p, row_fresh, it, nqt2);
       if (!w.live) continue;
       const int rows_k = (k == 0) ? w.rows0 : w.rows1;
       if (rows_k <= 0) continue;
+     for (int f = w.f0; f < w.f1 && ok; ++f) {
+      const PairRange pr = pair_at(p, f);
       float m_used = -INFINITY;   // running maximum used for exponentiation (log2 units)
       float l = 0.f;
-      for (int t = 0; t < w.T; ++t) {
+      for (int t = 0; t < pr.T; ++t) {
         if (!(ok = wait_bounded(s_full(k), sc & 1, ctl))) break;
         ++sc;
         tc_fence_after();
-        float s[BN];
-        {
-          uint32_t v[32];
+        // the whole S row of this thread: eight loads in flight, one wait
+        uint32_t sv[BN];
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-            tmem_ld32(tS + c * 32, v);
-            tc_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(v[e]);
-          }
-        }
-        const int valid = w.Lk - t * BN;
+        for (int c = 0; c < BN / 16; ++c) tmem_ld16p(tS + c * 16, &sv[c * 16]);
+        tc_wait_ld();
+        const int valid = pr.Lk - t * BN;
         if (valid < BN) {
 #pragma unroll
           for (int c = 0; c < BN; ++c)
-            if (c >= valid) s[c] = -INFINITY;
+            if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
         }
-        float mx = s[0];
+        // row maximum: 8 independent chains of 3-input max, then a tree
+        float m8[8];
 #pragma unroll
-        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        for (int q = 0; q < 8; ++q)
+          m8[q] = max3(__uint_as_float(sv[q]), __uint_as_float(sv[q + 8]), __uint_as_float(sv[q + 16]));
+#pragma unroll
+        for (int c = 24; c < BN; c += 16)
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            m8[q] = max3(m8[q], __uint_as_float(sv[c + q]), __uint_as_float(sv[c + q + 8]));
+        const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
         const float mx2 = mx * sl2;
         if (t == 0) {
           m_used = mx2;
@@ -386,63 +527,102 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
           }
         }
+        // P = 2^(s*scale*log2e - m), rounded to bf16 into the first 64 S columns
         const float neg = -m_used;
-        uint32_t pk[32];
+        const uint64_t sl2x2 = f2(sl2, sl2), negx2 = f2(neg, neg);
+        uint64_t lsum0 = 0, lsum1 = 0;   // packed partial row sums (+0.0f bits)
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
+        for (int g8 = 0; g8 < BN / 16; ++g8) {
+          // 16 probabilities -> 8 packed bf16 pairs -> TMEM columns [8*g8, 8*g8+8)
+          uint32_t pk[8];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float a = ex2(fmaf(s[h2 * 64 + 2 * e], sl2, neg));
-            const float b = ex2(fmaf(s[h2 * 64 + 2 * e + 1], sl2, neg));
-            l += a + b;
+          for (int e = 0; e < 8; ++e) {
+            const int c = g8 * 16 + 2 * e;
+            float xa, xb;
+            unf2(fma2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, negx2), xa, xb);
+            const float a = (2 * e < emu_per16<D>()) ? exp2_poly(xa) : ex2(xa);
+            const float b = (2 * e + 1 < emu_per16<D>()) ? exp2_poly(xb) : ex2(xb);
+            if (e & 1) lsum1 = add2(lsum1, f2(a, b)); else lsum0 = add2(lsum0, f2(a, b));
             pk[e] = pack_bf16(a, b);
           }
-          tmem_st32(tS + h2 * 32, pk);
+          tmem_st8(tS + g8 * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+        }
+        {
+          float s0, s1, s2, s3;
+          unf2(lsum0, s0, s1);
+          unf2(lsum1, s2, s3);
+          l += (s0 + s1) + (s2 + s3);
         }
         tc_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full(k));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(k));   // one arrival per warp
       }
       if (!ok) break;
-      // ---- epilogue: normalise and store the state of this row
+      // ---- epilogue: O of this row into registers, release the TMEM
+      // accumulator to the next pair at once, then normalise and store.
       if (!(ok = wait_bounded(o_full(k), ofc & 1, ctl))) break;
       ++ofc;
       tc_fence_after();
-      const int idx = p.out_by_slot ? slot_of(p.g, w.i, w.j) : w.f;
+      // O is read in halves of up to 64 columns (fewer live registers); the
+      // accumulator is released to the next pair once the last half is in
+      // registers.  The 32 rows of this warp are one contiguous block of the
+      // state buffer: each half is transposed through this warp's 4 KB of
+      // shared memory, 32 columns at a time, so that every store writes whole
+      // 128-byte row segments (XOR swizzle: both phases free of bank
+      // conflicts).
+      constexpr int HALF = (D > 64) ? 64 : D;
+      const int idx = p.out_by_slot ? slot_of(p.g, w.i, pr.j) : pr.f;
       const int rloc = w.rloc0 + k * BM + r;
       const size_t row_off = ((size_t)idx * p.g.BH + w.bh) * (size_t)p.g.Lmax + rloc;
-      const bool row_ok = r < rows_k;
       const float inv_l = 1.f / l;
-      float4 *dst = reinterpret_cast<float4 *>(p.out_O + row_off * D);
-      uint32_t v[32];
+      float4 *epi = reinterpret_cast<float4 *>(smem + C::OFF_EPI + (warp & 7) * 4096);
+      const int row_valid = rows_k - (r & ~31);         // valid rows of this warp
+      float *blk = p.out_O + (row_off - lane) * D;      // row 0 of the warp's block
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        tmem_ld32(tO + c * 32, v);
+      for (int h0 = 0; h0 < D; h0 += HALF) {
+        constexpr int W = HALF;
+        const int width = (D - h0 < W) ? (D - h0) : W;  // 64, or 32 for the tail of d = 96
+        uint32_t ov[W];
+#pragma unroll
+        for (int c = 0; c < W / 16; ++c)
+          if (c * 16 < width) tmem_ld16p(tO + h0 + c * 16, &ov[c * 16]);
         tc_wait_ld();
-        if (row_ok) {
+        if (h0 + HALF >= D) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_empty(k));
+        }
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
+        for (int c = 0; c < W / 32; ++c) {
+          if (c * 32 >= width) break;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
             float4 o;
-            o.x = __uint_as_float(v[4 * e + 0]) * inv_l;
-            o.y = __uint_as_float(v[4 * e + 1]) * inv_l;
-            o.z = __uint_as_float(v[4 * e + 2]) * inv_l;
-            o.w = __uint_as_float(v[4 * e + 3]) * inv_l;
-            dst[c * 8 + e] = o;
+            o.x = __uint_as_float(ov[c * 32 + 4 * q + 0]) * inv_l;
+            o.y = __uint_as_float(ov[c * 32 + 4 * q + 1]) * inv_l;
+            o.z = __uint_as_float(ov[c * 32 + 4 * q + 2]) * inv_l;
+            o.w = __uint_as_float(ov[c * 32 + 4 * q + 3]) * inv_l;
+            epi[lane * 8 + (q ^ (lane & 7))] = o;
           }
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int row = (lane >> 3) + 4 * q;
+            const int seg = lane & 7;
+            if (row < row_valid)
+              reinterpret_cast<float4 *>(blk + (size_t)row * D + h0 + c * 32)[seg] =
+                  epi[row * 8 + (seg ^ (row & 7))];
+          }
+          __syncwarp();
         }
       }
-      if (row_ok) p.out_lse[row_off] = (m_used + __log2f(l)) * 0.69314718055994531f;
+      if (r < rows_k) p.out_lse[row_off] = (m_used + __log2f(l)) * 0.69314718055994531f;
       if (p.out_by_slot && p.out_valid && k == 0 && r == 0) p.out_valid[idx] = 1;
-      tc_fence_before();
-      mbar_arrive(o_empty(k));
+     }
     }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 9) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tc_fence_before();
+    named_bar_arrive(1, kThreads);
   }
 }
 
@@ -474,6 +654,10 @@ cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const C
 #define DITANGO_LAUNCH(DD)                                                                       \
   case DD: {                                                                                     \
     auto kfn = attn::attn_partial_kernel<DD>;                                                    \
+    cudaFuncAttributes fa;                                                                       \
+    e = cudaFuncGetAttributes(&fa, kfn);                                                         \
+    if (e != cudaSuccess) return e;                                                              \
+    if (fa.numRegs != attn::kLaunchRegs) return cudaErrorInvalidConfiguration;                   \
     e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,                   \
                              attn::Cfg<DD>::SMEM);                                               \
     if (e != cudaSuccess) return e;                                                              \

@@ -22,7 +22,7 @@ namespace merge {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowsPerBlock = 128;
-constexpr int kUnroll = 8;
+constexpr int kBatch = 4;    // O vectors per row in flight per lane
 
 struct Src {
   const float *O;    // [Lmax][d] block of this (index, b*h)
@@ -44,8 +44,33 @@ __device__ __forceinline__ void store_out(void *out, int is_fp32, size_t off, fl
   }
 }
 
+__device__ __forceinline__ void fma4(float4 &acc, float w, const float4 &v) {
+  acc.x = fmaf(w, v.x, acc.x);
+  acc.y = fmaf(w, v.y, acc.y);
+  acc.z = fmaf(w, v.z, acc.z);
+  acc.w = fmaf(w, v.w, acc.w);
+}
+
+// Weights of one row: lane a holds lse of state a (l0) and a + 32 (l1);
+// returns exp(lse_a - L) for both and L = log sum_a exp(lse_a).
+__device__ __forceinline__ void lse_weights(float l0, float l1, float &w0, float &w1, float &L) {
+  float M = fmaxf(l0, l1);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const bool dead = !(M > -INFINITY);
+  const float Ms = dead ? 0.f : M;
+  const float e0 = expf(l0 - Ms), e1 = expf(l1 - Ms);
+  float S = e0 + e1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+  const float invS = dead ? 0.f : 1.f / S;
+  w0 = e0 * invS;
+  w1 = e1 * invS;
+  L = dead ? -INFINITY : Ms + logf(S);
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
 merge_kernel(DevGeom g, const signed char *__restrict__ plan, const float *__restrict__ part_O,
              const float *__restrict__ part_lse, float *cache_O, float *cache_lse,
              unsigned char *cache_valid, int writeback, void *out, int out_is_fp32, long long osb,
@@ -113,55 +138,79 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const float *__res
   const int b = bh / g.H, h = bh - (bh / g.H) * g.H;
   const int rend = (r0 + kRowsPerBlock < Li) ? r0 + kRowsPerBlock : Li;
 
-  for (int r = r0 + warp; r < rend; r += kWarps) {
-    // weights: lane a holds state a (and a + 32)
-    float l0 = -INFINITY, l1 = -INFINITY;
-    if (lane < nact) l0 = __ldg(src[lane].lse + r);
-    if (lane + 32 < nact) l1 = __ldg(src[lane + 32].lse + r);
-    float M = fmaxf(l0, l1);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const bool dead = !(M > -INFINITY);
-    const float Ms = dead ? 0.f : M;
-    float e0 = expf(l0 - Ms), e1 = expf(l1 - Ms);
-    float S = e0 + e1;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
-    const float invS = dead ? 0.f : 1.f / S;
-    const float w0 = e0 * invS, w1 = e1 * invS;
-    const float L = dead ? -INFINITY : Ms + logf(S);
-
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  // Two rows per warp iteration; every load of a row (its states' lse and the
+  // first kBatch O vectors) is issued before any of it is used.
+  for (int r = r0 + 2 * warp; r < rend; r += 2 * kWarps) {
+    const bool has_b = (r + 1) < rend;
+    float la0 = -INFINITY, la1 = -INFINITY, lb0 = -INFINITY, lb1 = -INFINITY;
+    if (lane < nact) {
+      la0 = __ldg(src[lane].lse + r);
+      if (has_b) lb0 = __ldg(src[lane].lse + r + 1);
+    }
+    if (lane + 32 < nact) {
+      la1 = __ldg(src[lane + 32].lse + r);
+      if (has_b) lb1 = __ldg(src[lane + 32].lse + r + 1);
+    }
     const bool act = lane < G;
-    for (int a0 = 0; a0 < nact; a0 += kUnroll) {
-      float4 v[kUnroll];
+    float4 va[kBatch], vb[kBatch];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int a = a0 + u;
-        if (act && a < nact)
-          v[u] = __ldg(reinterpret_cast<const float4 *>(src[a].O + (size_t)r * D) + lane);
-        else
-          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < kBatch; ++u) {
+      va[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      vb[u] = va[u];
+      if (act && u < nact) {
+        va[u] = __ldg(reinterpret_cast<const float4 *>(src[u].O + (size_t)r * D) + lane);
+        if (has_b) vb[u] = __ldg(reinterpret_cast<const float4 *>(src[u].O + (size_t)(r + 1) * D) + lane);
+      }
+    }
+    float wa0, wa1, wb0, wb1, La, Lb;
+    lse_weights(la0, la1, wa0, wa1, La);
+    lse_weights(lb0, lb1, wb0, wb1, Lb);
+    float4 acca = make_float4(0.f, 0.f, 0.f, 0.f), accb = acca;
+    for (int a0 = 0; a0 < nact; a0 += kBatch) {
+      if (a0 > 0) {
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int a = a0 + u;
+          if (act && a < nact) {
+            va[u] = __ldg(reinterpret_cast<const float4 *>(src[a].O + (size_t)r * D) + lane);
+            if (has_b) vb[u] = __ldg(reinterpret_cast<const float4 *>(src[a].O + (size_t)(r + 1) * D) + lane);
+          }
+        }
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kBatch; ++u) {
         const int a = a0 + u;
-        const float wa = __shfl_sync(0xffffffffu, (a < 32) ? w0 : w1, a & 31);
+        const float wa = __shfl_sync(0xffffffffu, (a < 32) ? wa0 : wa1, a & 31);
+        const float wb = __shfl_sync(0xffffffffu, (a < 32) ? wb0 : wb1, a & 31);
         if (a < nact) {
-          acc.x = fmaf(wa, v[u].x, acc.x);
-          acc.y = fmaf(wa, v[u].y, acc.y);
-          acc.z = fmaf(wa, v[u].z, acc.z);
-          acc.w = fmaf(wa, v[u].w, acc.w);
-          if (act && src[a].wbO) reinterpret_cast<float4 *>(src[a].wbO + (size_t)r * D)[lane] = v[u];
+          fma4(acca, wa, va[u]);
+          fma4(accb, wb, vb[u]);
+          if (act && src[a].wbO) {
+            reinterpret_cast<float4 *>(src[a].wbO + (size_t)r * D)[lane] = va[u];
+            if (has_b) reinterpret_cast<float4 *>(src[a].wbO + (size_t)(r + 1) * D)[lane] = vb[u];
+          }
         }
       }
     }
     // write back the lse of fresh states
-    if (lane < nact && src[lane].wblse) src[lane].wblse[r] = l0;
-    if (lane + 32 < nact && src[lane + 32].wblse) src[lane + 32].wblse[r] = l1;
+    if (lane < nact && src[lane].wblse) {
+      src[lane].wblse[r] = la0;
+      if (has_b) src[lane].wblse[r + 1] = lb0;
+    }
+    if (lane + 32 < nact && src[lane + 32].wblse) {
+      src[lane + 32].wblse[r] = la1;
+      if (has_b) src[lane + 32].wblse[r + 1] = lb1;
+    }
     const int n = g.part_off[i] + r;
-    if (act) store_out(out, out_is_fp32, (size_t)b * osb + (size_t)h * osh + (size_t)n * osn + lane * 4, acc);
-    if (out_lse && lane == 0) out_lse[((size_t)b * g.H + h) * g.N + n] = L;
+    const size_t obase = (size_t)b * osb + (size_t)h * osh + lane * 4;
+    if (act) {
+      store_out(out, out_is_fp32, obase + (size_t)n * osn, acca);
+      if (has_b) store_out(out, out_is_fp32, obase + (size_t)(n + 1) * osn, accb);
+    }
+    if (out_lse && lane == 0) {
+      out_lse[((size_t)b * g.H + h) * g.N + n] = La;
+      if (has_b) out_lse[((size_t)b * g.H + h) * g.N + n + 1] = Lb;
+    }
   }
 }
 
