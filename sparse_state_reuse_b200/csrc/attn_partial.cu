@@ -280,7 +280,9 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
    if (warp == 8) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // Warp-uniform loop; one elected lane arms the barriers and issues TMA.
+    {
+      const bool leader = elect_one();
       uint32_t kc = 0, vc = 0, uc = 0;
       // last armed phase per full barrier (for a clean stop on abort)
       // bit 2s: stage s armed at least once; bit 2s+1: parity of its last arming
@@ -290,32 +292,36 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
         const Item w = decode_item(p, row_fresh, it, nqt2);
         if (!w.live) continue;
-        if (!(ok = wait_bounded(q_empty, (uc & 1) ^ 1, ctl))) break;
+        if (!(ok = wait_warp(q_empty, (uc & 1) ^ 1, ctl))) break;
         const uint32_t qbytes = C::TILE * (w.rows1 > 0 ? 2 : 1);
-        mbar_arrive_expect_tx(q_full, qbytes);
+        if (leader) mbar_arrive_expect_tx(q_full, qbytes);
         q_armed = uc & 1;
-        for (int c = 0; c < C::NCH; ++c)
-          tma_load_4d(sQ + c * C::CHUNK, &tmQ, q_full, c * 64, w.q0, w.h, w.b);
-        if (w.rows1 > 0)
+        if (leader) {
           for (int c = 0; c < C::NCH; ++c)
-            tma_load_4d(sQ + C::TILE + c * C::CHUNK, &tmQ, q_full, c * 64, w.q0 + BM, w.h, w.b);
+            tma_load_4d(sQ + c * C::CHUNK, &tmQ, q_full, c * 64, w.q0, w.h, w.b);
+          if (w.rows1 > 0)
+            for (int c = 0; c < C::NCH; ++c)
+              tma_load_4d(sQ + C::TILE + c * C::CHUNK, &tmQ, q_full, c * 64, w.q0 + BM, w.h, w.b);
+        }
         for (int f = w.f0; f < w.f1 && ok; ++f) {
           const PairRange pr = pair_at(p, f);
           for (int t = 0; t < pr.T && ok; ++t) {
             const int row = pr.k0 + t * BN;
             int s = kc % kStages;
-            if (!(ok = wait_bounded(k_empty(s), ((kc / kStages) & 1) ^ 1, ctl))) break;
-            mbar_arrive_expect_tx(k_full(s), C::TILE);
+            if (!(ok = wait_warp(k_empty(s), ((kc / kStages) & 1) ^ 1, ctl))) break;
+            if (leader) mbar_arrive_expect_tx(k_full(s), C::TILE);
             k_armed = (k_armed & ~(3u << (2 * s))) | ((1u | (((kc / kStages) & 1u) << 1)) << (2 * s));
-            for (int c = 0; c < C::NCH; ++c)
-              tma_load_4d(sK + s * C::TILE + c * C::CHUNK, &tmK, k_full(s), c * 64, row, w.h, w.b);
+            if (leader)
+              for (int c = 0; c < C::NCH; ++c)
+                tma_load_4d(sK + s * C::TILE + c * C::CHUNK, &tmK, k_full(s), c * 64, row, w.h, w.b);
             ++kc;
             s = vc % kStages;
-            if (!(ok = wait_bounded(v_empty(s), ((vc / kStages) & 1) ^ 1, ctl))) break;
-            mbar_arrive_expect_tx(v_full(s), C::TILE);
+            if (!(ok = wait_warp(v_empty(s), ((vc / kStages) & 1) ^ 1, ctl))) break;
+            if (leader) mbar_arrive_expect_tx(v_full(s), C::TILE);
             v_armed = (v_armed & ~(3u << (2 * s))) | ((1u | (((vc / kStages) & 1u) << 1)) << (2 * s));
-            for (int c = 0; c < C::NCH; ++c)
-              tma_load_4d(sV + s * C::TILE + c * C::CHUNK, &tmV, v_full(s), c * 64, row, w.h, w.b);
+            if (leader)
+              for (int c = 0; c < C::NCH; ++c)
+                tma_load_4d(sV + s * C::TILE + c * C::CHUNK, &tmV, v_full(s), c * 64, row, w.h, w.b);
             ++vc;
           }
         }
@@ -336,7 +342,11 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop (warp-uniform control flow keeps the
+    // descriptors in uniform registers); one elected lane issues every MMA
+    // and commit, so the commits track exactly the MMAs that lane issued.
+    {
+      const bool leader = elect_one();
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);
       uint32_t kc = 0, vc = 0, uc = 0;
@@ -360,7 +370,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = (uint64_t)(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
-          mma_ss(d_tmem, a0 + off, b0 + off, idesc_qk, kk > 0);
+          if (leader) mma_ss(d_tmem, a0 + off, b0 + off, idesc_qk, kk > 0);
         }
       };
       auto pv = [&](int k, int vs, bool acc) {
@@ -370,78 +380,78 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const uint32_t a_tmem = tmem + k * 128;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(d_tmem, a_tmem + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv, (acc || kk > 0));
+          if (leader) mma_ts(d_tmem, a_tmem + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv, (acc || kk > 0));
       };
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
         const Item w = decode_item(p, row_fresh, it, nqt2);
         if (!w.live) continue;
         const bool has1 = w.rows1 > 0;
-        if (!(ok = wait_bounded(q_full, uc & 1, ctl))) break;
+        if (!(ok = wait_warp(q_full, uc & 1, ctl))) break;
         for (int f = w.f0; f < w.f1 && ok; ++f) {
           const PairRange pr = pair_at(p, f);
           const bool last_pair = (f + 1 == w.f1);
           int ks = kc % kStages;
-          if (!(ok = wait_bounded(k_full(ks), (kc / kStages) & 1, ctl))) break;
+          if (!(ok = wait_warp(k_full(ks), (kc / kStages) & 1, ctl))) break;
           tc_fence_after();
           qk(0, ks);
-          tc_commit(s_full(0));
+          commit_by(leader, s_full(0));
           if (has1) {
             qk(1, ks);
-            tc_commit(s_full(1));
+            commit_by(leader, s_full(1));
           }
-          tc_commit(k_empty(ks));
+          commit_by(leader, k_empty(ks));
           ++kc;
-          if (pr.T == 1 && last_pair) tc_commit(q_empty);
+          if (pr.T == 1 && last_pair) commit_by(leader, q_empty);
           for (int t = 0; t < pr.T && ok; ++t) {
             const int vs = vc % kStages;
-            if (!(ok = wait_bounded(v_full(vs), (vc / kStages) & 1, ctl))) break;
+            if (!(ok = wait_warp(v_full(vs), (vc / kStages) & 1, ctl))) break;
             const bool more = (t + 1 < pr.T);
             // ---- Q tile 0
-            if (!(ok = wait_bounded(p_full(0), pc[0] & 1, ctl))) break;
+            if (!(ok = wait_warp(p_full(0), pc[0] & 1, ctl))) break;
             ++pc[0];
             if (t == 0) {
-              if (!(ok = wait_bounded(o_empty(0), (oc[0] & 1) ^ 1, ctl))) break;
+              if (!(ok = wait_warp(o_empty(0), (oc[0] & 1) ^ 1, ctl))) break;
               ++oc[0];
             }
             tc_fence_after();
             pv(0, vs, t > 0);
-            if (!more) tc_commit(o_full(0));
+            if (!more) commit_by(leader, o_full(0));
             const int ks2 = kc % kStages;
             if (more) {
-              if (!(ok = wait_bounded(k_full(ks2), (kc / kStages) & 1, ctl))) break;
+              if (!(ok = wait_warp(k_full(ks2), (kc / kStages) & 1, ctl))) break;
               tc_fence_after();
               qk(0, ks2);
-              tc_commit(s_full(0));
+              commit_by(leader, s_full(0));
             }
             // ---- Q tile 1
             if (has1) {
-              if (!(ok = wait_bounded(p_full(1), pc[1] & 1, ctl))) break;
+              if (!(ok = wait_warp(p_full(1), pc[1] & 1, ctl))) break;
               ++pc[1];
               if (t == 0) {
-                if (!(ok = wait_bounded(o_empty(1), (oc[1] & 1) ^ 1, ctl))) break;
+                if (!(ok = wait_warp(o_empty(1), (oc[1] & 1) ^ 1, ctl))) break;
                 ++oc[1];
               }
               tc_fence_after();
               pv(1, vs, t > 0);
-              if (!more) tc_commit(o_full(1));
+              if (!more) commit_by(leader, o_full(1));
               if (more) {
                 qk(1, ks2);
-                tc_commit(s_full(1));
+                commit_by(leader, s_full(1));
               }
             }
-            tc_commit(v_empty(vs));
+            commit_by(leader, v_empty(vs));
             ++vc;
             if (more) {
-              tc_commit(k_empty(ks2));
+              commit_by(leader, k_empty(ks2));
               ++kc;
-              if (t + 2 == pr.T && last_pair) tc_commit(q_empty);
+              if (t + 2 == pr.T && last_pair) commit_by(leader, q_empty);
             }
           }
         }
         ++uc;
       }
       // drain: every MMA issued so far must finish before TMEM is released
-      tc_commit(drain);
+      commit_by(leader, drain);
       WaitCtl drain_ctl{nullptr, nullptr, 100000000LL};
       volatile int never = 0;
       drain_ctl.abort_flag = &never;

@@ -120,6 +120,23 @@ __device__ __forceinline__ void named_bar_arrive(int id, int count) {
   asm volatile("barrier.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Warp-wide bounded wait: every lane polls, the warp proceeds only if all
+// lanes saw the phase complete (a lane that gave up makes the whole warp
+// stop, keeping control flow warp-uniform).
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const WaitCtl &c) {
+  const bool ok = wait_bounded(bar, parity, c);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// One lane of a fully active warp (the same lane every call).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r));
+  return r != 0;
+}
+
 // --- TMA --------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const void *desc) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(desc)) : "memory");
@@ -167,6 +184,10 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
       : "memory");
+}
+
+__device__ __forceinline__ void commit_by(bool leader, uint32_t bar) {
+  if (leader) tc_commit(bar);
 }
 
 // D(tmem) (+)= A(smem desc) * B(smem desc)
