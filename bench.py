@@ -240,40 +240,65 @@ def run_ours(args, w, rank, world, local_rank):
     if status != 0:
         raise RuntimeError(f"device status {status}")
 
-    # end to end through the public API: pinned host inputs in, result out
+    # End to end through the public API: every step copies its Q/K/V in from
+    # pinned host memory and its output (bf16 O and fp32 lse) back out.  Two
+    # sets of device buffers let step s+1's uploads overlap step s's compute
+    # (copy-in stream -> compute stream -> copy-out stream, ordered by events).
     hq_p, hk_p, hv_p = (x.pin_memory() for x in (hq, hk, hv))
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h_lse = torch.empty(out_lse.shape, dtype=out_lse.dtype).pin_memory()
-    e2e_steps = max(3, min(args.steps, 10))
+    bufs = [(Q, K, V, out, out_lse)]
+    bufs.append((torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V),
+                 torch.empty_like(out), torch.empty_like(out_lse)))
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    done = [torch.cuda.Event() for _ in range(2)]
+    loaded = [torch.cuda.Event() for _ in range(2)]
+    drained = [torch.cuda.Event() for _ in range(2)]
+    e2e_steps = max(3, min(args.steps, 20))
 
-    def e2e_step():
-        with torch.cuda.stream(stream):
-            Q.copy_(hq_p, non_blocking=True)
-            K.copy_(hk_p, non_blocking=True)
-            V.copy_(hv_p, non_blocking=True)
-            pa.step(Q, K, V, out, out_lse, stream=stream, **kw)
-            h_out.copy_(out, non_blocking=True)
-            h_lse.copy_(out_lse, non_blocking=True)
+    def e2e_run(n):
+        for i in range(n):
+            bq, bk, bv, bo, bl = bufs[i % 2]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(done[i % 2])
+                bq.copy_(hq_p, non_blocking=True)
+                bk.copy_(hk_p, non_blocking=True)
+                bv.copy_(hv_p, non_blocking=True)
+                loaded[i % 2].record(s_in)
+            with torch.cuda.stream(stream):
+                stream.wait_event(loaded[i % 2])
+                if i >= 2:
+                    stream.wait_event(drained[i % 2])
+                pa.step(bq, bk, bv, bo, bl, stream=stream, **kw)
+                done[i % 2].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[i % 2])
+                h_out.copy_(bo, non_blocking=True)
+                h_lse.copy_(bl, non_blocking=True)
+                drained[i % 2].record(s_out)
 
-    e2e_step()
-    stream.synchronize()
+    e2e_run(2)
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     a, b = ev(), ev()
-    a.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    b.record(stream)
-    stream.synchronize()
+    a.record(s_in)
+    e2e_run(e2e_steps)
+    s_in.wait_stream(s_out)
+    b.record(s_in)
+    torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / e2e_steps
     e2e_ms = max_over_ranks(e2e_ms, dev, dist)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
     d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
+    del bufs
 
     ms_step = ms / args.steps
     peaks, peak_src = load_peaks()
     tflops_part = flops / (part_ms * 1e-3) / 1e12
-    peak_t = float(peaks.get("bf16_tflops_sustained" if args.steps * ms_step > 2000 else "bf16_tflops"))
+    peak_t = float(peaks.get("bf16_tflops"))          # burst figure: the conservative denominator
+    peak_ts = float(peaks.get("bf16_tflops_sustained", peak_t))
     merge_gbs = mbytes / (merge_ms * 1e-3) / 1e9
     traffic = recorded_traffic("attn_partial.cu", w.name)
     res = {
@@ -298,6 +323,7 @@ def run_ours(args, w, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "attn_partial", "achieved": round(tflops_part, 2),
                      "peak": peak_t, "unit": "TFLOP/s", "frac": round(tflops_part / peak_t, 4),
                      "peak_source": peak_src, "traffic": traffic,
+                     "frac_of_sustained_peak": round(tflops_part / peak_ts, 4),
                      "kernel_ms": round(part_ms, 4),
                      "algorithmic_flops_per_launch": flops},
         "merge_roofline": {"bound": "hbm", "achieved": round(merge_gbs, 1),
@@ -389,7 +415,7 @@ def run_reference(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(configs.BY_NAME))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
