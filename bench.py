@@ -49,16 +49,18 @@ def effective_flops(w, fresh_mask):
     return float(4.0 * w.d * w.BH * (np.outer(L, L) * fresh_mask).sum())
 
 
-def merge_bytes(w, A, fresh_mask, out_bytes_per_elem=2, writeback=False):
+def merge_bytes(w, A, fresh_mask, out_bytes_per_elem=2, writeback=False, state_o_bytes=4):
     """Algorithmic HBM bytes of the merge: every active state read once
-    ((d+1) fp32 per row), the output written once (d elements + fp32 lse),
-    plus the write-back of fresh states when they are copied."""
+    (d O values of state_o_bytes each + an fp32 lse per row), the output
+    written once (d elements + fp32 lse), plus the write-back of fresh states
+    when they are copied."""
     po = np.array(w.part_off())
     L = np.diff(po)
     rows_states = (A.sum(axis=1) * L).sum() * w.BH
-    b = rows_states * (w.d + 1) * 4 + w.BH * w.N * (w.d * out_bytes_per_elem + 4)
+    row_state = w.d * state_o_bytes + 4
+    b = rows_states * row_state + w.BH * w.N * (w.d * out_bytes_per_elem + 4)
     if writeback:
-        b += (fresh_mask.sum(axis=1) * L).sum() * w.BH * (w.d + 1) * 4
+        b += (fresh_mask.sum(axis=1) * L).sum() * w.BH * row_state
     return float(b)
 
 
@@ -171,7 +173,7 @@ def run_ours(args, w, rank, world, local_rank):
     hq, hk, hv = (up(inputs.full(w, t)) for t in "qkv")
     Q, K, V = (x.to(dev) for x in (hq, hk, hv))
     pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask(),
-                                 device=dev)
+                                 device=dev, state_bf16=args.state_bf16)
     if w.reuses:
         Kp = up(inputs.full(w, "k", prev=True)).to(dev)
         Vp = up(inputs.full(w, "v", prev=True)).to(dev)
@@ -191,7 +193,7 @@ def run_ours(args, w, rank, world, local_rank):
     A = plan != 0
     fresh = plan == 1
     flops = effective_flops(w, fresh)
-    mbytes = merge_bytes(w, A, fresh)
+    mbytes = merge_bytes(w, A, fresh, state_o_bytes=2 if args.state_bf16 else 4)
     launches_per_step = (1 if w.anchor else 2) + 1 + 1
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
@@ -317,6 +319,7 @@ def run_ours(args, w, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) bf16, shaped like the pages' workloads)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "P": w.P,
                    "frames": w.F, "fresh_pairs": int(fresh.sum()), "active_pairs": int(A.sum()),
+                   "state_format": "bf16 O + fp32 lse" if args.state_bf16 else "fp32 O + fp32 lse",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (Q/K/V %.0f MB, states %.0f MB)" % (
                        h2d / 1e6, pa.state_O.numel() * 4 / 1e6)},
@@ -420,6 +423,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(configs.BY_NAME))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
+    ap.add_argument("--state-bf16", action="store_true",
+                    help="compressed attention-state cache: O stored as bf16")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

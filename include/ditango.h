@@ -30,8 +30,9 @@
  *    Device-side failures (a pipeline wait that exceeded its time limit) are
  *    written as a status code into `dev_status` where a call takes one.
  *  - Token order is frame-major; partitions are contiguous token ranges.
- *  - State layout ("state buffer"): O is float32 [n_idx][B*H][Lmax][d] and
- *    lse is float32 [n_idx][B*H][Lmax], where Lmax = max partition length
+ *  - State layout ("state buffer"): O is [n_idx][B*H][Lmax][d], float32 or
+ *    (state_bf16 = 1, a compressed cache) bfloat16 bit patterns, and lse is
+ *    float32 [n_idx][B*H][Lmax], where Lmax = max partition length
  *    (ditango_state_rows) and the leading index is either the slot of an
  *    active pair (row-major rank of the active pairs, see ditango_slot_table)
  *    or the position of a pair in the fresh list.  Row r of pair (i, j)
@@ -147,6 +148,11 @@ ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
  *   out_O/out_lse  dev state buffer; index = f (out_by_slot = 0) or the
  *                pair's slot (out_by_slot = 1, e.g. writing the cache in
  *                place).  Must hold counts[0] (resp. all slots) indices.
+ *   state_bf16   nonzero: O is stored as bf16 (the normalised fp32 O rounded
+ *                to nearest even); lse stays float32.  A compressed cache
+ *                halves the cache memory and the merge's read traffic
+ *                (DiTango, "Significato e Claim": cache memory is the
+ *                method's limitation and cache compression its next step).
  *   out_valid    dev uint8 [slots] or NULL; with out_by_slot = 1 the written
  *                slots are set to 1.
  *   dev_status   dev int32 or NULL; set to DITANGO_ERR_TIMEOUT if a pipeline
@@ -155,9 +161,10 @@ ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
 ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q,
                                     const uint16_t *K, const uint16_t *V,
                                     const int32_t *fresh_list, const int32_t *counts,
-                                    float scale, float *out_O, float *out_lse,
-                                    int32_t out_by_slot, uint8_t *out_valid,
-                                    int32_t *dev_status, ditango_stream stream);
+                                    float scale, void *out_O, float *out_lse,
+                                    int32_t out_by_slot, int32_t state_bf16,
+                                    uint8_t *out_valid, int32_t *dev_status,
+                                    ditango_stream stream);
 
 /* Merge: the final output of every token is the log-sum-exp composition of
  * the states of its partition's active pairs (DiTango, "Composizione dello
@@ -169,25 +176,27 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q,
  *   plan          dev int8 [P*P] from ditango_plan.
  *   writeback     nonzero: also copy each fresh state into its cache slot
  *                 and mark cache_valid (ignored when part_O is NULL).
+ *   state_bf16    format of every state buffer passed (see ditango_attn_partial).
  *   out           dev [B, H, N, d] (element strides out_strides for b, h, n;
  *                 NULL = contiguous), bf16 bits (out_is_fp32 = 0) or float32.
  *   out_lse       dev float32 [B, H, N] or NULL.
  * A token whose partition has no active pair gets O = 0, lse = -inf. */
 ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan,
-                             const float *part_O, const float *part_lse,
-                             float *cache_O, float *cache_lse, uint8_t *cache_valid,
-                             int32_t writeback, void *out, int32_t out_is_fp32,
-                             const int64_t *out_strides, float *out_lse,
-                             ditango_stream stream);
+                             const void *part_O, const float *part_lse,
+                             void *cache_O, float *cache_lse, uint8_t *cache_valid,
+                             int32_t writeback, int32_t state_bf16, void *out,
+                             int32_t out_is_fp32, const int64_t *out_strides,
+                             float *out_lse, ditango_stream stream);
 
 /* Cache update: copy the fresh states (indexed by fresh position) into their
  * cache slots and mark them valid -- the write half of an anchor step
  * (DiTango, "Anchor Steps": everything is recomputed and the cache
  * refreshed). */
 ditango_status ditango_cache_update(const ditango_geom *g, const int8_t *plan,
-                                    const float *part_O, const float *part_lse,
-                                    float *cache_O, float *cache_lse,
-                                    uint8_t *cache_valid, ditango_stream stream);
+                                    const void *part_O, const float *part_lse,
+                                    void *cache_O, float *cache_lse,
+                                    uint8_t *cache_valid, int32_t state_bf16,
+                                    ditango_stream stream);
 
 /* Allocation-free variant of ditango_plan (no counterpart in the papers: it
  * exists for callers, not for the method).  For callers that cannot allocate

@@ -27,14 +27,15 @@ from ._abi import (  # noqa: F401
 class PartitionedAttention:
     """Device buffers for one geometry and the three-call step.
 
-    The state buffer (O float32 [slots, B*H, Lmax, d], lse float32
-    [slots, B*H, Lmax]) is the attention-state cache: a step writes its fresh
-    states into their slots and the merge reads every active pair from it, so
-    after a step the cache holds this step's fresh states and the reused ones.
+    The state buffer (O [slots, B*H, Lmax, d] float32, or bfloat16 with
+    state_bf16=True, a compressed cache; lse float32 [slots, B*H, Lmax]) is
+    the attention-state cache: a step writes its fresh states into their
+    slots and the merge reads every active pair from it, so after a step the
+    cache holds this step's fresh states and the reused ones.
     """
 
     def __init__(self, B, H, N, d, part_off, frame_off=None, frame_mask=None,
-                 device="cuda", strides=None):
+                 device="cuda", strides=None, state_bf16=False):
         import torch
         self.B, self.H, self.N, self.d = B, H, N, d
         self.part_off = list(part_off)
@@ -47,7 +48,10 @@ class PartitionedAttention:
         self.Lmax = ditango_state_rows(self.geom)
         BH = B * H
         dev = self.device
-        self.state_O = torch.empty((self.n_slots, BH, self.Lmax, d), dtype=torch.float32, device=dev)
+        self.state_bf16 = bool(state_bf16)
+        self.state_O = torch.empty((self.n_slots, BH, self.Lmax, d),
+                                   dtype=torch.bfloat16 if self.state_bf16 else torch.float32,
+                                   device=dev)
         self.state_lse = torch.empty((self.n_slots, BH, self.Lmax), dtype=torch.float32, device=dev)
         self.valid = torch.zeros(self.n_slots, dtype=torch.uint8, device=dev)
         self.plan = torch.zeros(self.P * self.P, dtype=torch.int8, device=dev)
@@ -77,12 +81,14 @@ class PartitionedAttention:
     def partial(self, Q, K, V, scale=0.0, stream=None):
         self._bind(Q, K, V)
         ditango_attn_partial(self.geom, Q, K, V, self.fresh_list, self.counts, scale,
-                             self.state_O, self.state_lse, 1, self.valid, self.status, stream)
+                             self.state_O, self.state_lse, 1, self.valid, self.status, stream,
+                             state_bf16=self.state_bf16)
 
     def merge(self, out, out_lse=None, stream=None):
         import torch
         ditango_merge(self.geom, self.plan, None, None, self.state_O, self.state_lse, self.valid, 0,
-                      out, out.dtype == torch.float32, tuple(out.stride()[:3]), out_lse, stream)
+                      out, out.dtype == torch.float32, tuple(out.stride()[:3]), out_lse, stream,
+                      state_bf16=self.state_bf16)
 
     def step(self, Q, K, V, out, out_lse=None, band_k=0, budget=1.0, anchor=False, scale=0.0,
              stream=None):

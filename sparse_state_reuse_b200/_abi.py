@@ -58,10 +58,11 @@ _SIGS = {
     "ditango_plan_workspace_size": (C.c_size_t, [_G]),
     "ditango_plan": (C.c_int, [_G, _P, _P, C.c_int32, C.c_double, C.c_int32, _P, _P, _P, _P, _P,
                                C.c_size_t, _P]),
-    "ditango_attn_partial": (C.c_int, [_G, _P, _P, _P, _P, _P, C.c_float, _P, _P, C.c_int32, _P,
-                                       _P, _P]),
-    "ditango_merge": (C.c_int, [_G, _P, _P, _P, _P, _P, _P, C.c_int32, _P, C.c_int32, _P, _P, _P]),
-    "ditango_cache_update": (C.c_int, [_G, _P, _P, _P, _P, _P, _P, _P]),
+    "ditango_attn_partial": (C.c_int, [_G, _P, _P, _P, _P, _P, C.c_float, _P, _P, C.c_int32,
+                                       C.c_int32, _P, _P, _P]),
+    "ditango_merge": (C.c_int, [_G, _P, _P, _P, _P, _P, _P, C.c_int32, C.c_int32, _P, C.c_int32,
+                                _P, _P, _P]),
+    "ditango_cache_update": (C.c_int, [_G, _P, _P, _P, _P, _P, _P, C.c_int32, _P]),
     "ditango_plan_noalloc": (C.c_int, [_G, _P, _P, C.c_int32, C.c_double, C.c_int32, _P, _P, _P,
                                        _P, _P]),
     "ditango_set_wait_limit_ns": (None, [C.c_int64]),
@@ -176,30 +177,32 @@ def ditango_plan(geom, cache_lse, cache_valid, band_k, budget, anchor, plan, fre
 
 
 def ditango_attn_partial(geom, Q, K, V, fresh_list, counts, scale, out_O, out_lse,
-                         out_by_slot=0, out_valid=None, dev_status=None, stream=None):
+                         out_by_slot=0, out_valid=None, dev_status=None, stream=None,
+                         state_bf16=0):
     _check("ditango_attn_partial", _lib.ditango_attn_partial(
         geom.ref, _ptr(Q), _ptr(K), _ptr(V), _ptr(fresh_list), _ptr(counts), float(scale),
-        _ptr(out_O), _ptr(out_lse), int(out_by_slot), _ptr(out_valid), _ptr(dev_status),
-        _stream(stream)))
+        _ptr(out_O), _ptr(out_lse), int(out_by_slot), int(bool(state_bf16)), _ptr(out_valid),
+        _ptr(dev_status), _stream(stream)))
 
 
 def ditango_merge(geom, plan, part_O, part_lse, cache_O, cache_lse, cache_valid, writeback,
-                  out, out_is_fp32, out_strides=None, out_lse=None, stream=None):
+                  out, out_is_fp32, out_strides=None, out_lse=None, stream=None, state_bf16=0):
     strides = None
     if out_strides is not None:
         strides = (C.c_int64 * 3)(*[int(s) for s in out_strides])
     _check("ditango_merge", _lib.ditango_merge(
         geom.ref, _ptr(plan), _ptr(part_O), _ptr(part_lse), _ptr(cache_O), _ptr(cache_lse),
-        _ptr(cache_valid), int(bool(writeback)), _ptr(out), int(bool(out_is_fp32)),
+        _ptr(cache_valid), int(bool(writeback)), int(bool(state_bf16)), _ptr(out),
+        int(bool(out_is_fp32)),
         C.cast(strides, C.c_void_p) if strides is not None else None, _ptr(out_lse),
         _stream(stream)))
 
 
 def ditango_cache_update(geom, plan, part_O, part_lse, cache_O, cache_lse, cache_valid,
-                         stream=None):
+                         stream=None, state_bf16=0):
     _check("ditango_cache_update", _lib.ditango_cache_update(
         geom.ref, _ptr(plan), _ptr(part_O), _ptr(part_lse), _ptr(cache_O), _ptr(cache_lse),
-        _ptr(cache_valid), _stream(stream)))
+        _ptr(cache_valid), int(bool(state_bf16)), _stream(stream)))
 
 
 def ditango_set_wait_limit_ns(ns: int) -> None:

@@ -63,7 +63,7 @@ struct Params {
   const int *fresh_list;
   const int *counts;
   float scale_log2;       // logit scale * log2(e)
-  float *out_O;
+  void *out_O;             // float32, or bf16 when the state format is bf16
   float *out_lse;
   int out_by_slot;
   unsigned char *out_valid;
@@ -194,7 +194,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
-template <int D>
+template <int D, bool SB>   // SB: states stored with bf16 O (compressed cache)
 __global__ void __launch_bounds__(kThreads, 1)
 attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params p) {
@@ -588,7 +588,6 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       const float inv_l = 1.f / l;
       float4 *epi = reinterpret_cast<float4 *>(smem + C::OFF_EPI + (warp & 7) * 4096);
       const int row_valid = rows_k - (r & ~31);         // valid rows of this warp
-      float *blk = p.out_O + (row_off - lane) * D;      // row 0 of the warp's block
 #pragma unroll
       for (int h0 = 0; h0 < D; h0 += HALF) {
         constexpr int W = HALF;
@@ -606,23 +605,47 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
         for (int c = 0; c < W / 32; ++c) {
           if (c * 32 >= width) break;
+          if constexpr (!SB) {
+            float *blk = static_cast<float *>(p.out_O) + (row_off - lane) * D;  // row 0 of the warp's block
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float4 o;
-            o.x = __uint_as_float(ov[c * 32 + 4 * q + 0]) * inv_l;
-            o.y = __uint_as_float(ov[c * 32 + 4 * q + 1]) * inv_l;
-            o.z = __uint_as_float(ov[c * 32 + 4 * q + 2]) * inv_l;
-            o.w = __uint_as_float(ov[c * 32 + 4 * q + 3]) * inv_l;
-            epi[lane * 8 + (q ^ (lane & 7))] = o;
-          }
-          __syncwarp();
+            for (int q = 0; q < 8; ++q) {
+              float4 o;
+              o.x = __uint_as_float(ov[c * 32 + 4 * q + 0]) * inv_l;
+              o.y = __uint_as_float(ov[c * 32 + 4 * q + 1]) * inv_l;
+              o.z = __uint_as_float(ov[c * 32 + 4 * q + 2]) * inv_l;
+              o.w = __uint_as_float(ov[c * 32 + 4 * q + 3]) * inv_l;
+              epi[lane * 8 + (q ^ (lane & 7))] = o;
+            }
+            __syncwarp();
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int row = (lane >> 3) + 4 * q;
-            const int seg = lane & 7;
-            if (row < row_valid)
-              reinterpret_cast<float4 *>(blk + (size_t)row * D + h0 + c * 32)[seg] =
-                  epi[row * 8 + (seg ^ (row & 7))];
+            for (int q = 0; q < 8; ++q) {
+              const int row = (lane >> 3) + 4 * q;
+              const int seg = lane & 7;
+              if (row < row_valid)
+                reinterpret_cast<float4 *>(blk + (size_t)row * D + h0 + c * 32)[seg] =
+                    epi[row * 8 + (seg ^ (row & 7))];
+            }
+          } else {
+            // bf16 O: 32 columns = 64 bytes per row; 4 stores of 8 rows each
+            uint16_t *blk = static_cast<uint16_t *>(p.out_O) + (row_off - lane) * D;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 u;
+              u.x = pack_bf16(__uint_as_float(ov[c * 32 + 8 * q + 0]) * inv_l, __uint_as_float(ov[c * 32 + 8 * q + 1]) * inv_l);
+              u.y = pack_bf16(__uint_as_float(ov[c * 32 + 8 * q + 2]) * inv_l, __uint_as_float(ov[c * 32 + 8 * q + 3]) * inv_l);
+              u.z = pack_bf16(__uint_as_float(ov[c * 32 + 8 * q + 4]) * inv_l, __uint_as_float(ov[c * 32 + 8 * q + 5]) * inv_l);
+              u.w = pack_bf16(__uint_as_float(ov[c * 32 + 8 * q + 6]) * inv_l, __uint_as_float(ov[c * 32 + 8 * q + 7]) * inv_l);
+              reinterpret_cast<uint4 *>(epi)[lane * 4 + (q ^ ((lane >> 1) & 3))] = u;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int row = (lane >> 2) + 8 * i;
+              const int seg = lane & 3;
+              if (row < row_valid)
+                reinterpret_cast<uint4 *>(blk + (size_t)row * D + h0 + c * 32)[seg] =
+                    reinterpret_cast<const uint4 *>(epi)[row * 4 + (seg ^ ((row >> 1) & 3))];
+            }
           }
           __syncwarp();
         }
@@ -641,9 +664,9 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 // Host launcher (called from the C ABI after validation).
 cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const CUtensorMap &tk,
                                 const CUtensorMap &tv, const int *fresh_list, const int *counts,
-                                float scale, float *out_O, float *out_lse, int out_by_slot,
-                                unsigned char *out_valid, int *dev_status, long long wait_limit_ns,
-                                int num_sms, cudaStream_t stream) {
+                                float scale, void *out_O, float *out_lse, int out_by_slot,
+                                int state_bf16, unsigned char *out_valid, int *dev_status,
+                                long long wait_limit_ns, int num_sms, cudaStream_t stream) {
   attn::Params p;
   p.g = g;
   p.fresh_list = fresh_list;
@@ -663,7 +686,7 @@ cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const C
   switch (g.d) {
 #define DITANGO_LAUNCH(DD)                                                                       \
   case DD: {                                                                                     \
-    auto kfn = attn::attn_partial_kernel<DD>;                                                    \
+    auto kfn = state_bf16 ? attn::attn_partial_kernel<DD, true> : attn::attn_partial_kernel<DD, false>; \
     cudaFuncAttributes fa;                                                                       \
     e = cudaFuncGetAttributes(&fa, kfn);                                                         \
     if (e != cudaSuccess) return e;                                                              \

@@ -11,21 +11,22 @@
 namespace ditango {
 cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const CUtensorMap &tk,
                                 const CUtensorMap &tv, const int *fresh_list, const int *counts,
-                                float scale, float *out_O, float *out_lse, int out_by_slot,
-                                unsigned char *out_valid, int *dev_status, long long wait_limit_ns,
-                                int num_sms, cudaStream_t stream);
+                                float scale, void *out_O, float *out_lse, int out_by_slot,
+                                int state_bf16, unsigned char *out_valid, int *dev_status,
+                                long long wait_limit_ns, int num_sms, cudaStream_t stream);
 size_t plan_workspace_bytes(const DevGeom &g);
 cudaError_t launch_plan(const DevGeom &g, const float *cache_lse, const unsigned char *cache_valid,
                         int band_k, int target, int anchor, signed char *plan_out, int *fresh_list,
                         int *counts, float *score_out, void *workspace, cudaStream_t stream);
-cudaError_t launch_merge(const DevGeom &g, const signed char *plan, const float *part_O,
-                         const float *part_lse, float *cache_O, float *cache_lse,
-                         unsigned char *cache_valid, int writeback, void *out, int out_is_fp32,
-                         long long osb, long long osh, long long osn, float *out_lse,
-                         cudaStream_t stream);
-cudaError_t launch_cache_update(const DevGeom &g, const signed char *plan, const float *part_O,
-                                const float *part_lse, float *cache_O, float *cache_lse,
-                                unsigned char *cache_valid, int num_sms, cudaStream_t stream);
+cudaError_t launch_merge(const DevGeom &g, const signed char *plan, const void *part_O,
+                         const float *part_lse, void *cache_O, float *cache_lse,
+                         unsigned char *cache_valid, int writeback, int state_bf16, void *out,
+                         int out_is_fp32, long long osb, long long osh, long long osn,
+                         float *out_lse, cudaStream_t stream);
+cudaError_t launch_cache_update(const DevGeom &g, const signed char *plan, const void *part_O,
+                                const float *part_lse, void *cache_O, float *cache_lse,
+                                unsigned char *cache_valid, int state_bf16, int num_sms,
+                                cudaStream_t stream);
 cudaError_t launch_bounded_wait_selftest(long long limit_ns, int *dev_status,
                                          cudaStream_t stream);
 }  // namespace ditango
@@ -231,9 +232,10 @@ ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
 
 ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q, const uint16_t *K,
                                     const uint16_t *V, const int32_t *fresh_list,
-                                    const int32_t *counts, float scale, float *out_O,
-                                    float *out_lse, int32_t out_by_slot, uint8_t *out_valid,
-                                    int32_t *dev_status, ditango_stream stream) {
+                                    const int32_t *counts, float scale, void *out_O,
+                                    float *out_lse, int32_t out_by_slot, int32_t state_bf16,
+                                    uint8_t *out_valid, int32_t *dev_status,
+                                    ditango_stream stream) {
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
   if (st != DITANGO_OK) return st;
@@ -249,16 +251,16 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q, co
       !make_qkv_map(&tv, V, dg, g->v_strides))
     return DITANGO_ERR_CUDA;
   return cuda_status(launch_attn_partial(dg, tq, tk, tv, fresh_list, counts, scale, out_O, out_lse,
-                                         out_by_slot ? 1 : 0, out_valid, dev_status,
-                                         g_wait_limit_ns, num_sms_current(),
+                                         out_by_slot ? 1 : 0, state_bf16 ? 1 : 0, out_valid,
+                                         dev_status, g_wait_limit_ns, num_sms_current(),
                                          static_cast<cudaStream_t>(stream)));
 }
 
-ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan, const float *part_O,
-                             const float *part_lse, float *cache_O, float *cache_lse,
-                             uint8_t *cache_valid, int32_t writeback, void *out,
-                             int32_t out_is_fp32, const int64_t *out_strides, float *out_lse,
-                             ditango_stream stream) {
+ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan, const void *part_O,
+                             const float *part_lse, void *cache_O, float *cache_lse,
+                             uint8_t *cache_valid, int32_t writeback, int32_t state_bf16,
+                             void *out, int32_t out_is_fp32, const int64_t *out_strides,
+                             float *out_lse, ditango_stream stream) {
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
   if (st != DITANGO_OK) return st;
@@ -280,13 +282,14 @@ ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan, const fl
     return DITANGO_ERR_INVALID;
   return cuda_status(launch_merge(dg, reinterpret_cast<const signed char *>(plan), part_O,
                                   part_lse, cache_O, cache_lse, cache_valid,
-                                  (writeback && part_O) ? 1 : 0, out, out_is_fp32 ? 1 : 0, osb,
-                                  osh, osn, out_lse, static_cast<cudaStream_t>(stream)));
+                                  (writeback && part_O) ? 1 : 0, state_bf16 ? 1 : 0, out,
+                                  out_is_fp32 ? 1 : 0, osb, osh, osn, out_lse,
+                                  static_cast<cudaStream_t>(stream)));
 }
 
 ditango_status ditango_cache_update(const ditango_geom *g, const int8_t *plan,
-                                    const float *part_O, const float *part_lse, float *cache_O,
-                                    float *cache_lse, uint8_t *cache_valid,
+                                    const void *part_O, const float *part_lse, void *cache_O,
+                                    float *cache_lse, uint8_t *cache_valid, int32_t state_bf16,
                                     ditango_stream stream) {
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
@@ -294,7 +297,8 @@ ditango_status ditango_cache_update(const ditango_geom *g, const int8_t *plan,
   if (!plan || !part_O || !part_lse || !cache_O || !cache_lse) return DITANGO_ERR_INVALID;
   return cuda_status(launch_cache_update(dg, reinterpret_cast<const signed char *>(plan), part_O,
                                          part_lse, cache_O, cache_lse, cache_valid,
-                                         num_sms_current(), static_cast<cudaStream_t>(stream)));
+                                         state_bf16 ? 1 : 0, num_sms_current(),
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 void ditango_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns = ns > 0 ? ns : 1; }

@@ -25,11 +25,75 @@ constexpr int kRowsPerBlock = 128;
 constexpr int kBatch = 4;    // O vectors per row in flight per lane
 
 struct Src {
-  const float *O;    // [Lmax][d] block of this (index, b*h)
+  const char *O;     // [Lmax][d] block of this (index, b*h): float32, or bf16 (SB)
   const float *lse;  // [Lmax]
-  float *wbO;        // cache block to write back into, or null
+  char *wbO;         // cache block to write back into, or null
   float *wblse;
 };
+
+// Four consecutive O values of a state row (float32, or bf16 when SB).
+template <bool SB>
+__device__ __forceinline__ float4 load_o4(const char *p) {
+  if constexpr (SB) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+  } else {
+    return __ldg(reinterpret_cast<const float4 *>(p));
+  }
+}
+
+// Raw form of four stored O values (kept packed until used).
+template <bool SB>
+struct Raw4 {
+  using T = float4;
+};
+template <>
+struct Raw4<true> {
+  using T = uint2;
+};
+template <bool SB>
+__device__ __forceinline__ typename Raw4<SB>::T load_raw4(const char *p) {
+  if constexpr (SB)
+    return __ldg(reinterpret_cast<const uint2 *>(p));
+  else
+    return __ldg(reinterpret_cast<const float4 *>(p));
+}
+template <bool SB>
+__device__ __forceinline__ float4 widen4(typename Raw4<SB>::T u) {
+  if constexpr (SB)
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+  else
+    return u;
+}
+template <bool SB>
+__device__ __forceinline__ typename Raw4<SB>::T zero_raw4() {
+  if constexpr (SB)
+    return make_uint2(0u, 0u);
+  else
+    return make_float4(0.f, 0.f, 0.f, 0.f);
+}
+template <bool SB>
+__device__ __forceinline__ void store_raw4(char *p, typename Raw4<SB>::T u) {
+  if constexpr (SB)
+    *reinterpret_cast<uint2 *>(p) = u;
+  else
+    *reinterpret_cast<float4 *>(p) = u;
+}
+
+// Store four values that came from load_o4 (exact in either format).
+template <bool SB>
+__device__ __forceinline__ void store_o4(char *p, float4 v) {
+  if constexpr (SB) {
+    uint2 u;
+    u.x = (__float_as_uint(v.x) >> 16) | (__float_as_uint(v.y) & 0xffff0000u);
+    u.y = (__float_as_uint(v.z) >> 16) | (__float_as_uint(v.w) & 0xffff0000u);
+    *reinterpret_cast<uint2 *>(p) = u;
+  } else {
+    *reinterpret_cast<float4 *>(p) = v;
+  }
+}
 
 __device__ __forceinline__ void store_out(void *out, int is_fp32, size_t off, float4 v) {
   if (is_fp32) {
@@ -69,13 +133,15 @@ __device__ __forceinline__ void lse_weights(float l0, float l1, float &w0, float
   L = dead ? -INFINITY : Ms + logf(S);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 4)
-merge_kernel(DevGeom g, const signed char *__restrict__ plan, const float *__restrict__ part_O,
-             const float *__restrict__ part_lse, float *cache_O, float *cache_lse,
+template <int D, bool SB>
+__global__ void __launch_bounds__(kThreads, SB ? 3 : 4)
+merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__restrict__ part_O,
+             const float *__restrict__ part_lse, char *cache_O, float *cache_lse,
              unsigned char *cache_valid, int writeback, void *out, int out_is_fp32, long long osb,
              long long osh, long long osn, float *__restrict__ out_lse) {
   constexpr int G = D / 4;  // lanes carrying one row
+  constexpr int ES = SB ? 2 : 4;            // bytes per stored O element
+  constexpr size_t ROWB = (size_t)D * ES;   // bytes per state row
   const int i = blockIdx.y;
   const int bh = blockIdx.z;
   const int Li = g.part_off[i + 1] - g.part_off[i];
@@ -85,6 +151,8 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const float *__res
   __shared__ Src src[kMaxP];
   __shared__ int s_nact, s_fresh_before;
   __shared__ int warp_cnt[kWarps];
+  __shared__ signed char s_plan[kMaxP];
+  if (threadIdx.x < P) s_plan[threadIdx.x] = plan[i * P + threadIdx.x];
 
   // fresh pairs before row i (row-major), for fresh-list positions
   int cnt = 0;
@@ -103,27 +171,27 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const float *__res
     int fpos = fb;
     for (int j = 0; j < P; ++j) {
       if (!((g.row_mask[i] >> j) & 1ull)) continue;
-      const int code = plan[i * P + j];
+      const int code = s_plan[j];
       const int slot = slot0 + __popcll(g.row_mask[i] & ((j == 0) ? 0ull : (~0ull >> (64 - j))));
       Src s;
       s.wbO = nullptr;
       s.wblse = nullptr;
       if (code == DITANGO_PLAN_FRESH) {
         if (part_O != nullptr) {
-          s.O = part_O + ((size_t)fpos * blk + (size_t)bh * g.Lmax) * D;
+          s.O = part_O + ((size_t)fpos * blk + (size_t)bh * g.Lmax) * ROWB;
           s.lse = part_lse + (size_t)fpos * blk + (size_t)bh * g.Lmax;
           if (writeback) {
-            s.wbO = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * D;
+            s.wbO = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * ROWB;
             s.wblse = cache_lse + (size_t)slot * blk + (size_t)bh * g.Lmax;
             if (cache_valid && bh == 0 && blockIdx.x == 0) cache_valid[slot] = 1;
           }
         } else {
-          s.O = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * D;
+          s.O = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * ROWB;
           s.lse = cache_lse + (size_t)slot * blk + (size_t)bh * g.Lmax;
         }
         ++fpos;
       } else if (code == DITANGO_PLAN_REUSE) {
-        s.O = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * D;
+        s.O = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * ROWB;
         s.lse = cache_lse + (size_t)slot * blk + (size_t)bh * g.Lmax;
       } else {
         continue;  // active pair the plan skipped: contributes nothing
@@ -138,78 +206,71 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const float *__res
   const int b = bh / g.H, h = bh - (bh / g.H) * g.H;
   const int rend = (r0 + kRowsPerBlock < Li) ? r0 + kRowsPerBlock : Li;
 
-  // Two rows per warp iteration; every load of a row (its states' lse and the
-  // first kBatch O vectors) is issued before any of it is used.
-  for (int r = r0 + 2 * warp; r < rend; r += 2 * kWarps) {
-    const bool has_b = (r + 1) < rend;
-    float la0 = -INFINITY, la1 = -INFINITY, lb0 = -INFINITY, lb1 = -INFINITY;
-    if (lane < nact) {
-      la0 = __ldg(src[lane].lse + r);
-      if (has_b) lb0 = __ldg(src[lane].lse + r + 1);
-    }
-    if (lane + 32 < nact) {
-      la1 = __ldg(src[lane + 32].lse + r);
-      if (has_b) lb1 = __ldg(src[lane + 32].lse + r + 1);
+  // R rows per warp iteration (2 for fp32 states, 4 for bf16 states, so both
+  // keep the same bytes in flight); every load of a row -- its states' lse
+  // and the first kBatch O vectors -- is issued before any of it is used.
+  constexpr int R = SB ? 4 : 2;
+  for (int r = r0 + R * warp; r < rend; r += R * kWarps) {
+    float l0[R], l1[R];
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      const bool ok = (r + q) < rend;
+      l0[q] = (ok && lane < nact) ? __ldg(src[lane].lse + r + q) : -INFINITY;
+      l1[q] = (ok && lane + 32 < nact) ? __ldg(src[lane + 32].lse + r + q) : -INFINITY;
     }
     const bool act = lane < G;
-    float4 va[kBatch], vb[kBatch];
+    typename Raw4<SB>::T v[R][kBatch];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      va[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      vb[u] = va[u];
-      if (act && u < nact) {
-        va[u] = __ldg(reinterpret_cast<const float4 *>(src[u].O + (size_t)r * D) + lane);
-        if (has_b) vb[u] = __ldg(reinterpret_cast<const float4 *>(src[u].O + (size_t)(r + 1) * D) + lane);
+    for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+      for (int q = 0; q < R; ++q) {
+        v[q][u] = zero_raw4<SB>();
+        if (act && u < nact && (r + q) < rend)
+          v[q][u] = load_raw4<SB>(src[u].O + (size_t)(r + q) * ROWB + lane * 4 * ES);
       }
-    }
-    float wa0, wa1, wb0, wb1, La, Lb;
-    lse_weights(la0, la1, wa0, wa1, La);
-    lse_weights(lb0, lb1, wb0, wb1, Lb);
-    float4 acca = make_float4(0.f, 0.f, 0.f, 0.f), accb = acca;
+    float w0[R], w1[R], L[R];
+#pragma unroll
+    for (int q = 0; q < R; ++q) lse_weights(l0[q], l1[q], w0[q], w1[q], L[q]);
+    float4 acc[R];
+#pragma unroll
+    for (int q = 0; q < R; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int a0 = 0; a0 < nact; a0 += kBatch) {
       if (a0 > 0) {
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-          const int a = a0 + u;
-          if (act && a < nact) {
-            va[u] = __ldg(reinterpret_cast<const float4 *>(src[a].O + (size_t)r * D) + lane);
-            if (has_b) vb[u] = __ldg(reinterpret_cast<const float4 *>(src[a].O + (size_t)(r + 1) * D) + lane);
-          }
-        }
+        for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+          for (int q = 0; q < R; ++q)
+            if (act && a0 + u < nact && (r + q) < rend)
+              v[q][u] = load_raw4<SB>(src[a0 + u].O + (size_t)(r + q) * ROWB + lane * 4 * ES);
       }
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         const int a = a0 + u;
-        const float wa = __shfl_sync(0xffffffffu, (a < 32) ? wa0 : wa1, a & 31);
-        const float wb = __shfl_sync(0xffffffffu, (a < 32) ? wb0 : wb1, a & 31);
-        if (a < nact) {
-          fma4(acca, wa, va[u]);
-          fma4(accb, wb, vb[u]);
-          if (act && src[a].wbO) {
-            reinterpret_cast<float4 *>(src[a].wbO + (size_t)r * D)[lane] = va[u];
-            if (has_b) reinterpret_cast<float4 *>(src[a].wbO + (size_t)(r + 1) * D)[lane] = vb[u];
+#pragma unroll
+        for (int q = 0; q < R; ++q) {
+          const float wq = __shfl_sync(0xffffffffu, (a < 32) ? w0[q] : w1[q], a & 31);
+          if (a < nact) {
+            fma4(acc[q], wq, widen4<SB>(v[q][u]));
+            if (act && src[a].wbO && (r + q) < rend)
+              store_raw4<SB>(src[a].wbO + (size_t)(r + q) * ROWB + lane * 4 * ES, v[q][u]);
           }
         }
       }
     }
     // write back the lse of fresh states
-    if (lane < nact && src[lane].wblse) {
-      src[lane].wblse[r] = la0;
-      if (has_b) src[lane].wblse[r + 1] = lb0;
-    }
-    if (lane + 32 < nact && src[lane + 32].wblse) {
-      src[lane + 32].wblse[r] = la1;
-      if (has_b) src[lane + 32].wblse[r + 1] = lb1;
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      if ((r + q) >= rend) continue;
+      if (lane < nact && src[lane].wblse) src[lane].wblse[r + q] = l0[q];
+      if (lane + 32 < nact && src[lane + 32].wblse) src[lane + 32].wblse[r + q] = l1[q];
     }
     const int n = g.part_off[i] + r;
     const size_t obase = (size_t)b * osb + (size_t)h * osh + lane * 4;
-    if (act) {
-      store_out(out, out_is_fp32, obase + (size_t)n * osn, acca);
-      if (has_b) store_out(out, out_is_fp32, obase + (size_t)(n + 1) * osn, accb);
-    }
-    if (out_lse && lane == 0) {
-      out_lse[((size_t)b * g.H + h) * g.N + n] = La;
-      if (has_b) out_lse[((size_t)b * g.H + h) * g.N + n + 1] = Lb;
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      if ((r + q) >= rend) continue;
+      if (act) store_out(out, out_is_fp32, obase + (size_t)(n + q) * osn, acc[q]);
+      if (out_lse && lane == 0) out_lse[((size_t)b * g.H + h) * g.N + n + q] = L[q];
     }
   }
 }
@@ -219,8 +280,8 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const float *__res
 // counts the fresh pairs before it (row-major) to find its fresh position.
 __global__ void __launch_bounds__(256)
 cache_update_kernel(DevGeom g, const signed char *__restrict__ plan,
-                    const float *__restrict__ part_O, const float *__restrict__ part_lse,
-                    float *cache_O, float *cache_lse, unsigned char *cache_valid, int D) {
+                    const char *__restrict__ part_O, const float *__restrict__ part_lse,
+                    char *cache_O, float *cache_lse, unsigned char *cache_valid, int row_bytes) {
   const int slot = blockIdx.y;
   int i = 0;
   while (i + 1 < g.P && g.row_start[i + 1] <= slot) ++i;
@@ -246,9 +307,9 @@ cache_update_kernel(DevGeom g, const signed char *__restrict__ plan,
   __syncthreads();
   const int f = s_fpos;
   const size_t blk = (size_t)g.BH * g.Lmax;
-  const float4 *s = reinterpret_cast<const float4 *>(part_O + (size_t)f * blk * D);
-  float4 *d = reinterpret_cast<float4 *>(cache_O + (size_t)slot * blk * D);
-  const size_t n4 = blk * D / 4;
+  const float4 *s = reinterpret_cast<const float4 *>(part_O + (size_t)f * blk * row_bytes);
+  float4 *d = reinterpret_cast<float4 *>(cache_O + (size_t)slot * blk * row_bytes);
+  const size_t n4 = blk * row_bytes / 16;
   for (size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x; t < n4;
        t += (size_t)gridDim.x * blockDim.x)
     d[t] = __ldg(s + t);
@@ -262,18 +323,24 @@ cache_update_kernel(DevGeom g, const signed char *__restrict__ plan,
 
 }  // namespace merge
 
-cudaError_t launch_merge(const DevGeom &g, const signed char *plan, const float *part_O,
-                         const float *part_lse, float *cache_O, float *cache_lse,
-                         unsigned char *cache_valid, int writeback, void *out, int out_is_fp32,
+cudaError_t launch_merge(const DevGeom &g, const signed char *plan, const void *part_O,
+                         const float *part_lse, void *cache_O, float *cache_lse,
+                         unsigned char *cache_valid, int writeback, int state_bf16, void *out,
+                         int out_is_fp32,
                          long long osb, long long osh, long long osn, float *out_lse,
                          cudaStream_t stream) {
   dim3 grid((g.Lmax + merge::kRowsPerBlock - 1) / merge::kRowsPerBlock, g.P, g.BH);
   switch (g.d) {
 #define DITANGO_MERGE(DD)                                                                        \
   case DD:                                                                                       \
-    merge::merge_kernel<DD><<<grid, merge::kThreads, 0, stream>>>(                               \
-        g, plan, part_O, part_lse, cache_O, cache_lse, cache_valid, writeback, out, out_is_fp32, \
-        osb, osh, osn, out_lse);                                                                 \
+    if (state_bf16)                                                                              \
+      merge::merge_kernel<DD, true><<<grid, merge::kThreads, 0, stream>>>(                       \
+          g, plan, static_cast<const char *>(part_O), part_lse, static_cast<char *>(cache_O),   \
+          cache_lse, cache_valid, writeback, out, out_is_fp32, osb, osh, osn, out_lse);          \
+    else                                                                                         \
+      merge::merge_kernel<DD, false><<<grid, merge::kThreads, 0, stream>>>(                      \
+          g, plan, static_cast<const char *>(part_O), part_lse, static_cast<char *>(cache_O),   \
+          cache_lse, cache_valid, writeback, out, out_is_fp32, osb, osh, osn, out_lse);          \
     return cudaGetLastError();
     DITANGO_MERGE(64)
     DITANGO_MERGE(96)
@@ -284,17 +351,20 @@ cudaError_t launch_merge(const DevGeom &g, const signed char *plan, const float 
   }
 }
 
-cudaError_t launch_cache_update(const DevGeom &g, const signed char *plan, const float *part_O, const float *part_lse, float *cache_O,
-                                float *cache_lse, unsigned char *cache_valid, int num_sms,
+cudaError_t launch_cache_update(const DevGeom &g, const signed char *plan, const void *part_O,
+                                const float *part_lse, void *cache_O, float *cache_lse,
+                                unsigned char *cache_valid, int state_bf16, int num_sms,
                                 cudaStream_t stream) {
   if (g.n_active == 0) return cudaSuccess;
-  const size_t n4 = (size_t)g.BH * g.Lmax * g.d / 4;
+  const int row_bytes = g.d * (state_bf16 ? 2 : 4);
+  const size_t n4 = (size_t)g.BH * g.Lmax * row_bytes / 16;
   int bx = (int)((n4 + 255) / 256);
   const int cap = (num_sms * 8 + g.n_active - 1) / g.n_active;
   if (bx > cap) bx = cap < 1 ? 1 : cap;
   dim3 grid(bx, g.n_active);
-  merge::cache_update_kernel<<<grid, 256, 0, stream>>>(g, plan, part_O, part_lse, cache_O,
-                                                        cache_lse, cache_valid, g.d);
+  merge::cache_update_kernel<<<grid, 256, 0, stream>>>(
+      g, plan, static_cast<const char *>(part_O), part_lse, static_cast<char *>(cache_O), cache_lse,
+      cache_valid, row_bytes);
   return cudaGetLastError();
 }
 

@@ -29,9 +29,10 @@ def sample_rows(w, i, n=24):
     return lo + np.unique(np.clip(picks, 0, L - 1))
 
 
-def run_workload(w, out_dtype=torch.float32):
+def run_workload(w, out_dtype=torch.float32, state_bf16=False):
     Q, K, V = G.upload(w)
-    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask())
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask(),
+                                 state_bf16=state_bf16)
     if w.reuses:
         Kp, Vp = G.upload_prev(w)
         pa.plan_step(anchor=True)
@@ -45,10 +46,13 @@ def run_workload(w, out_dtype=torch.float32):
     return pa, out, out_lse
 
 
-@pytest.mark.parametrize("w", [configs.FRAME_TILE, configs.DITANGO_REUSE, configs.LONG_VIDEO,
-                               configs.DENSE], ids=lambda w: w.name)
-def test_full_size_sampled_rows(w):
-    pa, out, out_lse = run_workload(w)
+@pytest.mark.parametrize("w,sb", [(configs.FRAME_TILE, False), (configs.DITANGO_REUSE, False),
+                                  (configs.LONG_VIDEO, False), (configs.DENSE, False),
+                                  (configs.DITANGO_REUSE, True), (configs.LONG_VIDEO, True)],
+                         ids=["frame_tile", "reuse_p32", "long_video", "dense",
+                              "reuse_p32_bf16_cache", "long_video_bf16_cache"])
+def test_full_size_sampled_rows(w, sb):
+    pa, out, out_lse = run_workload(w, state_bf16=sb)
     plan = pa.plan.cpu().numpy().reshape(w.P, w.P)
     G.check_plan_valid(w, plan)
     counts = pa.counts.cpu().numpy()

@@ -31,19 +31,21 @@ def geom_of(w, part_off=None):
     return dt.Geometry(w.B, w.H, w.N, w.d, part_off or w.part_off(), w.frame_off(), w.frame_mask())
 
 
-def all_pairs_partial(geom, Q, K, V, n, Lmax, d, BH):
+def all_pairs_partial(geom, Q, K, V, n, Lmax, d, BH, state_bf16=False):
     P = geom.P
     plan = torch.zeros(P * P, dtype=torch.int8, device="cuda")
     fresh = torch.full((max(n, 1),), -1, dtype=torch.int32, device="cuda")
     counts = torch.zeros(2, dtype=torch.int32, device="cuda")
     dt.ditango_plan(geom, None, None, 0, 1.0, True, plan, fresh, counts)
-    O = torch.full((n, BH, Lmax, d), float("nan"), dtype=torch.float32, device="cuda")
+    O = torch.full((n, BH, Lmax, d), float("nan"), dtype=torch.bfloat16 if state_bf16 else torch.float32,
+                   device="cuda")
     lse = torch.full((n, BH, Lmax), float("nan"), dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    dt.ditango_attn_partial(geom, Q, K, V, fresh, counts, 0.0, O, lse, 0, None, st)
+    dt.ditango_attn_partial(geom, Q, K, V, fresh, counts, 0.0, O, lse, 0, None, st, state_bf16=state_bf16)
     torch.cuda.synchronize()
     assert st.item() == 0
-    return plan.cpu().numpy(), fresh.cpu().numpy(), counts.cpu().numpy(), O.cpu().numpy(), lse.cpu().numpy()
+    return (plan.cpu().numpy(), fresh.cpu().numpy(), counts.cpu().numpy(), O.float().cpu().numpy(),
+            lse.cpu().numpy())
 
 
 def test_bounded_wait_reports_timeout_and_context_survives():
@@ -55,15 +57,18 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert float(x.sum()) == 28.0
 
 
-@pytest.mark.parametrize("d,part_off,frames", [
-    (64, None, None),                                  # the tiny workload's geometry
-    (64, [0, 100, 130, 300, 555, 1000], None),         # ragged: short and multi-tile partitions
-    (96, [0, 100, 130, 300, 555, 1000], None),
-    (128, [0, 100, 130, 300, 555, 1000], None),
-    (96, [0, 130, 300, 555, 1000], ([0, 300, 1000], [[1, 0], [1, 1]])),  # frame mask
-    (128, [0, 257, 512, 640, 1024], None),             # 256-row unit boundaries +-1
+@pytest.mark.parametrize("d,part_off,frames,sb", [
+    (64, None, None, False),                           # the tiny workload's geometry
+    (64, [0, 100, 130, 300, 555, 1000], None, False),  # ragged: short and multi-tile partitions
+    (96, [0, 100, 130, 300, 555, 1000], None, False),
+    (128, [0, 100, 130, 300, 555, 1000], None, False),
+    (96, [0, 130, 300, 555, 1000], ([0, 300, 1000], [[1, 0], [1, 1]]), False),  # frame mask
+    (128, [0, 257, 512, 640, 1024], None, False),      # 256-row unit boundaries +-1
+    (64, [0, 100, 130, 300, 555, 1000], None, True),   # bf16 states (compressed cache)
+    (96, [0, 130, 300, 555, 1000], ([0, 300, 1000], [[1, 0], [1, 1]]), True),
+    (128, [0, 257, 512, 640, 1024], None, True),
 ])
-def test_partial_states_every_row(d, part_off, frames):
+def test_partial_states_every_row(d, part_off, frames, sb):
     if part_off is None:
         w = configs.TINY
         part_off = w.part_off()
@@ -75,7 +80,7 @@ def test_partial_states_every_row(d, part_off, frames):
     A = OM.pair_mask(part_off, fo, fm)
     n, Lmax = int(A.sum()), max(np.diff(part_off))
     Q, K, V = G.upload(w)
-    plan, fresh, counts, O, lse = all_pairs_partial(geom, Q, K, V, n, Lmax, w.d, w.BH)
+    plan, fresh, counts, O, lse = all_pairs_partial(geom, Q, K, V, n, Lmax, w.d, w.BH, state_bf16=sb)
     P = len(part_off) - 1
     assert counts.tolist() == [n, 0]
     assert (fresh[:n] == np.nonzero(A.ravel())[0]).all()
@@ -109,11 +114,12 @@ def build_cache(pa, Q, Kp, Vp):
     pa.partial(Q, Kp, Vp)
 
 
-def test_tiny_reuse_step_plan_and_output():
+@pytest.mark.parametrize("sb", [False, True], ids=["fp32_cache", "bf16_cache"])
+def test_tiny_reuse_step_plan_and_output(sb):
     w = configs.TINY
     Q, K, V = G.upload(w)
     Kp, Vp = G.upload_prev(w)
-    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), state_bf16=sb)
     build_cache(pa, Q, Kp, Vp)
     out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
     out_lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
@@ -141,21 +147,22 @@ def test_tiny_reuse_step_plan_and_output():
             G.assert_close(ol[b, h, rows], lo, f"out lse bh {bh} part {i}")
 
 
-def test_tiny_compact_partials_merge_writeback_and_cache_update_agree():
+@pytest.mark.parametrize("sb", [False, True], ids=["fp32_states", "bf16_states"])
+def test_tiny_compact_partials_merge_writeback_and_cache_update_agree(sb):
     """Three routes to the same step must give bit-identical states and outputs:
     in-place partials, compact partials + merge write-back, compact partials +
     cache update + merge from the cache."""
     w = configs.TINY
     Q, K, V = G.upload(w)
     Kp, Vp = G.upload_prev(w)
-    ref = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    ref = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), state_bf16=sb)
     build_cache(ref, Q, Kp, Vp)
     cache0_O, cache0_l = ref.state_O.clone(), ref.state_lse.clone()
     out_ref = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
     ref.step(Q, K, V, out_ref, band_k=w.band_k, budget=w.budget)
     g = ref.geom
     nf = 12
-    part_O = torch.empty((nf, w.BH, w.Lp, w.d), dtype=torch.float32, device="cuda")
+    part_O = torch.empty((nf, w.BH, w.Lp, w.d), dtype=torch.bfloat16 if sb else torch.float32, device="cuda")
     part_l = torch.empty((nf, w.BH, w.Lp), dtype=torch.float32, device="cuda")
     for route in ("writeback", "cache_update"):
         cO, cl = cache0_O.clone(), cache0_l.clone()
@@ -165,13 +172,14 @@ def test_tiny_compact_partials_merge_writeback_and_cache_update_agree():
         counts = torch.zeros(2, dtype=torch.int32, device="cuda")
         ws = torch.empty(ref.ws_bytes, dtype=torch.uint8, device="cuda")
         dt.ditango_plan(g, cl, valid, w.band_k, w.budget, 0, plan, fresh, counts, None, ws, ref.ws_bytes)
-        dt.ditango_attn_partial(g, Q, K, V, fresh, counts, 0.0, part_O, part_l, 0, None, None)
+        dt.ditango_attn_partial(g, Q, K, V, fresh, counts, 0.0, part_O, part_l, 0, None, None,
+                                state_bf16=sb)
         out = torch.empty_like(out_ref)
         if route == "writeback":
-            dt.ditango_merge(g, plan, part_O, part_l, cO, cl, valid, 1, out, 1)
+            dt.ditango_merge(g, plan, part_O, part_l, cO, cl, valid, 1, out, 1, state_bf16=sb)
         else:
-            dt.ditango_cache_update(g, plan, part_O, part_l, cO, cl, valid)
-            dt.ditango_merge(g, plan, None, None, cO, cl, valid, 0, out, 1)
+            dt.ditango_cache_update(g, plan, part_O, part_l, cO, cl, valid, state_bf16=sb)
+            dt.ditango_merge(g, plan, None, None, cO, cl, valid, 0, out, 1, state_bf16=sb)
         torch.cuda.synchronize()
         assert torch.equal(plan, ref.plan)
         assert torch.equal(out, out_ref), route
