@@ -12,21 +12,24 @@ Sources (pages, by title and section):
     Attention State Reuse", technical summary ("Riepilogo Tecnico"):
       - Metodologia (spatial locality of attention contributions);
       - 1. Anchor-Guided Selection Planner (error model with partition
-        importance w, anchor steps, group strategy);
+        importance w, anchor steps, group strategy "Strategia per Gruppi");
       - 2. State-Centric Parallel Runtime, "Composizione dello Stato"
         (attention state = output + log-sum-exp, composed associatively and
-        commutatively; cached instead of raw KV).
+        commutatively; cached instead of raw KV), "Calcolo dello Stato di
+        Gruppo" and "Composizione Dinamica dei Gruppi" (group states; cached
+        states merged recursively into coarser groups).
   * "Efficient-vDiT: Efficient Video Diffusion Transformers With Attention
     Tile", abstract (tile-style repeating pattern, sparse 3D attention linear
     in the number of frames).
 
 Parity status per function:
   attention.partial_state, attention.merge_states, attention.dense_attention,
-  masks.*, plan.select, plan.mass_scores, step.*  -- pinned (tests/test_oracle_*.py)
+  masks.*, plan.select, plan.mass_scores, step.*, groups.*
+  -- pinned (tests/test_oracle_*.py)
   The quality of reuse (how far a reuse step drifts from an all-fresh step)
   -- parity unpinned: the pages print no error values; it is reported only.
 """
 from .attention import partial_state, merge_states, dense_attention  # noqa: F401
 from .masks import pair_mask, slot_table, token_allowed, frame_of  # noqa: F401
 from .plan import mass_scores, select, budget_target, PLAN_SKIP, PLAN_FRESH, PLAN_REUSE  # noqa: F401
-from . import step  # noqa: F401
+from . import step, groups  # noqa: F401

@@ -33,19 +33,21 @@ PLAN_SKIP, PLAN_FRESH, PLAN_REUSE = 0, 1, 2
 
 
 def mass_scores(cache_lse, A, part_off, valid=None):
-    """w [P, P] (fp64) from cached log-sum-exps.
+    """w [P, C] (fp64) from cached log-sum-exps.
 
+    A: [P, C] active mask, one row per query partition and one column per KV
+    partition (C = P) or per KV group (see oracle.groups).
     cache_lse: [slots, BH, Lmax] array indexed by slot (row-major rank of the
-    active pair); row r of pair (i, j) is cache_lse[slot(i,j), :, r] for
-    r < L_i.  Inactive pairs get w = 0.  valid: optional bool [slots]; a slot
-    that was never written holds no state and therefore no mass.
+    active entry); row r of entry (i, j) is cache_lse[slot(i,j), :, r] for
+    r < L_i.  Inactive entries get w = 0.  valid: optional bool [slots]; a
+    slot that was never written holds no state and therefore no mass.
     """
     A = np.asarray(A, dtype=bool)
     P = A.shape[0]
     lse_all = np.asarray(cache_lse)
     if valid is not None:
         lse_all = np.where(np.asarray(valid, dtype=bool)[:, None, None], lse_all, -np.inf)
-    w = np.zeros((P, P), dtype=np.float64)
+    w = np.zeros(A.shape, dtype=np.float64)
     slot = 0
     for i in range(P):
         js = np.nonzero(A[i])[0]
@@ -69,20 +71,24 @@ def budget_target(n_band, n_active, budget):
     return max(int(n_band), int(math.floor(float(budget) * int(n_active) + 1e-9)))
 
 
-def select(w, A, band_k, budget, anchor=False, valid=None, rank_dtype=np.float32):
-    """Plan int8 [P, P] in {0 skip, 1 fresh, 2 reuse} and the fresh list.
+def select(w, A, band_k, budget, anchor=False, valid=None, rank_dtype=np.float32, band=None):
+    """Plan int8 [P, C] in {0 skip, 1 fresh, 2 reuse} and the fresh list.
 
-    The fresh list holds the linear pair indices i * P + j of the fresh pairs
-    in row-major order.
+    The fresh list holds the linear indices i * C + j of the fresh entries
+    in row-major order.  The band is |i - j| <= band_k on a square A; a
+    caller with KV groups passes its own band mask (oracle.groups.unit_band).
     """
     A = np.asarray(A, dtype=bool)
-    P = A.shape[0]
-    ii, jj = np.meshgrid(np.arange(P), np.arange(P), indexing="ij")
-    fresh = np.zeros((P, P), dtype=bool)
+    P, C = A.shape
+    ii, jj = np.meshgrid(np.arange(P), np.arange(C), indexing="ij")
+    fresh = np.zeros((P, C), dtype=bool)
     if anchor:
         fresh[:] = A
     else:
-        band = A & (np.abs(ii - jj) <= band_k)
+        if band is None:
+            band = A & (np.abs(ii - jj) <= band_k)
+        else:
+            band = A & np.asarray(band, dtype=bool)
         fresh |= band
         if valid is not None:
             fresh |= A & ~np.asarray(valid, dtype=bool)

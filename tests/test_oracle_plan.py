@@ -15,7 +15,7 @@ import numpy as np
 import pytest
 
 import oracle
-from oracle import masks
+from oracle import groups, masks
 from oracle.plan import PLAN_FRESH, PLAN_REUSE, PLAN_SKIP, budget_target, mass_scores, select
 from workloads import configs
 
@@ -31,16 +31,20 @@ def test_golden_counts(w):
     g = GOLD[w.name]
     po, fo, fm = geometry(w)
     A = masks.pair_mask(po, fo, fm)
-    assert int(A.sum()) == g["active"]
     P = w.P
+    ii, jj = np.indices((P, P))
+    band = A & (np.abs(ii - jj) <= w.band_k)
+    if w.grouped:
+        A = groups.unit_mask(A, w.group_off())
+        band = groups.unit_band(masks.pair_mask(po, fo, fm), w.group_off(), w.band_k)
+        assert A.shape == (P, g["G"])
+    assert int(A.sum()) == g["active"]
     rng = np.random.default_rng(0)
-    wts = rng.random((P, P))
-    plan, fl = select(wts, A, w.band_k, w.budget, anchor=w.anchor)
+    wts = rng.random(A.shape)
+    plan, fl = select(wts, A, w.band_k, w.budget, anchor=w.anchor, band=band if w.grouped else None)
     assert int((plan == PLAN_FRESH).sum()) == g["fresh"] == len(fl)
     assert int((plan == PLAN_REUSE).sum()) == g["reuse"]
     if g["band"] is not None:
-        ii, jj = np.indices((P, P))
-        band = A & (np.abs(ii - jj) <= w.band_k)
         assert int(band.sum()) == g["band"]
         assert budget_target(band.sum(), A.sum(), w.budget) == g["target"]
 

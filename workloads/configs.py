@@ -29,6 +29,7 @@ class Workload:
     anchor: bool = True         # all active pairs fresh (no reuse)
     drift_sigma: float = 0.0    # previous-step K/V = K/V + sigma * N(0, 1)
     frame_component: float = 0.0  # per-frame shared component amplitude
+    group_size: int = 0         # partitions per KV group (0: one group per partition)
     seed: int = 0
     drift_seed: int = 0
     description: str = ""
@@ -57,6 +58,20 @@ class Workload:
         F = self.F
         return [[1 if (abs(f - g) <= 1 or g == 0) else 0 for g in range(F)]
                 for f in range(F)]
+
+    @property
+    def G(self) -> int:
+        """KV groups (columns of the plan)."""
+        return len(self.group_off()) - 1
+
+    def group_off(self) -> List[int]:
+        """Partition offsets of the KV groups: runs of group_size adjacent partitions."""
+        s = self.group_size if self.group_size > 0 else 1
+        return list(range(0, self.P, s)) + [self.P]
+
+    @property
+    def grouped(self) -> bool:
+        return self.group_size > 1
 
     @property
     def reuses(self) -> bool:
@@ -91,7 +106,14 @@ DENSE = Workload(
     anchor=True, seed=5,
     description="all-fresh dense case, 16-way merge, equals unpartitioned attention")
 
-ALL = [TINY, FRAME_TILE, DITANGO_REUSE, LONG_VIDEO, DENSE]
+DITANGO_GROUPS = Workload(
+    name="ditango_groups_p32_g4", B=1, H=40, N=76800, d=128, P=32,
+    band_k=2, budget=0.25, anchor=False, drift_sigma=0.03, group_size=4,
+    seed=3, drift_seed=103,
+    description="the 32-partition reuse case with decisions and cached states per group of "
+                "4 adjacent KV partitions (8 groups): a 4x smaller cache")
+
+ALL = [TINY, FRAME_TILE, DITANGO_REUSE, LONG_VIDEO, DENSE, DITANGO_GROUPS]
 BY_NAME = {w.name: w for w in ALL}
 
 
