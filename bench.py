@@ -44,9 +44,20 @@ def pair_mask(w):
 
 
 def effective_flops(w, fresh_mask):
+    """4 d B H sum over fresh active pairs of L_i L_j (fresh_mask: [P, P])."""
     po = np.array(w.part_off())
     L = np.diff(po)
     return float(4.0 * w.d * w.BH * (np.outer(L, L) * fresh_mask).sum())
+
+
+def fresh_pairs_of_units(w, plan_units, A_pairs):
+    """[P, P] fresh active pairs of a plan over KV groups: pair (i, j) is
+    computed when it is active and the unit (i, group of j) is fresh."""
+    go = w.group_off()
+    col = np.zeros(w.P, dtype=np.int64)
+    for c in range(len(go) - 1):
+        col[go[c]:go[c + 1]] = c
+    return A_pairs & (plan_units[:, col] == 1)
 
 
 def merge_bytes(w, A, fresh_mask, out_bytes_per_elem=2, writeback=False, state_o_bytes=4):
@@ -172,8 +183,9 @@ def run_ours(args, w, rank, world, local_rank):
 
     hq, hk, hv = (up(inputs.full(w, t)) for t in "qkv")
     Q, K, V = (x.to(dev) for x in (hq, hk, hv))
+    group_off = w.group_off() if w.grouped else None
     pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask(),
-                                 device=dev, state_bf16=args.state_bf16)
+                                 device=dev, state_bf16=args.state_bf16, group_off=group_off)
     if w.reuses:
         Kp = up(inputs.full(w, "k", prev=True)).to(dev)
         Vp = up(inputs.full(w, "v", prev=True)).to(dev)
@@ -189,10 +201,10 @@ def run_ours(args, w, rank, world, local_rank):
     with torch.cuda.stream(stream):
         pa.step(Q, K, V, out, out_lse, stream=stream, **kw)
     stream.synchronize()
-    plan = pa.plan.cpu().numpy().reshape(w.P, w.P)
+    plan = pa.plan.cpu().numpy().reshape(w.P, pa.G)
     A = plan != 0
     fresh = plan == 1
-    flops = effective_flops(w, fresh)
+    flops = effective_flops(w, fresh_pairs_of_units(w, plan, pair_mask(w)))
     mbytes = merge_bytes(w, A, fresh, state_o_bytes=2 if args.state_bf16 else 4)
     launches_per_step = (1 if w.anchor else 2) + 1 + 1
 
@@ -298,6 +310,9 @@ def run_ours(args, w, rank, world, local_rank):
 
     ms_step = ms / args.steps
     peaks, peak_src = load_peaks()
+    compose = None
+    if w.grouped:
+        compose = measure_compose(w, pa, Q, K, V, dev, stream, args, peaks)
     tflops_part = flops / (part_ms * 1e-3) / 1e12
     peak_t = float(peaks.get("bf16_tflops"))          # burst figure: the conservative denominator
     peak_ts = float(peaks.get("bf16_tflops_sustained", peak_t))
@@ -318,11 +333,12 @@ def run_ours(args, w, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16, shaped like the pages' workloads)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "P": w.P,
-                   "frames": w.F, "fresh_pairs": int(fresh.sum()), "active_pairs": int(A.sum()),
+                   "frames": w.F, "kv_groups": int(pa.G), "fresh_units": int(fresh.sum()),
+                   "active_units": int(A.sum()),
                    "state_format": "bf16 O + fp32 lse" if args.state_bf16 else "fp32 O + fp32 lse",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (Q/K/V %.0f MB, states %.0f MB)" % (
-                       h2d / 1e6, pa.state_O.numel() * 4 / 1e6)},
+                       h2d / 1e6, pa.state_O.numel() * pa.state_O.element_size() / 1e6)},
         "roofline": {"bound": "tensor", "kernel": "attn_partial", "achieved": round(tflops_part, 2),
                      "peak": peak_t, "unit": "TFLOP/s", "frac": round(tflops_part / peak_t, 4),
                      "peak_source": peak_src, "traffic": traffic,
@@ -341,17 +357,64 @@ def run_ours(args, w, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if compose is not None:
+        res["compose"] = compose
     return res
+
+
+def measure_compose(w, pa, Q, K, V, dev, stream, args, peaks):
+    """Dynamic group composition: a cache of one state per (query partition,
+    KV partition) merged into this workload's KV groups, no recomputation.
+    The pair cache is built by an anchor step on the current K/V; the
+    composition is timed alone (CUDA events, after warm-up).  Algorithmic
+    bytes: every pair state read once, every group state written once."""
+    import torch
+    import sparse_state_reuse_b200 as dt
+    fine = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask(),
+                                   device=dev, state_bf16=args.state_bf16)
+    with torch.cuda.stream(stream):
+        fine.plan_step(anchor=True, stream=stream)
+        fine.partial(Q, K, V, stream=stream)
+    stream.synchronize()
+    row = w.d * (2 if args.state_bf16 else 4) + 4
+    nbytes = float((fine.n_slots + pa.n_slots) * w.BH * w.Lp * row)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    reps = 5
+    for _ in range(2):
+        dt.ditango_cache_compose(fine.geom, pa.geom, fine.state_O, fine.state_lse, fine.valid,
+                                 pa.state_O, pa.state_lse, pa.valid, args.state_bf16, stream)
+    a, b = ev(), ev()
+    a.record(stream)
+    for _ in range(reps):
+        dt.ditango_cache_compose(fine.geom, pa.geom, fine.state_O, fine.state_lse, fine.valid,
+                                 pa.state_O, pa.state_lse, pa.valid, args.state_bf16, stream)
+    b.record(stream)
+    stream.synchronize()
+    ms = a.elapsed_time(b) / reps
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out = {"from_slots": int(fine.n_slots), "to_slots": int(pa.n_slots),
+           "cache_bytes_before": int(fine.state_O.numel() * fine.state_O.element_size()
+                                     + fine.state_lse.numel() * 4),
+           "cache_bytes_after": int(pa.state_O.numel() * pa.state_O.element_size()
+                                    + pa.state_lse.numel() * 4),
+           "ms": round(ms, 4), "bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s",
+           "peak": float(peaks.get("hbm_gbs")), "frac": round(gbs / float(peaks.get("hbm_gbs")), 4),
+           "algorithmic_bytes_per_launch": nbytes, "traffic": recorded_traffic("merge.cu", w.name + ":compose")}
+    del fine
+    torch.cuda.empty_cache()
+    return out
 
 
 # ------------------------------------------------------------------ CPU oracle
 def oracle_sample(w, rng_seed, rows_per_sample, deadline_s):
     """Time the fp64 oracle on seeded (b, h, partition, row-block) samples of
     the workload until deadline_s of CPU work; returns (flops, seconds, desc)."""
-    from oracle import masks as OM, step as OS
+    from oracle import groups as OG, masks as OM, step as OS
     from oracle.plan import PLAN_FRESH
     A = OM.pair_mask(w.part_off(), w.frame_off(), w.frame_mask())
     plan = np.where(A, PLAN_FRESH, 0).astype(np.int8)  # the fresh work of the step
+    if w.grouped:
+        plan = np.where(OG.unit_mask(A, w.group_off()), PLAN_FRESH, 0).astype(np.int8)
     rng = np.random.default_rng(rng_seed)
     po = w.part_off()
     flops, secs, n = 0.0, 0.0, 0
@@ -366,7 +429,11 @@ def oracle_sample(w, rng_seed, rows_per_sample, deadline_s):
         k = inputs.slab_f64(w, "k", b, h)
         v = inputs.slab_f64(w, "v", b, h)
         t0 = time.perf_counter()
-        OS.step_rows(q, k, v, k, v, plan, po, i, rows, w.frame_off(), w.frame_mask())
+        if w.grouped:
+            OG.step_rows_units(q, k, v, k, v, plan, po, w.group_off(), i, rows, w.frame_off(),
+                               w.frame_mask())
+        else:
+            OS.step_rows(q, k, v, k, v, plan, po, i, rows, w.frame_off(), w.frame_mask())
         secs += time.perf_counter() - t0
         keys = sum(po[j + 1] - po[j] for j in range(w.P) if A[i, j])
         flops += 4.0 * w.d * rows.size * keys

@@ -10,10 +10,14 @@
  *        near partitions contribute most (spatial locality).
  *      1. Anchor-Guided Selection Planner: per pair, recompute ("fresh") or
  *        reuse the previous denoising step's attention state, guided by the
- *        partition's importance w; anchor steps recompute everything.
+ *        partition's importance w; anchor steps recompute everything;
+ *        "Strategia per Gruppi": decisions per group of adjacent partitions.
  *      2. State-Centric Parallel Runtime, "Composizione dello Stato": an
  *        attention state is (output, log-sum-exp); states are cached instead
- *        of raw K/V and compose associatively and commutatively.
+ *        of raw K/V and compose associatively and commutatively;
+ *        "Calcolo dello Stato di Gruppo": one state per group;
+ *        "Composizione Dinamica dei Gruppi": cached states are merged
+ *        recursively into coarser groups to shrink the cache.
  *  - "Efficient-vDiT: Efficient Video Diffusion Transformers With Attention
  *    Tile", abstract: a frame-tile sparse mask whose cost grows linearly
  *    with the number of frames.
@@ -30,16 +34,23 @@
  *    Device-side failures (a pipeline wait that exceeded its time limit) are
  *    written as a status code into `dev_status` where a call takes one.
  *  - Token order is frame-major; partitions are contiguous token ranges.
+ *  - Units: the KV side may be grouped into G runs of adjacent partitions
+ *    (ditango_geom.G, group_off).  The unit of planning and of storage is
+ *    (query partition i, KV group c); its state is attention of partition
+ *    i's rows against every allowed key of the group's partitions.  Without
+ *    groups (G = 0) each partition is its own group, G = P and a unit is the
+ *    pair (i, j).  A unit is active when some pair (i, j), j in c, is.
  *  - State layout ("state buffer"): O is [n_idx][B*H][Lmax][d], float32 or
  *    (state_bf16 = 1, a compressed cache) bfloat16 bit patterns, and lse is
  *    float32 [n_idx][B*H][Lmax], where Lmax = max partition length
  *    (ditango_state_rows) and the leading index is either the slot of an
- *    active pair (row-major rank of the active pairs, see ditango_slot_table)
- *    or the position of a pair in the fresh list.  Row r of pair (i, j)
+ *    active unit (row-major rank of the active units, see ditango_slot_table)
+ *    or the position of a unit in the fresh list.  Row r of unit (i, c)
  *    holds query token part_off[i] + r; rows r >= L_i are never written.
  *    O is normalised (sum_k softmax_k v_k) and lse is the natural
  *    log-sum-exp of the scaled logits.
- *  - Plan codes: 0 skip (masked pair), 1 fresh, 2 reuse.
+ *  - Plan: int8 [P * G], entry i * G + c; codes 0 skip (masked unit),
+ *    1 fresh, 2 reuse.
  */
 #ifndef DITANGO_H
 #define DITANGO_H
@@ -76,7 +87,11 @@ typedef void *ditango_stream; /* cudaStream_t */
  *   q/k/v_strides  element strides of the (b, h, n) dimensions of the bf16
  *            Q, K, V tensors; the d dimension is contiguous.  Strides times 2
  *            bytes must be multiples of 16 and the base pointers 16-byte
- *            aligned (TMA). */
+ *            aligned (TMA).
+ *   G        KV groups; 0 = one group per partition (group_off ignored).
+ *            Else 1 <= G <= P and group_off host int32 [G+1] holds partition
+ *            indices, group_off[0] = 0 < ... < group_off[G] = P: group c is
+ *            partitions group_off[c] .. group_off[c+1]-1. */
 typedef struct {
   int32_t B, H, N, d;
   int32_t P, F;
@@ -86,6 +101,8 @@ typedef struct {
   int64_t q_strides[3];
   int64_t k_strides[3];
   int64_t v_strides[3];
+  int32_t G;
+  const int32_t *group_off;
 } ditango_geom;
 
 /* Library version (major * 10000 + minor * 100 + patch). */
@@ -97,39 +114,41 @@ const char *ditango_status_string(int32_t status);
 /* Validate a geometry without launching anything. */
 ditango_status ditango_check_geom(const ditango_geom *g);
 
-/* Number of active pairs (= slots): pairs (i, j) whose tokens the frame mask
- * lets attend each other (all P*P when F = 0).  Returns -1 on a bad geometry. */
+/* Number of active units (= slots): units (i, c) with a pair (i, j), j in c,
+ * whose tokens the frame mask lets attend each other (all P*G when F = 0).
+ * Returns -1 on a bad geometry. */
 int64_t ditango_num_active(const ditango_geom *g);
 
 /* Lmax, rows per (index, b*h) block of a state buffer. -1 on a bad geometry. */
 int64_t ditango_state_rows(const ditango_geom *g);
 
-/* Host helper: slot_out host int32 [P*P] receives the slot of each pair,
- * -1 for masked pairs (row-major rank of the active pairs). */
+/* Host helper: slot_out host int32 [P*G] receives the slot of each unit,
+ * -1 for masked units (row-major rank of the active units). */
 ditango_status ditango_slot_table(const ditango_geom *g, int32_t *slot_out);
 
 /* Bytes of device scratch ditango_plan needs. */
 size_t ditango_plan_workspace_size(const ditango_geom *g);
 
-/* Plan: per pair, fresh or reuse (DiTango, 1. Anchor-Guided Selection
- * Planner; spatial locality from Metodologia).
+/* Plan: per unit, fresh or reuse (DiTango, 1. Anchor-Guided Selection
+ * Planner and its group strategy; spatial locality from Metodologia).
  *   cache_lse    dev float32 state-buffer lse indexed by slot (the previous
  *                step's cached states); may be NULL when anchor != 0.
  *   cache_valid  dev uint8 [slots] (nonzero = slot holds a state) or NULL
  *                (all valid).  An invalid slot is forced fresh and holds no
  *                mass.
- *   band_k       pairs with |i - j| <= band_k are always fresh.
- *   budget       fraction of active pairs to recompute: the fresh count is
- *                max(|band|, floor(budget * active + 1e-9)); the pairs added
+ *   band_k       the band: unit (i, c) is always fresh when some active
+ *                pair (i, j), j in c, has |i - j| <= band_k.
+ *   budget       fraction of active units to recompute: the fresh count is
+ *                max(|band|, floor(budget * active + 1e-9)); the units added
  *                beyond the band are those of largest mass w, ties to the
- *                lower linear index i*P + j.
- *   anchor       nonzero: every active pair fresh (an anchor step).
- * w[i][j] = mean over (b, h, rows r of partition i) of
- *           exp(lse_ij[r]) / sum_{j' active, valid} exp(lse_ij'[r]),
+ *                lower linear index i*G + c.
+ *   anchor       nonzero: every active unit fresh (an anchor step).
+ * w[i][c] = mean over (b, h, rows r of partition i) of
+ *           exp(lse_ic[r]) / sum_{c' active, valid} exp(lse_ic'[r]),
  * computed in float32 with a fixed reduction order (deterministic).
- * Outputs (dev): plan int8 [P*P]; fresh_list int32 [slots] = linear indices
- * i*P + j of the fresh pairs in row-major order; counts int32 [2] = {fresh,
- * reuse}; score_out float32 [P*P] (w, 0 for masked pairs) or NULL.
+ * Outputs (dev): plan int8 [P*G]; fresh_list int32 [slots] = linear indices
+ * i*G + c of the fresh units in row-major order; counts int32 [2] = {fresh,
+ * reuse}; score_out float32 [P*G] (w, 0 for masked units) or NULL.
  * workspace: dev, >= ditango_plan_workspace_size bytes. */
 ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
                             const uint8_t *cache_valid, int32_t band_k, double budget,
@@ -137,16 +156,17 @@ ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
                             int32_t *counts, float *score_out, void *workspace,
                             size_t workspace_bytes, ditango_stream stream);
 
-/* Partial attention states of the fresh pairs (tcgen05 tensor cores, TMA).
- * For each fresh pair (i, j) = fresh_list[f], f < counts[0] (read on the
- * device), and each (b, h): S = Q_i K_j^T * scale, O = softmax(S) V_j
- * (normalised), lse = logsumexp(S) -- the state of DiTango's
- * "Composizione dello Stato".  bf16 inputs, fp32 accumulation and softmax;
+/* Partial attention states of the fresh units (tcgen05 tensor cores, TMA).
+ * For each fresh unit (i, c) = fresh_list[f], f < counts[0] (read on the
+ * device), and each (b, h): S = Q_i K_c^T * scale over the keys K_c of the
+ * active pairs of group c, O = softmax(S) V_c (normalised), lse =
+ * logsumexp(S) -- the state of DiTango's "Composizione dello Stato" (one
+ * pair, or a whole group: "Calcolo dello Stato di Gruppo").  bf16 inputs, fp32 accumulation and softmax;
  * the probabilities are rounded to bf16 for the P V product.
  *   Q, K, V      dev bf16 (uint16 bit patterns) with the geometry's strides.
  *   scale        logit scale; 0 means 1/sqrt(d).
  *   out_O/out_lse  dev state buffer; index = f (out_by_slot = 0) or the
- *                pair's slot (out_by_slot = 1, e.g. writing the cache in
+ *                unit's slot (out_by_slot = 1, e.g. writing the cache in
  *                place).  Must hold counts[0] (resp. all slots) indices.
  *   state_bf16   nonzero: O is stored as bf16 (the normalised fp32 O rounded
  *                to nearest even); lse stays float32.  A compressed cache
@@ -167,13 +187,13 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q,
                                     ditango_stream stream);
 
 /* Merge: the final output of every token is the log-sum-exp composition of
- * the states of its partition's active pairs (DiTango, "Composizione dello
- * Stato"): L = log sum_j exp(lse_j), O = sum_j exp(lse_j - L) O_j, with
+ * the states of its partition's active units (DiTango, "Composizione dello
+ * Stato"): L = log sum_c exp(lse_c), O = sum_c exp(lse_c - L) O_c, with
  * fresh states read from part_O/part_lse (indexed by fresh-list position)
  * and reused ones from cache_O/cache_lse (indexed by slot).  part_O = NULL
  * means the fresh states were already written into the cache slots
  * (ditango_attn_partial with out_by_slot = 1).
- *   plan          dev int8 [P*P] from ditango_plan.
+ *   plan          dev int8 [P*G] from ditango_plan.
  *   writeback     nonzero: also copy each fresh state into its cache slot
  *                 and mark cache_valid (ignored when part_O is NULL).
  *   state_bf16    format of every state buffer passed (see ditango_attn_partial).
@@ -197,6 +217,27 @@ ditango_status ditango_cache_update(const ditango_geom *g, const int8_t *plan,
                                     void *cache_O, float *cache_lse,
                                     uint8_t *cache_valid, int32_t state_bf16,
                                     ditango_stream stream);
+
+/* Dynamic group composition (DiTango, "Composizione Dinamica dei Gruppi"):
+ * merge the cached states of a fine grouping into the states of a coarser
+ * one, with no recomputation: the coarse unit (i, C) gets the log-sum-exp
+ * composition of the fine units (i, c), c inside C, that are active.
+ *   fine, coarse  geometries identical except for G/group_off, and every
+ *                 coarse group boundary a fine group boundary (else INVALID);
+ *                 applied repeatedly (groups of 1 -> 2 -> 4 ...) the cache
+ *                 halves at every level.
+ *   fine_O/fine_lse/fine_valid      dev state buffer of the fine slots
+ *                 (fine_valid may be NULL: all valid).
+ *   coarse_O/coarse_lse/coarse_valid  dev state buffer of the coarse slots
+ *                 (coarse_valid may be NULL); must not overlap the fine one.
+ * A coarse slot is valid only if every fine slot it covers is; an invalid
+ * one is marked 0 and its rows are not written.  Both buffers use the
+ * state format state_bf16 (bf16 results are rounded to nearest even). */
+ditango_status ditango_cache_compose(const ditango_geom *fine, const ditango_geom *coarse,
+                                     const void *fine_O, const float *fine_lse,
+                                     const uint8_t *fine_valid, void *coarse_O,
+                                     float *coarse_lse, uint8_t *coarse_valid,
+                                     int32_t state_bf16, ditango_stream stream);
 
 /* Allocation-free variant of ditango_plan (no counterpart in the papers: it
  * exists for callers, not for the method).  For callers that cannot allocate

@@ -1,13 +1,15 @@
 """B200 partitioned attention with selective attention-state reuse.
 
 The token sequence is split into P context partitions; for every (query
-partition, KV partition) pair the plan either recomputes the attention state
-(output, log-sum-exp) or reuses the one cached at the previous denoising
-step, and the states of each query partition are composed by an exact
-log-sum-exp merge (DiTango: "Cost-Effective Parallel Diffusion Generation
-with Selective Attention State Reuse").  An optional frame-tile mask keeps
-only some frame tiles (Efficient-vDiT: "Efficient Video Diffusion
-Transformers With Attention Tile").
+partition, KV partition) pair -- or, with KV groups, every (query partition,
+group of adjacent KV partitions) unit -- the plan either recomputes the
+attention state (output, log-sum-exp) or reuses the one cached at the
+previous denoising step, and the states of each query partition are composed
+by an exact log-sum-exp merge (DiTango: "Cost-Effective Parallel Diffusion
+Generation with Selective Attention State Reuse").  A cache can be merged
+into coarser groups without recomputation to shrink it.  An optional
+frame-tile mask keeps only some frame tiles (Efficient-vDiT: "Efficient Video
+Diffusion Transformers With Attention Tile").
 
 All compute runs in libditango.so (CUDA, sm_100a) through its C ABI
 (include/ditango.h); this package only marshals arguments.  PyTorch is used
@@ -20,7 +22,7 @@ from ._abi import (  # noqa: F401
     ditango_version, ditango_check_geom, ditango_num_active, ditango_state_rows,
     ditango_slot_table, ditango_plan_workspace_size, ditango_plan, ditango_attn_partial,
     ditango_merge, ditango_cache_update, ditango_set_wait_limit_ns,
-    ditango_selftest_bounded_wait, ditango_plan_noalloc, status_string,
+    ditango_selftest_bounded_wait, ditango_plan_noalloc, ditango_cache_compose, status_string,
 )
 
 
@@ -30,20 +32,24 @@ class PartitionedAttention:
     The state buffer (O [slots, B*H, Lmax, d] float32, or bfloat16 with
     state_bf16=True, a compressed cache; lse float32 [slots, B*H, Lmax]) is
     the attention-state cache: a step writes its fresh states into their
-    slots and the merge reads every active pair from it, so after a step the
-    cache holds this step's fresh states and the reused ones.
+    slots and the merge reads every active unit from it, so after a step the
+    cache holds this step's fresh states and the reused ones.  group_off
+    (partition offsets of the KV groups) makes the units (query partition,
+    KV group); None keeps one group per partition.
     """
 
     def __init__(self, B, H, N, d, part_off, frame_off=None, frame_mask=None,
-                 device="cuda", strides=None, state_bf16=False):
+                 device="cuda", strides=None, state_bf16=False, group_off=None):
         import torch
         self.B, self.H, self.N, self.d = B, H, N, d
         self.part_off = list(part_off)
         self.frame_off = None if frame_off is None else list(frame_off)
         self.frame_mask = frame_mask
+        self.group_off = None if group_off is None else list(group_off)
         self.device = torch.device(device)
         self.geom = self._geometry(strides)
         self.P = self.geom.P
+        self.G = self.geom.G
         self.n_slots = ditango_num_active(self.geom)
         self.Lmax = ditango_state_rows(self.geom)
         BH = B * H
@@ -54,10 +60,10 @@ class PartitionedAttention:
                                    device=dev)
         self.state_lse = torch.empty((self.n_slots, BH, self.Lmax), dtype=torch.float32, device=dev)
         self.valid = torch.zeros(self.n_slots, dtype=torch.uint8, device=dev)
-        self.plan = torch.zeros(self.P * self.P, dtype=torch.int8, device=dev)
+        self.plan = torch.zeros(self.P * self.G, dtype=torch.int8, device=dev)
         self.fresh_list = torch.zeros(max(self.n_slots, 1), dtype=torch.int32, device=dev)
         self.counts = torch.zeros(2, dtype=torch.int32, device=dev)
-        self.score = torch.zeros(self.P * self.P, dtype=torch.float32, device=dev)
+        self.score = torch.zeros(self.P * self.G, dtype=torch.float32, device=dev)
         self.ws_bytes = ditango_plan_workspace_size(self.geom)
         self.workspace = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -65,7 +71,8 @@ class PartitionedAttention:
     def _geometry(self, strides):
         s = strides or (None, None, None)
         return Geometry(self.B, self.H, self.N, self.d, self.part_off, self.frame_off,
-                        self.frame_mask, q_strides=s[0], k_strides=s[1], v_strides=s[2])
+                        self.frame_mask, q_strides=s[0], k_strides=s[1], v_strides=s[2],
+                        group_off=self.group_off)
 
     def _bind(self, Q, K, V):
         want = tuple(tuple(t.stride()[:3]) for t in (Q, K, V))
@@ -92,7 +99,20 @@ class PartitionedAttention:
 
     def step(self, Q, K, V, out, out_lse=None, band_k=0, budget=1.0, anchor=False, scale=0.0,
              stream=None):
-        """plan -> partial attention of the fresh pairs -> merge, on one stream."""
+        """plan -> partial attention of the fresh units -> merge, on one stream."""
         self.plan_step(band_k, budget, anchor, stream)
         self.partial(Q, K, V, scale, stream)
         self.merge(out, out_lse, stream)
+
+    def compose(self, group_off, stream=None):
+        """A new PartitionedAttention with coarser KV groups whose cache is this
+        cache's states merged group by group (no attention is recomputed).
+        Every boundary of group_off must be one of this object's boundaries.
+        The caller may drop this object afterwards to free the finer cache."""
+        coarse = PartitionedAttention(self.B, self.H, self.N, self.d, self.part_off, self.frame_off,
+                                      self.frame_mask, self.device, None, self.state_bf16,
+                                      group_off)
+        ditango_cache_compose(self.geom, coarse.geom, self.state_O, self.state_lse, self.valid,
+                              coarse.state_O, coarse.state_lse, coarse.valid, self.state_bf16,
+                              stream)
+        return coarse

@@ -34,6 +34,8 @@ class ditango_geom(C.Structure):
         ("q_strides", C.c_int64 * 3),
         ("k_strides", C.c_int64 * 3),
         ("v_strides", C.c_int64 * 3),
+        ("G", C.c_int32),
+        ("group_off", C.POINTER(C.c_int32)),
     ]
 
 
@@ -65,6 +67,7 @@ _SIGS = {
     "ditango_cache_update": (C.c_int, [_G, _P, _P, _P, _P, _P, _P, C.c_int32, _P]),
     "ditango_plan_noalloc": (C.c_int, [_G, _P, _P, C.c_int32, C.c_double, C.c_int32, _P, _P, _P,
                                        _P, _P]),
+    "ditango_cache_compose": (C.c_int, [_G, _G, _P, _P, _P, _P, _P, _P, C.c_int32, _P]),
     "ditango_set_wait_limit_ns": (None, [C.c_int64]),
     "ditango_selftest_bounded_wait": (C.c_int, [C.c_int64, _P, _P]),
 }
@@ -103,13 +106,20 @@ def _check(fn, st):
 
 
 class Geometry:
-    """Owns the host arrays a ditango_geom points to."""
+    """Owns the host arrays a ditango_geom points to.
+
+    group_off: partition offsets of the KV groups (None: one group per
+    partition); G, the number of plan columns, is len(group_off) - 1.
+    """
 
     def __init__(self, B, H, N, d, part_off, frame_off=None, frame_mask=None,
-                 q_strides=None, k_strides=None, v_strides=None):
+                 q_strides=None, k_strides=None, v_strides=None, group_off=None):
         P = len(part_off) - 1
         F = 0 if frame_off is None else len(frame_off) - 1
         self._part = (C.c_int32 * (P + 1))(*[int(x) for x in part_off])
+        self._groups = None
+        if group_off is not None:
+            self._groups = (C.c_int32 * len(group_off))(*[int(x) for x in group_off])
         self._frame = None
         self._fmask = None
         if F:
@@ -122,10 +132,14 @@ class Geometry:
         g.part_off = C.cast(self._part, C.POINTER(C.c_int32))
         g.frame_off = C.cast(self._frame, C.POINTER(C.c_int32)) if F else None
         g.frame_mask = C.cast(self._fmask, C.POINTER(C.c_uint8)) if F else None
+        g.G = 0 if group_off is None else len(group_off) - 1
+        g.group_off = C.cast(self._groups, C.POINTER(C.c_int32)) if group_off is not None else None
         for name, s in (("q_strides", q_strides), ("k_strides", k_strides), ("v_strides", v_strides)):
             getattr(g, name)[:] = list(s if s is not None else contig)
         self.g = g
         self.B, self.H, self.N, self.d, self.P, self.F = B, H, N, d, P, F
+        self.group_off = None if group_off is None else [int(x) for x in group_off]
+        self.G = P if group_off is None else len(group_off) - 1
 
     @property
     def ref(self):
@@ -159,9 +173,9 @@ def ditango_state_rows(geom: Geometry) -> int:
 
 
 def ditango_slot_table(geom: Geometry):
-    out = (C.c_int32 * (geom.P * geom.P))()
+    out = (C.c_int32 * (geom.P * geom.G))()
     _check("ditango_slot_table", _lib.ditango_slot_table(geom.ref, C.cast(out, C.c_void_p)))
-    return [[out[i * geom.P + j] for j in range(geom.P)] for i in range(geom.P)]
+    return [[out[i * geom.G + c] for c in range(geom.G)] for i in range(geom.P)]
 
 
 def ditango_plan_workspace_size(geom: Geometry) -> int:
@@ -203,6 +217,13 @@ def ditango_cache_update(geom, plan, part_O, part_lse, cache_O, cache_lse, cache
     _check("ditango_cache_update", _lib.ditango_cache_update(
         geom.ref, _ptr(plan), _ptr(part_O), _ptr(part_lse), _ptr(cache_O), _ptr(cache_lse),
         _ptr(cache_valid), int(bool(state_bf16)), _stream(stream)))
+
+
+def ditango_cache_compose(fine, coarse, fine_O, fine_lse, fine_valid, coarse_O, coarse_lse,
+                          coarse_valid, state_bf16=0, stream=None):
+    _check("ditango_cache_compose", _lib.ditango_cache_compose(
+        fine.ref, coarse.ref, _ptr(fine_O), _ptr(fine_lse), _ptr(fine_valid), _ptr(coarse_O),
+        _ptr(coarse_lse), _ptr(coarse_valid), int(bool(state_bf16)), _stream(stream)))
 
 
 def ditango_set_wait_limit_ns(ns: int) -> None:

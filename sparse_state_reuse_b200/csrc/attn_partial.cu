@@ -1,11 +1,15 @@
-// Partial attention states of the fresh (query partition, KV partition)
-// pairs on B200: tcgen05 MMA with TMEM accumulators, TMA-staged Q/K/V tiles.
+// Partial attention states of the fresh (query partition, KV group) units
+// on B200: tcgen05 MMA with TMEM accumulators, TMA-staged Q/K/V tiles.
 //
-// What a work unit computes (DiTango, "Riepilogo Tecnico" -> Metodologia ->
-// 2. State-Centric Parallel Runtime, "Composizione dello Stato"): for up to
-// 256 query rows of partition i and all keys of partition j of one (b, h),
-// the state O = softmax(Q K^T * scale) V (normalised) and
+// What a work item computes (DiTango, "Riepilogo Tecnico" -> Metodologia ->
+// 2. State-Centric Parallel Runtime, "Composizione dello Stato" and
+// "Calcolo dello Stato di Gruppo"): for up to 256 query rows of partition i
+// and all keys of the active partitions of KV group c of one (b, h), the
+// state O = softmax(Q K^T * scale) V (normalised) and
 // lse = log sum exp(Q K^T * scale), by an online softmax over 128-key tiles.
+// Without KV groups a group is one partition and a unit is a pair (i, j).
+// A group's active partitions are walked as runs of adjacent partitions,
+// each run one contiguous key range whose last tile is masked at its end.
 //
 // CTA organisation (one CTA per SM, persistent over work units, 384 threads):
 //   warps 0-3  softmax warpgroup 0: rows   0..127 of the unit (Q tile 0)
@@ -72,7 +76,7 @@ struct Params {
 };
 
 // A work item: up to 256 query rows of partition i for one (b, h).  The item
-// visits every fresh pair (i, j) of row i in fresh-list order, so its Q tiles
+// visits every fresh unit (i, c) of row i in fresh-list order, so its Q tiles
 // are loaded once and reused for all of them.
 struct Item {
   bool live;
@@ -83,9 +87,53 @@ struct Item {
   int f0, f1;      // fresh-list range of row i
 };
 
-struct PairRange {
-  int f, j;
-  int k0, Lk, T;   // first key token, keys, key tiles of partition j
+struct UnitRange {
+  int f, c;
+  int T;                     // key tiles over all runs of adjacent partitions
+  int k0, Lk;                // key range of the first run (the only one unless MR)
+};
+
+// Partitions whose keys unit (i, c) attends: its active pairs; for a masked
+// unit in the fresh list (never from the planner) the group's partitions
+// unmasked, so that every role still sees at least one tile.
+__device__ __forceinline__ unsigned long long unit_key_bits(const DevGeom &g, int i, int c) {
+  const unsigned long long b = unit_pairs(g, i, c);
+  return b ? b : bit_range(g.group_off[c], g.group_off[c + 1]);
+}
+
+// The first run of adjacent partitions in `bits` (nonzero): its key range
+// [k0, k0 + Lk) and the partition after it.
+__device__ __forceinline__ void first_run(const DevGeom &g, unsigned long long bits, int &k0,
+                                          int &Lk, int &jend) {
+  const int j0 = __ffsll((long long)bits) - 1;
+  const unsigned long long sh = bits >> j0;
+  const int len = (~sh == 0ull) ? 64 - j0 : __ffsll((long long)~sh) - 1;
+  jend = j0 + len;
+  k0 = g.part_off[j0];
+  Lk = g.part_off[jend] - k0;
+}
+
+// Key tiles of unit (i, c) in order: tile t of the current run.  Only the
+// end of the current run is held; the next run is found again from the
+// geometry (kernel parameters), which keeps the softmax warps' registers.
+struct KeyCursor {
+  int k0, Lk, t, jend;
+  __device__ __forceinline__ void start(const DevGeom &g, int i, int c) {
+    first_run(g, unit_key_bits(g, i, c), k0, Lk, jend);
+    t = 0;
+  }
+  __device__ __forceinline__ int row() const { return k0 + t * BN; }
+  __device__ __forceinline__ int valid() const { return Lk - t * BN; }
+  __device__ __forceinline__ void next(const DevGeom &g, int i, int c) {
+    ++t;
+    if (t * BN >= Lk) {
+      const unsigned long long rest = unit_key_bits(g, i, c) & ~bit_range(0, jend);
+      if (rest) {
+        first_run(g, rest, k0, Lk, jend);
+        t = 0;
+      }
+    }
+  }
 };
 
 __device__ __forceinline__ Item decode_item(const Params &p, const int *row_fresh, int it, int nqt2) {
@@ -109,15 +157,33 @@ __device__ __forceinline__ Item decode_item(const Params &p, const int *row_fres
   return w;
 }
 
-__device__ __forceinline__ PairRange pair_at(const Params &p, int f) {
-  PairRange q;
-  const int pair = __ldg(p.fresh_list + f);
-  q.f = f;
-  q.j = pair % p.g.P;
-  q.k0 = p.g.part_off[q.j];
-  q.Lk = p.g.part_off[q.j + 1] - q.k0;
-  q.T = (q.Lk + BN - 1) / BN;
-  return q;
+// MR: units may hold several runs of adjacent partitions (a frame mask that
+// leaves a gap inside a KV group); otherwise every unit is one key range.
+template <bool MR>
+__device__ __forceinline__ UnitRange unit_at(const Params &p, int i, int f) {
+  UnitRange u;
+  const int unit = __ldg(p.fresh_list + f);
+  u.f = f;
+  u.c = unit % p.g.G;
+  unsigned long long rest = unit_key_bits(p.g, i, u.c);
+  if constexpr (!MR) {
+    // one run: from the first to the last active partition
+    u.k0 = p.g.part_off[__ffsll((long long)rest) - 1];
+    u.Lk = p.g.part_off[64 - __clzll((long long)rest)] - u.k0;
+    u.T = (u.Lk + BN - 1) / BN;
+  } else {
+    int jend = 0;
+    first_run(p.g, rest, u.k0, u.Lk, jend);
+    u.T = (u.Lk + BN - 1) / BN;
+    rest &= ~bit_range(0, jend);
+    while (rest) {
+      int k0, Lk;
+      first_run(p.g, rest, k0, Lk, jend);
+      rest &= ~bit_range(0, jend);
+      u.T += (Lk + BN - 1) / BN;
+    }
+  }
+  return u;
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -194,7 +260,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
-template <int D, bool SB>   // SB: states stored with bf16 O (compressed cache)
+// SB: states stored with bf16 O (compressed cache); MR: see unit_at.
+template <int D, bool SB, bool MR>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params p) {
@@ -235,8 +302,11 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   __syncthreads();
   {
     const int n_fresh = __ldg(p.counts);
-    for (int f = threadIdx.x; f < n_fresh; f += blockDim.x)
-      atomicAdd(&row_fresh[__ldg(p.fresh_list + f) / p.g.P + 1], 1);
+    const int n_units = p.g.P * p.g.G;
+    for (int f = threadIdx.x; f < n_fresh; f += blockDim.x) {
+      const int u = __ldg(p.fresh_list + f);
+      if (u >= 0 && u < n_units) atomicAdd(&row_fresh[u / p.g.G + 1], 1);
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0)
@@ -304,9 +374,14 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
               tma_load_4d(sQ + C::TILE + c * C::CHUNK, &tmQ, q_full, c * 64, w.q0 + BM, w.h, w.b);
         }
         for (int f = w.f0; f < w.f1 && ok; ++f) {
-          const PairRange pr = pair_at(p, f);
+          const UnitRange pr = unit_at<MR>(p, w.i, f);
+          KeyCursor cur;
+          if constexpr (MR) cur.start(p.g, w.i, pr.c);
           for (int t = 0; t < pr.T && ok; ++t) {
-            const int row = pr.k0 + t * BN;
+            if constexpr (MR) {
+              if (t > 0) cur.next(p.g, w.i, pr.c);
+            }
+            const int row = MR ? cur.row() : pr.k0 + t * BN;
             int s = kc % kStages;
             if (!(ok = wait_warp(k_empty(s), ((kc / kStages) & 1) ^ 1, ctl))) break;
             if (leader) mbar_arrive_expect_tx(k_full(s), C::TILE);
@@ -388,7 +463,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const bool has1 = w.rows1 > 0;
         if (!(ok = wait_warp(q_full, uc & 1, ctl))) break;
         for (int f = w.f0; f < w.f1 && ok; ++f) {
-          const PairRange pr = pair_at(p, f);
+          const UnitRange pr = unit_at<MR>(p, w.i, f);
           const bool last_pair = (f + 1 == w.f1);
           int ks = kc % kStages;
           if (!(ok = wait_warp(k_full(ks), (kc / kStages) & 1, ctl))) break;
@@ -485,10 +560,15 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       const int rows_k = (k == 0) ? w.rows0 : w.rows1;
       if (rows_k <= 0) continue;
      for (int f = w.f0; f < w.f1 && ok; ++f) {
-      const PairRange pr = pair_at(p, f);
+      const UnitRange pr = unit_at<MR>(p, w.i, f);
+      KeyCursor cur;
+      if constexpr (MR) cur.start(p.g, w.i, pr.c);
       float m_used = -INFINITY;   // running maximum used for exponentiation (log2 units)
       float l = 0.f;
       for (int t = 0; t < pr.T; ++t) {
+        if constexpr (MR) {
+          if (t > 0) cur.next(p.g, w.i, pr.c);
+        }
         if (!(ok = wait_bounded(s_full(k), sc & 1, ctl))) break;
         ++sc;
         tc_fence_after();
@@ -497,7 +577,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
         for (int c = 0; c < BN / 16; ++c) tmem_ld16p(tS + c * 16, &sv[c * 16]);
         tc_wait_ld();
-        const int valid = pr.Lk - t * BN;
+        const int valid = MR ? cur.valid() : pr.Lk - t * BN;
         if (valid < BN) {
 #pragma unroll
           for (int c = 0; c < BN; ++c)
@@ -582,12 +662,14 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       // 128-byte row segments (XOR swizzle: both phases free of bank
       // conflicts).
       constexpr int HALF = (D > 64) ? 64 : D;
-      const int idx = p.out_by_slot ? slot_of(p.g, w.i, pr.j) : pr.f;
+      const int idx = p.out_by_slot ? slot_of(p.g, w.i, pr.c) : pr.f;
       const int rloc = w.rloc0 + k * BM + r;
       const size_t row_off = ((size_t)idx * p.g.BH + w.bh) * (size_t)p.g.Lmax + rloc;
       const float inv_l = 1.f / l;
       float4 *epi = reinterpret_cast<float4 *>(smem + C::OFF_EPI + (warp & 7) * 4096);
-      const int row_valid = rows_k - (r & ~31);         // valid rows of this warp
+      // a masked unit in the fresh list has no slot: nothing is stored by slot
+      const bool store = !p.out_by_slot || unit_pairs(p.g, w.i, pr.c) != 0ull;
+      const int row_valid = store ? rows_k - (r & ~31) : 0;   // rows of this warp to store
 #pragma unroll
       for (int h0 = 0; h0 < D; h0 += HALF) {
         constexpr int W = HALF;
@@ -650,8 +732,8 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           __syncwarp();
         }
       }
-      if (r < rows_k) p.out_lse[row_off] = (m_used + __log2f(l)) * 0.69314718055994531f;
-      if (p.out_by_slot && p.out_valid && k == 0 && r == 0) p.out_valid[idx] = 1;
+      if (store && r < rows_k) p.out_lse[row_off] = (m_used + __log2f(l)) * 0.69314718055994531f;
+      if (store && p.out_by_slot && p.out_valid && k == 0 && r == 0) p.out_valid[idx] = 1;
      }
     }
     tc_fence_before();
@@ -686,7 +768,10 @@ cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const C
   switch (g.d) {
 #define DITANGO_LAUNCH(DD)                                                                       \
   case DD: {                                                                                     \
-    auto kfn = state_bf16 ? attn::attn_partial_kernel<DD, true> : attn::attn_partial_kernel<DD, false>; \
+    auto kfn = state_bf16 ? (g.multi_run ? attn::attn_partial_kernel<DD, true, true>             \
+                                         : attn::attn_partial_kernel<DD, true, false>)           \
+                          : (g.multi_run ? attn::attn_partial_kernel<DD, false, true>            \
+                                         : attn::attn_partial_kernel<DD, false, false>);         \
     cudaFuncAttributes fa;                                                                       \
     e = cudaFuncGetAttributes(&fa, kfn);                                                         \
     if (e != cudaSuccess) return e;                                                              \

@@ -14,23 +14,51 @@ namespace ditango {
 constexpr int kMaxP = 64;
 
 // Geometry as the kernels see it.  Built on the host from ditango_geom.
+// Columns of the plan and of the slot table are KV groups (runs of adjacent
+// partitions); without groups every partition is its own group and G = P.
+// A unit (i, c) pairs query partition i with KV group c.
 struct DevGeom {
   int B, H, N, d, P, BH;
+  int G;              // KV groups
   int Lmax;           // longest partition
-  int n_active;       // slots
-  int n_band;         // band pairs (plan only)
+  int n_active;       // active units = slots
+  int n_band;         // band units (plan only)
+  int multi_run;      // some unit's active partitions are not adjacent
   int part_off[kMaxP + 1];
-  int row_start[kMaxP + 1];          // slot of the first active pair of row i
-  unsigned long long row_mask[kMaxP];  // bit j set: pair (i, j) active
+  int group_off[kMaxP + 1];            // first partition of each KV group
+  int row_start[kMaxP + 1];            // slot of the first active unit of row i
+  unsigned long long row_mask[kMaxP];  // bit c set: unit (i, c) active
+  unsigned long long pair_mask[kMaxP]; // bit j set: pair (i, j) active
 };
 
-__host__ __device__ inline int slot_of(const DevGeom &g, int i, int j) {
-  unsigned long long below = (j == 0) ? 0ull : (g.row_mask[i] & ((~0ull) >> (64 - j)));
+__host__ __device__ inline int slot_of(const DevGeom &g, int i, int c) {
+  unsigned long long below = (c == 0) ? 0ull : (g.row_mask[i] & ((~0ull) >> (64 - c)));
 #ifdef __CUDA_ARCH__
   return g.row_start[i] + __popcll(below);
 #else
   return g.row_start[i] + __builtin_popcountll(below);
 #endif
+}
+
+// Bits of the partitions j0 <= j < j1.
+__host__ __device__ inline unsigned long long bit_range(int j0, int j1) {
+  const unsigned long long hi = (j1 >= 64) ? ~0ull : ((1ull << j1) - 1ull);
+  const unsigned long long lo = (1ull << j0) - 1ull;
+  return hi & ~lo;
+}
+
+// Active pairs (i, j) of unit (i, c): the partitions of group c that the
+// frame mask lets partition i attend.
+__host__ __device__ inline unsigned long long unit_pairs(const DevGeom &g, int i, int c) {
+  return g.pair_mask[i] & bit_range(g.group_off[c], g.group_off[c + 1]);
+}
+
+// Unit (i, c) is in the distance band when one of its active pairs (i, j)
+// has |i - j| <= k.
+__host__ __device__ inline bool unit_in_band(const DevGeom &g, int i, int c, int k) {
+  const int lo = (i - k < 0) ? 0 : i - k;
+  const int hi = (i + k + 1 > g.P) ? g.P : i + k + 1;
+  return (unit_pairs(g, i, c) & bit_range(lo, hi)) != 0ull;
 }
 
 // ---------------------------------------------------------------------------

@@ -27,6 +27,10 @@ cudaError_t launch_cache_update(const DevGeom &g, const signed char *plan, const
                                 const float *part_lse, void *cache_O, float *cache_lse,
                                 unsigned char *cache_valid, int state_bf16, int num_sms,
                                 cudaStream_t stream);
+cudaError_t launch_cache_compose(const DevGeom &fine, const DevGeom &coarse, const void *fine_O,
+                                 const float *fine_lse, const unsigned char *fine_valid,
+                                 void *coarse_O, float *coarse_lse, unsigned char *coarse_valid,
+                                 int state_bf16, cudaStream_t stream);
 cudaError_t launch_bounded_wait_selftest(long long limit_ns, int *dev_status,
                                          cudaStream_t stream);
 }  // namespace ditango
@@ -78,24 +82,64 @@ ditango_status make_geom(const ditango_geom *in, DevGeom *out) {
     if (L > lmax) lmax = L;
   }
   g.Lmax = lmax;
-  int slot = 0;
+  // KV groups: runs of adjacent partitions (one per partition without groups)
+  if (in->G < 0 || in->G > in->P) return DITANGO_ERR_INVALID;
+  if (in->G == 0) {
+    g.G = in->P;
+    for (int c = 0; c <= in->P; ++c) g.group_off[c] = c;
+  } else {
+    if (!in->group_off || in->group_off[0] != 0 || in->group_off[in->G] != in->P)
+      return DITANGO_ERR_INVALID;
+    for (int c = 0; c < in->G; ++c)
+      if (in->group_off[c + 1] <= in->group_off[c]) return DITANGO_ERR_INVALID;
+    g.G = in->G;
+    for (int c = 0; c <= in->G; ++c) g.group_off[c] = in->group_off[c];
+  }
   for (int i = 0; i < in->P; ++i) {
-    g.row_start[i] = slot;
     unsigned long long m = 0;
     for (int j = 0; j < in->P; ++j) {
       bool act = true;
       if (in->F > 0) act = in->frame_mask[part_frame[i] * in->F + part_frame[j]] != 0;
-      if (act) {
-        m |= 1ull << j;
+      if (act) m |= 1ull << j;
+    }
+    g.pair_mask[i] = m;
+  }
+  int slot = 0;
+  for (int i = 0; i < in->P; ++i) {
+    g.row_start[i] = slot;
+    unsigned long long m = 0;
+    for (int c = 0; c < g.G; ++c)
+      if (unit_pairs(g, i, c)) {
+        m |= 1ull << c;
         ++slot;
       }
-    }
     g.row_mask[i] = m;
   }
   g.row_start[in->P] = slot;
   g.n_active = slot;
+  g.multi_run = 0;
+  for (int i = 0; i < in->P; ++i)
+    for (int c = 0; c < g.G; ++c) {
+      const unsigned long long b = unit_pairs(g, i, c);
+      if (!b) continue;
+      const unsigned long long sh = b >> __builtin_ctzll(b);
+      if (sh & (sh + 1ull)) g.multi_run = 1;   // a gap between active partitions
+    }
   *out = g;
   return DITANGO_OK;
+}
+
+// Fresh-unit count of a plan: max(|band|, floor(budget * active + 1e-9)).
+int plan_target(DevGeom *dg, int band_k, double budget) {
+  int n_band = 0;
+  for (int i = 0; i < dg->P; ++i)
+    for (int c = 0; c < dg->G; ++c)
+      if (((dg->row_mask[i] >> c) & 1ull) && unit_in_band(*dg, i, c, band_k)) ++n_band;
+  int target = (int)std::floor(budget * (double)dg->n_active + 1e-9);
+  if (target < n_band) target = n_band;
+  if (target > dg->n_active) target = dg->n_active;
+  dg->n_band = n_band;
+  return target;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -157,7 +201,7 @@ ditango_status cuda_status(cudaError_t e) {
 
 extern "C" {
 
-int32_t ditango_version(void) { return 10000; }
+int32_t ditango_version(void) { return 10100; }
 
 const char *ditango_status_string(int32_t s) {
   switch (s) {
@@ -193,8 +237,8 @@ ditango_status ditango_slot_table(const ditango_geom *g, int32_t *slot_out) {
   if (st != DITANGO_OK) return st;
   if (!slot_out) return DITANGO_ERR_INVALID;
   for (int i = 0; i < dg.P; ++i)
-    for (int j = 0; j < dg.P; ++j)
-      slot_out[i * dg.P + j] = ((dg.row_mask[i] >> j) & 1ull) ? slot_of(dg, i, j) : -1;
+    for (int c = 0; c < dg.G; ++c)
+      slot_out[i * dg.G + c] = ((dg.row_mask[i] >> c) & 1ull) ? slot_of(dg, i, c) : -1;
   return DITANGO_OK;
 }
 
@@ -217,14 +261,7 @@ ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
     if (!cache_lse || band_k < 0 || !(budget >= 0.0 && budget <= 1.0)) return DITANGO_ERR_INVALID;
     if (!workspace || workspace_bytes < plan_workspace_bytes(dg)) return DITANGO_ERR_INVALID;
   }
-  int n_band = 0;
-  for (int i = 0; i < dg.P; ++i)
-    for (int j = 0; j < dg.P; ++j)
-      if (((dg.row_mask[i] >> j) & 1ull) && std::abs(i - j) <= band_k) ++n_band;
-  int target = (int)std::floor(budget * (double)dg.n_active + 1e-9);
-  if (target < n_band) target = n_band;
-  if (target > dg.n_active) target = dg.n_active;
-  dg.n_band = n_band;
+  const int target = plan_target(&dg, band_k, budget);
   return cuda_status(launch_plan(dg, cache_lse, cache_valid, band_k, target, anchor ? 1 : 0,
                                  reinterpret_cast<signed char *>(plan), fresh_list, counts,
                                  score_out, workspace, static_cast<cudaStream_t>(stream)));
@@ -301,6 +338,46 @@ ditango_status ditango_cache_update(const ditango_geom *g, const int8_t *plan,
                                          static_cast<cudaStream_t>(stream)));
 }
 
+ditango_status ditango_cache_compose(const ditango_geom *fine, const ditango_geom *coarse,
+                                     const void *fine_O, const float *fine_lse,
+                                     const uint8_t *fine_valid, void *coarse_O,
+                                     float *coarse_lse, uint8_t *coarse_valid,
+                                     int32_t state_bf16, ditango_stream stream) {
+  DevGeom gf, gc;
+  ditango_status st = make_geom(fine, &gf);
+  if (st != DITANGO_OK) return st;
+  st = make_geom(coarse, &gc);
+  if (st != DITANGO_OK) return st;
+  // same attention call, only the KV grouping differs
+  if (gf.B != gc.B || gf.H != gc.H || gf.N != gc.N || gf.d != gc.d || gf.P != gc.P)
+    return DITANGO_ERR_INVALID;
+  for (int p = 0; p <= gf.P; ++p)
+    if (gf.part_off[p] != gc.part_off[p]) return DITANGO_ERR_INVALID;
+  for (int i = 0; i < gf.P; ++i)
+    if (gf.pair_mask[i] != gc.pair_mask[i]) return DITANGO_ERR_INVALID;
+  // every coarse group boundary is a fine group boundary
+  for (int C = 0, c = 0; C <= gc.G; ++C) {
+    while (c <= gf.G && gf.group_off[c] < gc.group_off[C]) ++c;
+    if (c > gf.G || gf.group_off[c] != gc.group_off[C]) return DITANGO_ERR_INVALID;
+  }
+  if (!fine_O || !fine_lse || !coarse_O || !coarse_lse) return DITANGO_ERR_INVALID;
+  const size_t align = state_bf16 ? 8 : 16;
+  if (reinterpret_cast<uintptr_t>(fine_O) % align || reinterpret_cast<uintptr_t>(coarse_O) % align)
+    return DITANGO_ERR_INVALID;
+  // the two state buffers must not overlap
+  const size_t rows = (size_t)gf.BH * gf.Lmax;
+  const size_t es = state_bf16 ? 2 : 4;
+  const char *f0 = static_cast<const char *>(fine_O), *f1 = f0 + (size_t)gf.n_active * rows * gf.d * es;
+  const char *c0 = static_cast<const char *>(coarse_O), *c1 = c0 + (size_t)gc.n_active * rows * gc.d * es;
+  if (f0 < c1 && c0 < f1) return DITANGO_ERR_INVALID;
+  const float *fl0 = fine_lse, *fl1 = fine_lse + (size_t)gf.n_active * rows;
+  const float *cl0 = coarse_lse, *cl1 = coarse_lse + (size_t)gc.n_active * rows;
+  if (fl0 < cl1 && cl0 < fl1) return DITANGO_ERR_INVALID;
+  return cuda_status(launch_cache_compose(gf, gc, fine_O, fine_lse, fine_valid, coarse_O,
+                                          coarse_lse, coarse_valid, state_bf16 ? 1 : 0,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 void ditango_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns = ns > 0 ? ns : 1; }
 
 ditango_status ditango_selftest_bounded_wait(int64_t limit_ns, int32_t *dev_status,
@@ -360,14 +437,7 @@ extern "C" ditango_status ditango_plan_noalloc(const ditango_geom *g, const floa
     }
     scratch = g_noalloc_scratch[dev];
   }
-  int n_band = 0;
-  for (int i = 0; i < dg.P; ++i)
-    for (int j = 0; j < dg.P; ++j)
-      if (((dg.row_mask[i] >> j) & 1ull) && std::abs(i - j) <= band_k) ++n_band;
-  int target = (int)std::floor(budget * (double)dg.n_active + 1e-9);
-  if (target < n_band) target = n_band;
-  if (target > dg.n_active) target = dg.n_active;
-  dg.n_band = n_band;
+  const int target = plan_target(&dg, band_k, budget);
   return cuda_status(launch_plan(dg, cache_lse, cache_valid, band_k, target, anchor ? 1 : 0,
                                  reinterpret_cast<signed char *>(plan), fresh_list, counts,
                                  score_out, scratch, static_cast<cudaStream_t>(stream)));

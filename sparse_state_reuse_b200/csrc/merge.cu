@@ -2,8 +2,9 @@
 //
 // DiTango, "Riepilogo Tecnico" -> Metodologia -> 2. State-Centric Parallel
 // Runtime, "Composizione dello Stato": the output of a query row is the
-// composition of the states of all active pairs of its partition,
-//   L = M + log sum_j exp(lse_j - M),  O = sum_j exp(lse_j - L) O_j,
+// composition of the states of all active units (KV partitions, or KV
+// groups) of its partition,
+//   L = M + log sum_c exp(lse_c - M),  O = sum_c exp(lse_c - L) O_c,
 // fresh states coming from this step's partial buffer and reused ones from
 // the cache.  "Anchor Steps": the states computed fresh refresh the cache.
 //
@@ -139,7 +140,7 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
              const float *__restrict__ part_lse, char *cache_O, float *cache_lse,
              unsigned char *cache_valid, int writeback, void *out, int out_is_fp32, long long osb,
              long long osh, long long osn, float *__restrict__ out_lse) {
-  constexpr int G = D / 4;  // lanes carrying one row
+  constexpr int G4 = D / 4;  // lanes carrying one row
   constexpr int ES = SB ? 2 : 4;            // bytes per stored O element
   constexpr size_t ROWB = (size_t)D * ES;   // bytes per state row
   const int i = blockIdx.y;
@@ -147,16 +148,16 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
   const int Li = g.part_off[i + 1] - g.part_off[i];
   const int r0 = blockIdx.x * kRowsPerBlock;
   if (r0 >= Li) return;
-  const int P = g.P;
+  const int G = g.G;
   __shared__ Src src[kMaxP];
   __shared__ int s_nact, s_fresh_before;
   __shared__ int warp_cnt[kWarps];
   __shared__ signed char s_plan[kMaxP];
-  if (threadIdx.x < P) s_plan[threadIdx.x] = plan[i * P + threadIdx.x];
+  if (threadIdx.x < G) s_plan[threadIdx.x] = plan[i * G + threadIdx.x];
 
-  // fresh pairs before row i (row-major), for fresh-list positions
+  // fresh units before row i (row-major), for fresh-list positions
   int cnt = 0;
-  for (int p = threadIdx.x; p < i * P; p += kThreads) cnt += (plan[p] == DITANGO_PLAN_FRESH);
+  for (int p = threadIdx.x; p < i * G; p += kThreads) cnt += (plan[p] == DITANGO_PLAN_FRESH);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
   if ((threadIdx.x & 31) == 0) warp_cnt[threadIdx.x >> 5] = cnt;
@@ -169,10 +170,10 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
     int a = 0;
     const int slot0 = g.row_start[i];
     int fpos = fb;
-    for (int j = 0; j < P; ++j) {
-      if (!((g.row_mask[i] >> j) & 1ull)) continue;
-      const int code = s_plan[j];
-      const int slot = slot0 + __popcll(g.row_mask[i] & ((j == 0) ? 0ull : (~0ull >> (64 - j))));
+    for (int c = 0; c < G; ++c) {
+      if (!((g.row_mask[i] >> c) & 1ull)) continue;
+      const int code = s_plan[c];
+      const int slot = slot0 + __popcll(g.row_mask[i] & ((c == 0) ? 0ull : (~0ull >> (64 - c))));
       Src s;
       s.wbO = nullptr;
       s.wblse = nullptr;
@@ -194,7 +195,7 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
         s.O = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * ROWB;
         s.lse = cache_lse + (size_t)slot * blk + (size_t)bh * g.Lmax;
       } else {
-        continue;  // active pair the plan skipped: contributes nothing
+        continue;  // active unit the plan skipped: contributes nothing
       }
       src[a++] = s;
     }
@@ -218,7 +219,7 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
       l0[q] = (ok && lane < nact) ? __ldg(src[lane].lse + r + q) : -INFINITY;
       l1[q] = (ok && lane + 32 < nact) ? __ldg(src[lane + 32].lse + r + q) : -INFINITY;
     }
-    const bool act = lane < G;
+    const bool act = lane < G4;
     typename Raw4<SB>::T v[R][kBatch];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u)
@@ -276,8 +277,8 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
 }
 
 // Copy the fresh states (fresh-list positions) into their cache slots.
-// blockIdx.y = slot; the block finds its pair, and if the plan marks it fresh
-// counts the fresh pairs before it (row-major) to find its fresh position.
+// blockIdx.y = slot; the block finds its unit, and if the plan marks it fresh
+// counts the fresh units before it (row-major) to find its fresh position.
 __global__ void __launch_bounds__(256)
 cache_update_kernel(DevGeom g, const signed char *__restrict__ plan,
                     const char *__restrict__ part_O, const float *__restrict__ part_lse,
@@ -288,8 +289,8 @@ cache_update_kernel(DevGeom g, const signed char *__restrict__ plan,
   int rank = slot - g.row_start[i];
   unsigned long long m = g.row_mask[i];
   for (int t = 0; t < rank; ++t) m &= m - 1;
-  const int j = __ffsll((long long)m) - 1;
-  const int pair = i * g.P + j;
+  const int c = __ffsll((long long)m) - 1;
+  const int pair = i * g.G + c;
   if (plan[pair] != DITANGO_PLAN_FRESH) return;
   __shared__ int warp_cnt[8];
   __shared__ int s_fpos;
@@ -319,6 +320,101 @@ cache_update_kernel(DevGeom g, const signed char *__restrict__ plan,
        t += (size_t)gridDim.x * blockDim.x)
     dl[t] = __ldg(sl + t);
   if (cache_valid && blockIdx.x == 0 && threadIdx.x == 0) cache_valid[slot] = 1;
+}
+
+// Dynamic group composition (DiTango, 2. State-Centric Parallel Runtime,
+// "Composizione Dinamica dei Gruppi"): the cached state of coarse unit
+// (i, C) is the log-sum-exp composition of the cached states of the fine
+// units (i, c), c inside C -- no attention is recomputed.  Those fine units
+// are consecutive slots of the fine cache.  blockIdx.y = coarse slot,
+// blockIdx.z = b*h, blockIdx.x = a block of kRowsPerBlock rows; one warp
+// merges R rows at a time with d/4 lanes per row, as in the merge.  A
+// coarse slot is valid only if every fine slot it covers is; an invalid one
+// is marked and left unwritten.
+template <int D, bool SB>
+__global__ void __launch_bounds__(kThreads, SB ? 3 : 4)
+compose_kernel(DevGeom fine, DevGeom coarse, const char *__restrict__ fO,
+               const float *__restrict__ flse, const unsigned char *__restrict__ fvalid,
+               char *__restrict__ cO, float *__restrict__ clse, unsigned char *cvalid) {
+  constexpr int G4 = D / 4;                 // lanes carrying one row
+  constexpr int ES = SB ? 2 : 4;
+  constexpr size_t ROWB = (size_t)D * ES;
+  const int cslot = blockIdx.y;
+  const int bh = blockIdx.z;
+  int i = 0;
+  while (i + 1 < coarse.P && coarse.row_start[i + 1] <= cslot) ++i;
+  unsigned long long m = coarse.row_mask[i];
+  for (int t = cslot - coarse.row_start[i]; t > 0; --t) m &= m - 1;
+  const int C = __ffsll((long long)m) - 1;
+  const int Li = coarse.part_off[i + 1] - coarse.part_off[i];
+  const int r0 = blockIdx.x * kRowsPerBlock;
+  if (r0 >= Li) return;
+  // the fine units inside C that are active: consecutive fine slots
+  int fs0 = -1, nf = 0;
+  for (int c = 0; c < fine.G; ++c) {
+    if (fine.group_off[c] < coarse.group_off[C] || fine.group_off[c + 1] > coarse.group_off[C + 1]) continue;
+    if (!((fine.row_mask[i] >> c) & 1ull)) continue;
+    if (fs0 < 0) fs0 = slot_of(fine, i, c);
+    ++nf;
+  }
+  bool valid = nf > 0;
+  if (fvalid)
+    for (int a = 0; a < nf; ++a) valid = valid && fvalid[fs0 + a] != 0;
+  if (cvalid && bh == 0 && blockIdx.x == 0) cvalid[cslot] = valid ? 1 : 0;
+  if (!valid) return;   // uniform per block
+
+  const size_t blk = (size_t)fine.BH * fine.Lmax;
+  const size_t base = (size_t)bh * fine.Lmax;
+  const char *srcO = fO + ((size_t)fs0 * blk + base) * ROWB;   // fine slot a: + a * blk * ROWB
+  const float *srcl = flse + (size_t)fs0 * blk + base;
+  char *dstO = cO + ((size_t)cslot * blk + base) * ROWB;
+  float *dstl = clse + (size_t)cslot * blk + base;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rend = (r0 + kRowsPerBlock < Li) ? r0 + kRowsPerBlock : Li;
+  const bool act = lane < G4;
+  constexpr int R = SB ? 4 : 2;
+  for (int r = r0 + R * warp; r < rend; r += R * kWarps) {
+    float l0[R], l1[R];
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      const bool ok = (r + q) < rend;
+      l0[q] = (ok && lane < nf) ? __ldg(srcl + (size_t)lane * blk + r + q) : -INFINITY;
+      l1[q] = (ok && lane + 32 < nf) ? __ldg(srcl + (size_t)(lane + 32) * blk + r + q) : -INFINITY;
+    }
+    typename Raw4<SB>::T v[R][kBatch];
+    float w0[R], w1[R], L[R];
+    float4 acc[R];
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      lse_weights(l0[q], l1[q], w0[q], w1[q], L[q]);
+      acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int a0 = 0; a0 < nf; a0 += kBatch) {
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+        for (int q = 0; q < R; ++q) {
+          v[q][u] = zero_raw4<SB>();
+          if (act && a0 + u < nf && (r + q) < rend)
+            v[q][u] = load_raw4<SB>(srcO + ((size_t)(a0 + u) * blk + r + q) * ROWB + lane * 4 * ES);
+        }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int a = a0 + u;
+#pragma unroll
+        for (int q = 0; q < R; ++q) {
+          const float wq = __shfl_sync(0xffffffffu, (a < 32) ? w0[q] : w1[q], a & 31);
+          if (a < nf) fma4(acc[q], wq, widen4<SB>(v[q][u]));
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      if ((r + q) >= rend) continue;
+      if (act) store_out(dstO, SB ? 0 : 1, (size_t)(r + q) * D + lane * 4, acc[q]);
+      if (lane == 0) dstl[r + q] = L[q];
+    }
+  }
 }
 
 }  // namespace merge
@@ -366,6 +462,34 @@ cudaError_t launch_cache_update(const DevGeom &g, const signed char *plan, const
       g, plan, static_cast<const char *>(part_O), part_lse, static_cast<char *>(cache_O), cache_lse,
       cache_valid, row_bytes);
   return cudaGetLastError();
+}
+
+cudaError_t launch_cache_compose(const DevGeom &fine, const DevGeom &coarse, const void *fine_O,
+                                 const float *fine_lse, const unsigned char *fine_valid,
+                                 void *coarse_O, float *coarse_lse, unsigned char *coarse_valid,
+                                 int state_bf16, cudaStream_t stream) {
+  if (coarse.n_active == 0) return cudaSuccess;
+  dim3 grid((coarse.Lmax + merge::kRowsPerBlock - 1) / merge::kRowsPerBlock, coarse.n_active,
+            coarse.BH);
+  switch (coarse.d) {
+#define DITANGO_COMPOSE(DD)                                                                      \
+  case DD:                                                                                       \
+    if (state_bf16)                                                                              \
+      merge::compose_kernel<DD, true><<<grid, merge::kThreads, 0, stream>>>(                     \
+          fine, coarse, static_cast<const char *>(fine_O), fine_lse, fine_valid,                 \
+          static_cast<char *>(coarse_O), coarse_lse, coarse_valid);                              \
+    else                                                                                         \
+      merge::compose_kernel<DD, false><<<grid, merge::kThreads, 0, stream>>>(                    \
+          fine, coarse, static_cast<const char *>(fine_O), fine_lse, fine_valid,                 \
+          static_cast<char *>(coarse_O), coarse_lse, coarse_valid);                              \
+    return cudaGetLastError();
+    DITANGO_COMPOSE(64)
+    DITANGO_COMPOSE(96)
+    DITANGO_COMPOSE(128)
+#undef DITANGO_COMPOSE
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace ditango

@@ -1,17 +1,20 @@
 // Fresh-versus-reuse plan (DiTango, "Riepilogo Tecnico" -> Metodologia ->
 // 1. Anchor-Guided Selection Planner).
 //
-// Stage 1 (mass_partial_kernel): importance of each active pair from the
+// The candidates are units (query partition i, KV group c); without KV
+// groups a unit is the pair (i, j) ("Strategia per Gruppi": decisions per
+// group of adjacent partitions).
+// Stage 1 (mass_partial_kernel): importance of each active unit from the
 // cached log-sum-exps.  For every cached row r of query partition i the
-// share of pair (i, j) in that row's softmax denominator is
-//   e_j / sum_j' e_j',  e_j = exp(lse_ij[r] - max_j' lse_ij'[r]),
+// share of unit (i, c) in that row's softmax denominator is
+//   e_c / sum_c' e_c',  e_c = exp(lse_ic[r] - max_c' lse_ic'[r]),
 // and each block sums these shares over a fixed chunk of (b*h, r) rows with
 // a fixed-order tree (warp shuffles, then warps in index order).  Invalid
 // (never written) slots hold no mass.
 // Stage 2 (plan_select_kernel, one block): chunk sums are added in chunk
 // order in double precision and divided by the row count (w = mean share),
-// then the band, the invalid slots and the top-w pairs up to the budget are
-// marked fresh.  Ranking sorts 64-bit keys (~bits(w) << 32 | i*P + j) with a
+// then the band, the invalid slots and the top-w units up to the budget are
+// marked fresh.  Ranking sorts 64-bit keys (~bits(w) << 32 | i*G + c) with a
 // bitonic network: larger w first, ties to the lower linear index.
 // Everything is deterministic; no floating-point atomics.
 #include "common.cuh"
@@ -80,7 +83,7 @@ mass_partial_kernel(DevGeom g, const float *__restrict__ cache_lse,
 #pragma unroll
   for (int t = 0; t < kRowsPerThread; ++t) rinv[t] = (rinv[t] > 0.f) ? 1.f / rinv[t] : 0.f;
 
-  // pass 2: per active pair, the block's sum of shares
+  // pass 2: per active unit, the block's sum of shares
   __shared__ float warp_part[kMassThreads / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned long long m = mask;
@@ -101,7 +104,7 @@ mass_partial_kernel(DevGeom g, const float *__restrict__ cache_lse,
     if (threadIdx.x == 0) {
       float s = 0.f;
       for (int w = 0; w < kMassThreads / 32; ++w) s += warp_part[w];
-      partial[((size_t)i * nchunks_max + chunk) * g.P + j] = s;
+      partial[((size_t)i * nchunks_max + chunk) * g.G + j] = s;
     }
     __syncthreads();
   }
@@ -116,8 +119,8 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial, int nchunks_max
   __shared__ unsigned char fresh[kMaxP * kMaxP];
   __shared__ int scan[kSelThreads / 32];
   __shared__ int n_forced;
-  const int P = g.P;
-  const int PP = P * P;
+  const int G = g.G;
+  const int PP = g.P * G;
   int n = 1;
   while (n < PP) n <<= 1;
   if (threadIdx.x == 0) n_forced = 0;
@@ -127,22 +130,21 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial, int nchunks_max
   for (int p = threadIdx.x; p < n; p += kSelThreads) {
     unsigned long long key = ~0ull;
     if (p < PP) {
-      const int i = p / P, j = p - (p / P) * P;
-      const bool act = (g.row_mask[i] >> j) & 1ull;
+      const int i = p / G, c = p - (p / G) * G;
+      const bool act = (g.row_mask[i] >> c) & 1ull;
       bool f = false;
       float w = 0.f;
       if (act) {
-        const int slot = slot_of(g, i, j);
+        const int slot = slot_of(g, i, c);
         const bool valid = cache_valid == nullptr || cache_valid[slot] != 0;
-        const int dij = i > j ? i - j : j - i;
         if (!anchor) {
           const int Li = g.part_off[i + 1] - g.part_off[i];
           const int nch = (int)(((long long)g.BH * Li + kRowsPerBlock - 1) / kRowsPerBlock);
           double acc = 0.0;
-          for (int c = 0; c < nch; ++c) acc += (double)partial[((size_t)i * nchunks_max + c) * P + j];
+          for (int ch = 0; ch < nch; ++ch) acc += (double)partial[((size_t)i * nchunks_max + ch) * G + c];
           w = (float)(acc / ((double)g.BH * Li));
         }
-        if (anchor || dij <= band_k || !valid) {
+        if (anchor || !valid || unit_in_band(g, i, c, band_k)) {
           f = true;
           ++my_forced;
         } else {
@@ -206,8 +208,8 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial, int nchunks_max
   __syncthreads();
   int pos = incl - cnt + (warp > 0 ? scan[warp - 1] : 0);
   for (int p = p0; p < p0 + per && p < PP; ++p) {
-    const int i = p / P, j = p - (p / P) * P;
-    const bool act = (g.row_mask[i] >> j) & 1ull;
+    const int i = p / G, c = p - (p / G) * G;
+    const bool act = (g.row_mask[i] >> c) & 1ull;
     plan_out[p] = fresh[p] ? (signed char)DITANGO_PLAN_FRESH
                            : (act ? (signed char)DITANGO_PLAN_REUSE : (signed char)DITANGO_PLAN_SKIP);
     if (fresh[p]) fresh_list[pos++] = p;
@@ -223,7 +225,7 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial, int nchunks_max
 size_t plan_workspace_bytes(const DevGeom &g) {
   const int nchunks_max =
       (int)(((long long)g.BH * g.Lmax + plan::kRowsPerBlock - 1) / plan::kRowsPerBlock);
-  return (size_t)g.P * nchunks_max * g.P * sizeof(float);
+  return (size_t)g.P * nchunks_max * g.G * sizeof(float);
 }
 
 cudaError_t launch_plan(const DevGeom &g, const float *cache_lse, const unsigned char *cache_valid,

@@ -5,6 +5,7 @@ from __future__ import annotations
 import numpy as np
 
 from oracle import attention as OA
+from oracle import groups as OG
 from oracle import masks as OM
 from oracle import step as OS
 from oracle.plan import PLAN_FRESH, PLAN_REUSE
@@ -58,24 +59,33 @@ def slabs(w, b, h, with_prev=True):
 
 
 def oracle_rows(w, plan, b, h, i, rows):
-    """Final (O, lse) and per-pair states of the given rows of partition i."""
+    """Final (O, lse) and per-pair states of the given rows of partition i
+    (states only without KV groups)."""
     q, k, v, kp, vp = slabs(w, b, h)
+    if w.grouped:
+        O, lse = OG.step_rows_units(q, k, v, kp, vp, plan, w.part_off(), w.group_off(), i, rows,
+                                    w.frame_off(), w.frame_mask())
+        return O, lse, None
     return OS.step_rows(q, k, v, kp, vp, plan, w.part_off(), i, rows,
                         w.frame_off(), w.frame_mask())
 
 
+def unit_masks(w):
+    """(active, band) masks over the plan's columns (KV partitions or groups)."""
+    A = OM.pair_mask(w.part_off(), w.frame_off(), w.frame_mask())
+    go = w.group_off()
+    return OG.unit_mask(A, go), OG.unit_band(A, go, w.band_k)
+
+
 def check_plan_valid(w, plan):
-    """Plan properties that hold for any w: skip exactly the masked pairs,
+    """Plan properties that hold for any w: skip exactly the masked units,
     band fresh, fresh count = max(|band|, floor(budget*|A|+1e-9))."""
     from oracle.plan import budget_target
-    A = OM.pair_mask(w.part_off(), w.frame_off(), w.frame_mask())
-    P = w.P
-    plan = np.asarray(plan).reshape(P, P)
+    A, band = unit_masks(w)
+    plan = np.asarray(plan).reshape(A.shape)
     assert ((plan != 0) == A).all()
     if w.anchor:
         assert (plan[A] == PLAN_FRESH).all()
         return
-    ii, jj = np.indices((P, P))
-    band = A & (np.abs(ii - jj) <= w.band_k)
     assert (plan[band] == PLAN_FRESH).all()
     assert int((plan == PLAN_FRESH).sum()) == budget_target(band.sum(), A.sum(), w.budget)

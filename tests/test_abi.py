@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 
 import sparse_state_reuse_b200 as dt
-from oracle import masks
+from oracle import groups, masks
 from workloads import configs
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "ditango.h")
@@ -38,8 +38,11 @@ def test_version_and_status_strings():
 
 @pytest.mark.parametrize("w", configs.ALL, ids=lambda w: w.name)
 def test_active_pairs_and_slots_match_oracle(w):
-    g = dt.Geometry(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask())
+    go = w.group_off() if w.grouped else None
+    g = dt.Geometry(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask(), group_off=go)
     A = masks.pair_mask(w.part_off(), w.frame_off(), w.frame_mask())
+    if go is not None:
+        A = groups.unit_mask(A, go)
     assert dt.ditango_check_geom(g) == 0
     assert dt.ditango_num_active(g) == int(A.sum())
     assert dt.ditango_state_rows(g) == w.Lp
@@ -88,3 +91,34 @@ def test_calls_reject_bad_arguments_before_launching():
     with pytest.raises(dt.DitangoError):
         dt.ditango_selftest_bounded_wait(0, 16, stream=0)
     assert dt.ditango_plan_workspace_size(g) > 0
+
+
+@pytest.mark.parametrize("go", [[0, 1, 3, 6, 24], [0, 24], [0, 2, 4, 8, 16, 24], list(range(25))])
+def test_unit_slots_match_oracle(go):
+    w = configs.LONG_VIDEO
+    g = dt.Geometry(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask(), group_off=go)
+    Au = groups.unit_mask(masks.pair_mask(w.part_off(), w.frame_off(), w.frame_mask()), go)
+    assert dt.ditango_num_active(g) == int(Au.sum())
+    assert (np.array(dt.ditango_slot_table(g)) == masks.slot_table(Au)).all()
+
+
+@pytest.mark.parametrize("go,status", [([0, 2, 2, 4], 1), ([0, 2, 3], 1), ([1, 4], 1), ([0, 4], 0),
+                                       ([0, 1, 2, 3, 4], 0)])
+def test_group_validation(go, status):
+    g = dt.Geometry(1, 2, 64, 64, [0, 16, 32, 48, 64], group_off=go)
+    assert dt.ditango_check_geom(g) == status
+
+
+def test_compose_rejects_bad_groupings_before_launching():
+    po = [0, 16, 32, 48, 64]
+    fine = dt.Geometry(1, 2, 64, 64, po, group_off=[0, 2, 4])
+    with pytest.raises(dt.DitangoError) as e:   # [0, 1, 4] is not a coarsening of [0, 2, 4]
+        dt.ditango_cache_compose(fine, dt.Geometry(1, 2, 64, 64, po, group_off=[0, 1, 4]),
+                                 16, 16, None, 4096, 4096, None, stream=0)
+    assert e.value.status == 1
+    with pytest.raises(dt.DitangoError):        # a different attention call
+        dt.ditango_cache_compose(fine, dt.Geometry(1, 3, 64, 64, po, group_off=[0, 4]),
+                                 16, 16, None, 4096, 4096, None, stream=0)
+    with pytest.raises(dt.DitangoError):        # overlapping state buffers
+        dt.ditango_cache_compose(fine, dt.Geometry(1, 2, 64, 64, po, group_off=[0, 4]),
+                                 16, 16, None, 16, 16, None, stream=0)

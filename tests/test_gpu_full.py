@@ -8,6 +8,7 @@ import pytest
 torch = pytest.importorskip("torch")
 
 import sparse_state_reuse_b200 as dt
+from oracle import groups as OG
 from oracle import masks as OM
 from oracle.plan import PLAN_FRESH, PLAN_REUSE, mass_scores, select, budget_target
 from workloads import configs, inputs
@@ -32,7 +33,8 @@ def sample_rows(w, i, n=24):
 def run_workload(w, out_dtype=torch.float32, state_bf16=False):
     Q, K, V = G.upload(w)
     pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask(),
-                                 state_bf16=state_bf16)
+                                 state_bf16=state_bf16,
+                                 group_off=w.group_off() if w.grouped else None)
     if w.reuses:
         Kp, Vp = G.upload_prev(w)
         pa.plan_step(anchor=True)
@@ -48,12 +50,13 @@ def run_workload(w, out_dtype=torch.float32, state_bf16=False):
 
 @pytest.mark.parametrize("w,sb", [(configs.FRAME_TILE, False), (configs.DITANGO_REUSE, False),
                                   (configs.LONG_VIDEO, False), (configs.DENSE, False),
-                                  (configs.DITANGO_REUSE, True), (configs.LONG_VIDEO, True)],
+                                  (configs.DITANGO_REUSE, True), (configs.LONG_VIDEO, True),
+                                  (configs.DITANGO_GROUPS, False)],
                          ids=["frame_tile", "reuse_p32", "long_video", "dense",
-                              "reuse_p32_bf16_cache", "long_video_bf16_cache"])
+                              "reuse_p32_bf16_cache", "long_video_bf16_cache", "groups_p32_g4"])
 def test_full_size_sampled_rows(w, sb):
     pa, out, out_lse = run_workload(w, state_bf16=sb)
-    plan = pa.plan.cpu().numpy().reshape(w.P, w.P)
+    plan = pa.plan.cpu().numpy().reshape(w.P, w.G)
     G.check_plan_valid(w, plan)
     counts = pa.counts.cpu().numpy()
     assert counts[0] == int((plan == PLAN_FRESH).sum())
@@ -122,3 +125,36 @@ def test_plan_full_size_synthetic_cache(w, invalid):
         i, j = pairs[s]
         assert got[i, j] == PLAN_FRESH
     assert counts.cpu().numpy()[0] == int((got == PLAN_FRESH).sum())
+
+
+@pytest.mark.parametrize("sb", [False, True], ids=["fp32_cache", "bf16_cache"])
+def test_compose_full_size_sampled_rows(sb):
+    """The 32-partition cache (1024 pair states) composed into 8 groups of 4
+    KV partitions on the GPU, against the oracle's group states on K/V."""
+    w = configs.DITANGO_REUSE
+    Q, K, V = G.upload(w)
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), state_bf16=sb)
+    pa.plan_step(anchor=True)
+    pa.partial(Q, K, V)
+    del Q, K, V
+    go = OG.uniform_group_off(w.P, 4)
+    coarse = pa.compose(go)
+    torch.cuda.synchronize()
+    assert pa.status.item() == 0
+    assert coarse.n_slots == w.P * 8 and bool(coarse.valid.all())
+    del pa
+    slot = OM.slot_table(OG.unit_mask(np.ones((w.P, w.P), bool), go))
+    for bh in sorted({0, w.BH - 1}):
+        b, h = divmod(bh, w.H)
+        q, k, v, _, _ = G.slabs(w, b, h, with_prev=False)
+        for i in sorted({0, 13, w.P - 1}):
+            rows = sample_rows(w, i)
+            loc = rows - w.part_off()[i]
+            for c in sorted({0, i // 4, 7}):
+                Oo, lo = OG.unit_state(q[rows], rows, k, v, w.part_off(), go, c)
+                s = int(slot[i, c])
+                idx = torch.as_tensor(loc, device="cuda")
+                G.assert_close(coarse.state_O[s, bh].index_select(0, idx).float().cpu().numpy(), Oo,
+                               f"composed O unit {(i, c)} bh {bh}")
+                G.assert_close(coarse.state_lse[s, bh].index_select(0, idx).cpu().numpy(), lo,
+                               f"composed lse unit {(i, c)} bh {bh}")
