@@ -492,10 +492,15 @@ def main():
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     ap.add_argument("--state-bf16", action="store_true",
                     help="compressed attention-state cache: O stored as bf16")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="replace the workload's head count (a reduced case for profiling; "
+                         "the line then names the reduced H and is not the workload's figure)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = configs.BY_NAME[args.workload]
+    if args.heads > 0 and args.heads != w.H:
+        w = configs.scaled(w, H=args.heads, name=f"{w.name}@H{args.heads}")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -514,10 +519,11 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     try:
         res = run_ours(args, w, rank, world, local_rank)
-        if rank == 0 and world == 1:
-            f, s, desc = oracle_sample(w, 5, 128, args.cpu_baseline_seconds)
-            res["cpu_baseline"] = {"value": round(f / s / 1e12, 6), "unit": "TFLOP/s",
-                                   "cores": blas_threads(), "kind": "oracle", "sample": desc}
+        if rank == 0:
+            if world == 1:
+                f, s, desc = oracle_sample(w, 5, 128, args.cpu_baseline_seconds)
+                res["cpu_baseline"] = {"value": round(f / s / 1e12, 6), "unit": "TFLOP/s",
+                                       "cores": blas_threads(), "kind": "oracle", "sample": desc}
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:
