@@ -26,10 +26,13 @@ Parity status per function:
   attention.partial_state, attention.merge_states, attention.dense_attention,
   masks.*, plan.select, plan.mass_scores, step.*, groups.*
   -- pinned (tests/test_oracle_*.py)
+  error_plan.* -- its rules and their invariants pinned
+  (tests/test_oracle_error_plan.py); the error model's predictive quality
+  -- parity unpinned: the pages give no formula and no values.
   The quality of reuse (how far a reuse step drifts from an all-fresh step)
   -- parity unpinned: the pages print no error values; it is reported only.
 """
 from .attention import partial_state, merge_states, dense_attention  # noqa: F401
 from .masks import pair_mask, slot_table, token_allowed, frame_of  # noqa: F401
 from .plan import mass_scores, select, budget_target, PLAN_SKIP, PLAN_FRESH, PLAN_REUSE  # noqa: F401
-from . import step, groups  # noqa: F401
+from . import step, groups, error_plan  # noqa: F401

@@ -7,7 +7,10 @@ the whole tensor.  Values are N(0, 1) in float32, optionally plus a per-frame
 shared component (amplitude * one N(0, 1) vector per (tensor, b, h, frame)),
 then rounded to bfloat16 (round to nearest, ties to even).  The previous
 denoising step's K/V are bf16(current + sigma * N(0, 1)) from a separate
-stream keyed by the drift seed.
+stream keyed by the drift seed.  A multi-step sequence (denoising steps
+s = 0, 1, ...) keeps Q fixed and lets K/V walk: step s adds
+sigma * (e_1 + ... + e_s) to the workload's tensor in float32, one N(0, 1)
+stream per (drift seed, tensor, b, h, step), then rounds to bf16.
 
 Nothing here computes attention, plans or merges.
 """
@@ -68,6 +71,34 @@ def prev_slab(w: Workload, which: str, b: int, h: int) -> np.ndarray:
 def slab_f64(w: Workload, which: str, b: int, h: int, prev: bool = False) -> np.ndarray:
     bits = prev_slab(w, which, b, h) if prev else slab(w, which, b, h)
     return bf16_to_f32(bits).astype(np.float64)
+
+
+def step_slabs(w: Workload, which: str, b: int, h: int, steps: int):
+    """bf16 bits [N, d] of K or V at denoising steps 0..steps of the walk."""
+    assert which in ("k", "v")
+    x = bf16_to_f32(slab(w, which, b, h))
+    out = [bf16_bits(x)]
+    acc = np.zeros_like(x)
+    for s in range(1, steps + 1):
+        acc += _rng(w.drift_seed, TENSOR_ID[which], b, h, 1000 + s).standard_normal(
+            (w.N, w.d), dtype=np.float32)
+        out.append(bf16_bits(x + np.float32(w.drift_sigma) * acc))
+    return out
+
+
+def step_full(w: Workload, which: str, steps: int, threads: int = 0):
+    """bf16 bits [steps + 1, B, H, N, d] of K or V along the walk."""
+    out = np.empty((steps + 1, w.B, w.H, w.N, w.d), dtype=np.uint16)
+
+    def work(bh):
+        b, h = divmod(bh, w.H)
+        for s, x in enumerate(step_slabs(w, which, b, h, steps)):
+            out[s, b, h] = x
+
+    threads = threads or min(16, os.cpu_count() or 1)
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(work, range(w.BH)))
+    return out
 
 
 def full(w: Workload, which: str, prev: bool = False, threads: int = 0) -> np.ndarray:
