@@ -359,7 +359,83 @@ def run_ours(args, w, rank, world, local_rank):
     }
     if compose is not None:
         res["compose"] = compose
+    if args.schedule > 0:
+        del pa
+        torch.cuda.empty_cache()
+        res["schedule"] = measure_schedule(w, args, dev, stream, Q, K, V, flops)
     return res
+
+
+def measure_schedule(w, args, dev, stream, Q, K0, V0, plain_flops):
+    """A run of denoising steps with the error-growth planner (DiTango,
+    1. Anchor-Guided Selection Planner): anchor steps every --anchor-every
+    steps, predicted-error reuse between them.  K/V walk from step to step
+    (K_s = bf16(K_0 + sigma * (e_1 + ... + e_s)), drawn on the device with
+    torch's seeded generator, outside the timed region).  For every step it
+    times the error planner's step, and the w planner's step on the same
+    inputs, and reports each output's mean |difference| from unpartitioned
+    all-fresh attention (computed by the library with one partition) -- the
+    quality of reuse, reported and not gated."""
+    import torch
+    import sparse_state_reuse_b200 as dt
+    go = w.group_off() if w.grouped else None
+    mk = lambda **kw: dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(),  # noqa: E731
+                                              w.frame_mask(), device=dev, state_bf16=args.state_bf16,
+                                              **kw)
+    pa_e = mk(group_off=go)
+    pa_w = mk(group_off=go)
+    ep = dt.ErrorPlanner(pa_e, w.band_k, w.budget, args.anchor_every)
+    # one partition: unpartitioned attention (unavailable under a frame mask,
+    # which needs partitions inside frames)
+    dense = None if w.F else dt.PartitionedAttention(w.B, w.H, w.N, w.d, [0, w.N], device=dev)
+    outs = {k: torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device=dev) for k in "ewf"}
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.drift_seed * 1000 + 17)
+    K0f, V0f = K0.float(), V0.float()
+    accK, accV = torch.zeros_like(K0f), torch.zeros_like(V0f)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    rows = []
+    for s in range(args.schedule + 1):
+        if s > 0:
+            accK.add_(torch.randn(accK.shape, generator=gen, device=dev))
+            accV.add_(torch.randn(accV.shape, generator=gen, device=dev))
+        K = (K0f + w.drift_sigma * accK).to(torch.bfloat16)
+        V = (V0f + w.drift_sigma * accV).to(torch.bfloat16)
+        stream.wait_stream(torch.cuda.current_stream())    # K/V were made on the default stream
+        anchor = ep.is_anchor(s)
+        e = [ev() for _ in range(4)]
+        with torch.cuda.stream(stream):
+            e[0].record(stream)
+            ep.step(Q, K, V, outs["e"], stream=stream)
+            e[1].record(stream)
+            pa_w.step(Q, K, V, outs["w"], band_k=w.band_k, budget=w.budget, anchor=anchor,
+                      stream=stream)
+            e[2].record(stream)
+            if dense is not None:
+                dense.step(Q, K, V, outs["f"], anchor=True, stream=stream)
+        stream.synchronize()
+        fresh_e = pa_e.plan.cpu().numpy().reshape(w.P, pa_e.G) == 1
+        fl = effective_flops(w, fresh_pairs_of_units(w, np.where(fresh_e, 1, 0), pair_mask(w)))
+        row = {"step": s, "anchor": bool(anchor), "error_planner_ms": round(e[0].elapsed_time(e[1]), 4),
+               "w_planner_ms": round(e[1].elapsed_time(e[2]), 4),
+               "error_planner_tflops": round(fl / (e[0].elapsed_time(e[1]) * 1e-3) / 1e12, 2),
+               "mean_local_drift": float(ep.delta.mean().item())}
+        if dense is not None:
+            row["error_planner_err"] = float((outs["e"] - outs["f"]).abs().mean().item())
+            row["w_planner_err"] = float((outs["w"] - outs["f"]).abs().mean().item())
+        rows.append(row)
+    if int(pa_e.status.item()) != 0 or int(pa_w.status.item()) != 0:
+        raise RuntimeError("device status in the schedule")
+    reuse = [r for r in rows if not r["anchor"]]
+    summary = {"steps": args.schedule + 1, "anchor_every": args.anchor_every,
+               "sigma_per_step": w.drift_sigma,
+               "mean_error_planner_ms_reuse_steps": round(float(np.mean([r["error_planner_ms"] for r in reuse])), 4),
+               "mean_w_planner_ms_reuse_steps": round(float(np.mean([r["w_planner_ms"] for r in reuse])), 4),
+               "per_step": rows}
+    if dense is not None:
+        summary["mean_abs_err_vs_fresh_error_planner"] = float(np.mean([r["error_planner_err"] for r in reuse]))
+        summary["mean_abs_err_vs_fresh_w_planner"] = float(np.mean([r["w_planner_err"] for r in reuse]))
+    return summary
 
 
 def measure_compose(w, pa, Q, K, V, dev, stream, args, peaks):
@@ -492,6 +568,10 @@ def main():
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     ap.add_argument("--state-bf16", action="store_true",
                     help="compressed attention-state cache: O stored as bf16")
+    ap.add_argument("--schedule", type=int, default=0,
+                    help="also run this many denoising steps with the error-growth planner "
+                         "(K/V drifting step by step) and report them under 'schedule'")
+    ap.add_argument("--anchor-every", type=int, default=5)
     ap.add_argument("--heads", type=int, default=0,
                     help="replace the workload's head count (a reduced case for profiling; "
                          "the line then names the reduced H and is not the workload's figure)")

@@ -87,7 +87,7 @@ typedef void *ditango_stream; /* cudaStream_t */
  *   q/k/v_strides  element strides of the (b, h, n) dimensions of the bf16
  *            Q, K, V tensors; the d dimension is contiguous.  Strides times 2
  *            bytes must be multiples of 16 and the base pointers 16-byte
- *            aligned (TMA).
+ *            aligned (TMA).  The stride of a dimension of size 1 is ignored.
  *   G        KV groups; 0 = one group per partition (group_off ignored).
  *            Else 1 <= G <= P and group_off host int32 [G+1] holds partition
  *            indices, group_off[0] = 0 < ... < group_off[G] = P: group c is
@@ -175,6 +175,13 @@ ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
  *                method's limitation and cache compression its next step).
  *   out_valid    dev uint8 [slots] or NULL; with out_by_slot = 1 the written
  *                slots are set to 1.
+ *   drift_rows   dev float32 [P][B*H][Lmax] or NULL (needs out_by_slot = 1):
+ *                for each fresh local unit -- the unit of partition i that
+ *                holds partition i, always in the band -- row r receives
+ *                |lse_new - lse_old|, lse_old being the slot's lse before
+ *                this call overwrites it (equal values, -inf included, give
+ *                0): the local state's change that ditango_plan_error reads
+ *                (DiTango, "Predizione Online").
  *   dev_status   dev int32 or NULL; set to DITANGO_ERR_TIMEOUT if a pipeline
  *                wait exceeded the limit (the kernel then stops cleanly).
  */
@@ -183,8 +190,8 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q,
                                     const int32_t *fresh_list, const int32_t *counts,
                                     float scale, void *out_O, float *out_lse,
                                     int32_t out_by_slot, int32_t state_bf16,
-                                    uint8_t *out_valid, int32_t *dev_status,
-                                    ditango_stream stream);
+                                    uint8_t *out_valid, float *drift_rows,
+                                    int32_t *dev_status, ditango_stream stream);
 
 /* Merge: the final output of every token is the log-sum-exp composition of
  * the states of its partition's active units (DiTango, "Composizione dello
@@ -238,6 +245,51 @@ ditango_status ditango_cache_compose(const ditango_geom *fine, const ditango_geo
                                      const uint8_t *fine_valid, void *coarse_O,
                                      float *coarse_lse, uint8_t *coarse_valid,
                                      int32_t state_bf16, ditango_stream stream);
+
+/* Error-growth planner state (DiTango, 1. Anchor-Guided Selection Planner:
+ * "Modellazione dell'Errore", "Anchor Steps", "Predizione Online").  Device
+ * buffers owned by the caller, zeroed once before the first (anchor) step and
+ * then carried from step to step by ditango_plan_error. */
+typedef struct {
+  float *w;                 /* dev float32 [P*G]: importance, refreshed after anchors */
+  float *age;               /* dev float32 [slots]: local drift accumulated since each
+                               cached state was computed */
+  float *delta;             /* dev float32 [P]: last measured local drift (output) */
+  uint8_t *local_ok;        /* dev uint8 [P]: the local unit held a state before the
+                               last step's attention call */
+  const float *drift_rows;  /* dev float32 [P][B*H][Lmax]: written by
+                               ditango_attn_partial (drift_rows argument) */
+} ditango_error_state;
+
+/* Plan by predicted reuse error.  The same contract as ditango_plan (band,
+ * invalid slots, budget, fresh list, counts, workspace) with the ranking
+ * score replaced:
+ *   delta_i = mean over (b, h, rows of partition i) of drift_rows, when
+ *             local_ok[i] (else 0) -- the local state's change in the last
+ *             step, standing in for the drift of the partition's remote
+ *             states;
+ *   age     = 0 for units the previous plan made fresh, age + delta_i for
+ *             the units it reused;
+ *   score   = w * (age + delta_i): the predicted error of reusing the unit
+ *             at this step; the non-band units of largest score fill the
+ *             budget (ties to the lower index i*G + c).
+ *   plan     in: the previous step's plan (zeros before the first step);
+ *            out: this step's plan.
+ *   anchor   nonzero: every active unit fresh (an anchor step, "Anchor
+ *            Steps"); w, age and delta are left alone.
+ *   refresh_w  nonzero (the step after an anchor): w is recomputed from the
+ *            cache as in ditango_plan and stored in es->w; otherwise es->w
+ *            is used as held.
+ *   score_out  dev float32 [P*G] or NULL: the score (0 for masked units).
+ * Every call also records es->local_ok for the next step (whether the local
+ * unit's slot is valid now, before this step's attention call). */
+ditango_status ditango_plan_error(const ditango_geom *g, const float *cache_lse,
+                                  const uint8_t *cache_valid, int32_t band_k, double budget,
+                                  int32_t anchor, int32_t refresh_w,
+                                  const ditango_error_state *es, int8_t *plan,
+                                  int32_t *fresh_list, int32_t *counts, float *score_out,
+                                  void *workspace, size_t workspace_bytes,
+                                  ditango_stream stream);
 
 /* Allocation-free variant of ditango_plan (no counterpart in the papers: it
  * exists for callers, not for the method).  For callers that cannot allocate

@@ -151,9 +151,16 @@ class Schedule:
                                   for i in range(self.P)])
         return plan, score
 
-    def step(self, s, k, v):
-        """k, v: [BH][N, d] of step s.  Returns (plan, score, O [BH][N, d], lse [BH][N])."""
+    def step(self, s, k, v, plan_override=None):
+        """k, v: [BH][N, d] of step s.  Returns (plan, score, O [BH][N, d], lse [BH][N]).
+
+        plan_override: execute this plan instead of the one planned (the
+        planner state still advances from the planned scores and the
+        executed plan), so that a run of another implementation can be
+        followed step by step."""
         plan, score = self.plan(s)
+        if plan_override is not None:
+            plan = np.asarray(plan_override, dtype=np.int8).reshape(self.Au.shape)
         N, d = self.q[0].shape
         out_O = np.zeros((self.BH, N, d))
         out_l = np.full((self.BH, N), -np.inf)

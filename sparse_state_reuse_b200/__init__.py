@@ -23,6 +23,7 @@ from ._abi import (  # noqa: F401
     ditango_slot_table, ditango_plan_workspace_size, ditango_plan, ditango_attn_partial,
     ditango_merge, ditango_cache_update, ditango_set_wait_limit_ns,
     ditango_selftest_bounded_wait, ditango_plan_noalloc, ditango_cache_compose, status_string,
+    ditango_plan_error, error_state,
 )
 
 
@@ -85,11 +86,11 @@ class PartitionedAttention:
                      anchor, self.plan, self.fresh_list, self.counts, self.score, self.workspace,
                      self.ws_bytes, stream)
 
-    def partial(self, Q, K, V, scale=0.0, stream=None):
+    def partial(self, Q, K, V, scale=0.0, stream=None, drift_rows=None):
         self._bind(Q, K, V)
         ditango_attn_partial(self.geom, Q, K, V, self.fresh_list, self.counts, scale,
                              self.state_O, self.state_lse, 1, self.valid, self.status, stream,
-                             state_bf16=self.state_bf16)
+                             state_bf16=self.state_bf16, drift_rows=drift_rows)
 
     def merge(self, out, out_lse=None, stream=None):
         import torch
@@ -116,3 +117,50 @@ class PartitionedAttention:
                               coarse.state_O, coarse.state_lse, coarse.valid, self.state_bf16,
                               stream)
         return coarse
+
+
+class ErrorPlanner:
+    """Anchor-guided, error-growth planning of a PartitionedAttention's steps
+    (DiTango, 1. Anchor-Guided Selection Planner).
+
+    Step 0 and every anchor_every-th step after it are anchor steps (every
+    active unit fresh).  The step after an anchor recomputes the importance w
+    from the cache; the others hold it.  Between anchors each unit's
+    predicted reuse error w * (age + delta_i) ranks the non-band units under
+    the budget, delta_i being the local state's drift that the attention
+    call of the previous step measured.  The schedule is host logic; every
+    number is computed on the device.
+    """
+
+    def __init__(self, pa, band_k, budget, anchor_every):
+        import torch
+        if anchor_every < 1:
+            raise ValueError("anchor_every must be >= 1")
+        self.pa = pa
+        self.band_k, self.budget, self.anchor_every = band_k, budget, anchor_every
+        dev = pa.device
+        self.w = torch.zeros(pa.P * pa.G, dtype=torch.float32, device=dev)
+        self.age = torch.zeros(max(pa.n_slots, 1), dtype=torch.float32, device=dev)
+        self.delta = torch.zeros(pa.P, dtype=torch.float32, device=dev)
+        self.local_ok = torch.zeros(pa.P, dtype=torch.uint8, device=dev)
+        self.drift_rows = torch.zeros((pa.P, pa.B * pa.H, pa.Lmax), dtype=torch.float32, device=dev)
+        self.es = error_state(self.w, self.age, self.delta, self.local_ok, self.drift_rows)
+        self.step_index = 0
+
+    def is_anchor(self, s):
+        return s % self.anchor_every == 0
+
+    def plan(self, stream=None):
+        s = self.step_index
+        pa = self.pa
+        ditango_plan_error(pa.geom, pa.state_lse, pa.valid, self.band_k, self.budget,
+                           self.is_anchor(s), s > 0 and self.is_anchor(s - 1), self.es, pa.plan,
+                           pa.fresh_list, pa.counts, pa.score, pa.workspace, pa.ws_bytes, stream)
+
+    def step(self, Q, K, V, out, out_lse=None, scale=0.0, stream=None):
+        """plan by predicted error -> attention of the fresh units (measuring the
+        local drift) -> merge."""
+        self.plan(stream)
+        self.pa.partial(Q, K, V, scale, stream, drift_rows=self.drift_rows)
+        self.pa.merge(out, out_lse, stream)
+        self.step_index += 1

@@ -39,6 +39,13 @@ class ditango_geom(C.Structure):
     ]
 
 
+class ditango_error_state(C.Structure):
+    _fields_ = [
+        ("w", C.c_void_p), ("age", C.c_void_p), ("delta", C.c_void_p),
+        ("local_ok", C.c_void_p), ("drift_rows", C.c_void_p),
+    ]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -61,7 +68,10 @@ _SIGS = {
     "ditango_plan": (C.c_int, [_G, _P, _P, C.c_int32, C.c_double, C.c_int32, _P, _P, _P, _P, _P,
                                C.c_size_t, _P]),
     "ditango_attn_partial": (C.c_int, [_G, _P, _P, _P, _P, _P, C.c_float, _P, _P, C.c_int32,
-                                       C.c_int32, _P, _P, _P]),
+                                       C.c_int32, _P, _P, _P, _P]),
+    "ditango_plan_error": (C.c_int, [_G, _P, _P, C.c_int32, C.c_double, C.c_int32, C.c_int32,
+                                     C.POINTER(ditango_error_state), _P, _P, _P, _P, _P,
+                                     C.c_size_t, _P]),
     "ditango_merge": (C.c_int, [_G, _P, _P, _P, _P, _P, _P, C.c_int32, C.c_int32, _P, C.c_int32,
                                 _P, _P, _P]),
     "ditango_cache_update": (C.c_int, [_G, _P, _P, _P, _P, _P, _P, C.c_int32, _P]),
@@ -192,11 +202,25 @@ def ditango_plan(geom, cache_lse, cache_valid, band_k, budget, anchor, plan, fre
 
 def ditango_attn_partial(geom, Q, K, V, fresh_list, counts, scale, out_O, out_lse,
                          out_by_slot=0, out_valid=None, dev_status=None, stream=None,
-                         state_bf16=0):
+                         state_bf16=0, drift_rows=None):
     _check("ditango_attn_partial", _lib.ditango_attn_partial(
         geom.ref, _ptr(Q), _ptr(K), _ptr(V), _ptr(fresh_list), _ptr(counts), float(scale),
         _ptr(out_O), _ptr(out_lse), int(out_by_slot), int(bool(state_bf16)), _ptr(out_valid),
-        _ptr(dev_status), _stream(stream)))
+        _ptr(drift_rows), _ptr(dev_status), _stream(stream)))
+
+
+def error_state(w, age, delta, local_ok, drift_rows):
+    """A ditango_error_state over five device buffers (tensors or addresses)."""
+    return ditango_error_state(_ptr(w), _ptr(age), _ptr(delta), _ptr(local_ok), _ptr(drift_rows))
+
+
+def ditango_plan_error(geom, cache_lse, cache_valid, band_k, budget, anchor, refresh_w, es, plan,
+                       fresh_list, counts, score_out=None, workspace=None, workspace_bytes=0,
+                       stream=None):
+    _check("ditango_plan_error", _lib.ditango_plan_error(
+        geom.ref, _ptr(cache_lse), _ptr(cache_valid), int(band_k), float(budget),
+        int(bool(anchor)), int(bool(refresh_w)), C.byref(es), _ptr(plan), _ptr(fresh_list),
+        _ptr(counts), _ptr(score_out), _ptr(workspace), int(workspace_bytes), _stream(stream)))
 
 
 def ditango_merge(geom, plan, part_O, part_lse, cache_O, cache_lse, cache_valid, writeback,

@@ -71,6 +71,7 @@ struct Params {
   float *out_lse;
   int out_by_slot;
   unsigned char *out_valid;
+  float *drift_rows;       // [P][B*H][Lmax] local-state drift, or null
   int *dev_status;
   long long wait_limit_ns;
 };
@@ -732,7 +733,16 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           __syncwarp();
         }
       }
-      if (store && r < rows_k) p.out_lse[row_off] = (m_used + __log2f(l)) * 0.69314718055994531f;
+      if (store && r < rows_k) {
+        const float lse = (m_used + __log2f(l)) * 0.69314718055994531f;
+        if (p.drift_rows && p.g.part_group[w.i] == pr.c) {
+          // the local unit: its change since the slot was last written
+          const float old = p.out_lse[row_off];
+          p.drift_rows[((size_t)w.i * p.g.BH + w.bh) * p.g.Lmax + rloc] =
+              (lse == old) ? 0.f : fabsf(lse - old);
+        }
+        p.out_lse[row_off] = lse;
+      }
       if (store && p.out_by_slot && p.out_valid && k == 0 && r == 0) p.out_valid[idx] = 1;
      }
     }
@@ -747,8 +757,9 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const CUtensorMap &tk,
                                 const CUtensorMap &tv, const int *fresh_list, const int *counts,
                                 float scale, void *out_O, float *out_lse, int out_by_slot,
-                                int state_bf16, unsigned char *out_valid, int *dev_status,
-                                long long wait_limit_ns, int num_sms, cudaStream_t stream) {
+                                int state_bf16, unsigned char *out_valid, float *drift_rows,
+                                int *dev_status, long long wait_limit_ns, int num_sms,
+                                cudaStream_t stream) {
   attn::Params p;
   p.g = g;
   p.fresh_list = fresh_list;
@@ -758,6 +769,7 @@ cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const C
   p.out_lse = out_lse;
   p.out_by_slot = out_by_slot;
   p.out_valid = out_valid;
+  p.drift_rows = out_by_slot ? drift_rows : nullptr;
   p.dev_status = dev_status;
   p.wait_limit_ns = wait_limit_ns;
   const long long nqt2 = (g.Lmax + 255) / 256;

@@ -29,6 +29,7 @@ struct DevGeom {
   int row_start[kMaxP + 1];            // slot of the first active unit of row i
   unsigned long long row_mask[kMaxP];  // bit c set: unit (i, c) active
   unsigned long long pair_mask[kMaxP]; // bit j set: pair (i, j) active
+  signed char part_group[kMaxP];       // KV group holding partition j
 };
 
 __host__ __device__ inline int slot_of(const DevGeom &g, int i, int c) {

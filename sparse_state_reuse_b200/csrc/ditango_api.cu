@@ -12,12 +12,15 @@ namespace ditango {
 cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const CUtensorMap &tk,
                                 const CUtensorMap &tv, const int *fresh_list, const int *counts,
                                 float scale, void *out_O, float *out_lse, int out_by_slot,
-                                int state_bf16, unsigned char *out_valid, int *dev_status,
-                                long long wait_limit_ns, int num_sms, cudaStream_t stream);
+                                int state_bf16, unsigned char *out_valid, float *drift_rows,
+                                int *dev_status, long long wait_limit_ns, int num_sms,
+                                cudaStream_t stream);
 size_t plan_workspace_bytes(const DevGeom &g);
 cudaError_t launch_plan(const DevGeom &g, const float *cache_lse, const unsigned char *cache_valid,
                         int band_k, int target, int anchor, signed char *plan_out, int *fresh_list,
-                        int *counts, float *score_out, void *workspace, cudaStream_t stream);
+                        int *counts, float *score_out, void *workspace, cudaStream_t stream,
+                        const float *drift_rows, float *w_hold, float *age, float *delta,
+                        unsigned char *local_ok, int refresh_w);
 cudaError_t launch_merge(const DevGeom &g, const signed char *plan, const void *part_O,
                          const float *part_lse, void *cache_O, float *cache_lse,
                          unsigned char *cache_valid, int writeback, int state_bf16, void *out,
@@ -95,6 +98,8 @@ ditango_status make_geom(const ditango_geom *in, DevGeom *out) {
     g.G = in->G;
     for (int c = 0; c <= in->G; ++c) g.group_off[c] = in->group_off[c];
   }
+  for (int c = 0; c < g.G; ++c)
+    for (int j = g.group_off[c]; j < g.group_off[c + 1]; ++j) g.part_group[j] = (signed char)c;
   for (int i = 0; i < in->P; ++i) {
     unsigned long long m = 0;
     for (int j = 0; j < in->P; ++j) {
@@ -264,33 +269,73 @@ ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
   const int target = plan_target(&dg, band_k, budget);
   return cuda_status(launch_plan(dg, cache_lse, cache_valid, band_k, target, anchor ? 1 : 0,
                                  reinterpret_cast<signed char *>(plan), fresh_list, counts,
-                                 score_out, workspace, static_cast<cudaStream_t>(stream)));
+                                 score_out, workspace, static_cast<cudaStream_t>(stream), nullptr,
+                                 nullptr, nullptr, nullptr, nullptr, 0));
+}
+
+ditango_status ditango_plan_error(const ditango_geom *g, const float *cache_lse,
+                                  const uint8_t *cache_valid, int32_t band_k, double budget,
+                                  int32_t anchor, int32_t refresh_w,
+                                  const ditango_error_state *es, int8_t *plan,
+                                  int32_t *fresh_list, int32_t *counts, float *score_out,
+                                  void *workspace, size_t workspace_bytes,
+                                  ditango_stream stream) {
+  DevGeom dg;
+  ditango_status st = make_geom(g, &dg);
+  if (st != DITANGO_OK) return st;
+  if (!plan || !fresh_list || !counts || !es) return DITANGO_ERR_INVALID;
+  if (!es->w || !es->age || !es->delta || !es->local_ok) return DITANGO_ERR_INVALID;
+  if (!anchor) {
+    if (!es->drift_rows || band_k < 0 || !(budget >= 0.0 && budget <= 1.0))
+      return DITANGO_ERR_INVALID;
+    if (refresh_w && !cache_lse) return DITANGO_ERR_INVALID;
+    if (!workspace || workspace_bytes < plan_workspace_bytes(dg)) return DITANGO_ERR_INVALID;
+  }
+  const int target = plan_target(&dg, band_k, budget);
+  return cuda_status(launch_plan(dg, cache_lse, cache_valid, band_k, target, anchor ? 1 : 0,
+                                 reinterpret_cast<signed char *>(plan), fresh_list, counts,
+                                 score_out, workspace, static_cast<cudaStream_t>(stream),
+                                 es->drift_rows, es->w, es->age, es->delta, es->local_ok,
+                                 refresh_w ? 1 : 0));
 }
 
 ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q, const uint16_t *K,
                                     const uint16_t *V, const int32_t *fresh_list,
                                     const int32_t *counts, float scale, void *out_O,
                                     float *out_lse, int32_t out_by_slot, int32_t state_bf16,
-                                    uint8_t *out_valid, int32_t *dev_status,
+                                    uint8_t *out_valid, float *drift_rows, int32_t *dev_status,
                                     ditango_stream stream) {
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
   if (st != DITANGO_OK) return st;
   if (!Q || !K || !V || !fresh_list || !counts || !out_O || !out_lse) return DITANGO_ERR_INVALID;
+  if (drift_rows && !out_by_slot) return DITANGO_ERR_INVALID;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out_O))
     return DITANGO_ERR_INVALID;
-  if (!strides_ok(g->q_strides) || !strides_ok(g->k_strides) || !strides_ok(g->v_strides))
-    return DITANGO_ERR_INVALID;
+  // the stride of a dimension of size 1 is never used (frameworks report 0
+  // or anything for it): give it the packed value
+  int64_t qs[3], ks[3], vs[3];
+  for (int k = 0; k < 3; ++k) {
+    qs[k] = g->q_strides[k];
+    ks[k] = g->k_strides[k];
+    vs[k] = g->v_strides[k];
+  }
+  for (int64_t *s : {qs, ks, vs}) {
+    if (dg.N == 1) s[2] = dg.d;
+    if (dg.H == 1) s[1] = s[2] * dg.N;
+    if (dg.B == 1) s[0] = s[1] * dg.H;
+  }
+  if (!strides_ok(qs) || !strides_ok(ks) || !strides_ok(vs)) return DITANGO_ERR_INVALID;
   if (!(scale >= 0.f) || !std::isfinite(scale)) return DITANGO_ERR_INVALID;
   if (scale == 0.f) scale = 1.f / std::sqrt((float)dg.d);
   CUtensorMap tq, tk, tv;
-  if (!make_qkv_map(&tq, Q, dg, g->q_strides) || !make_qkv_map(&tk, K, dg, g->k_strides) ||
-      !make_qkv_map(&tv, V, dg, g->v_strides))
+  if (!make_qkv_map(&tq, Q, dg, qs) || !make_qkv_map(&tk, K, dg, ks) ||
+      !make_qkv_map(&tv, V, dg, vs))
     return DITANGO_ERR_CUDA;
   return cuda_status(launch_attn_partial(dg, tq, tk, tv, fresh_list, counts, scale, out_O, out_lse,
                                          out_by_slot ? 1 : 0, state_bf16 ? 1 : 0, out_valid,
-                                         dev_status, g_wait_limit_ns, num_sms_current(),
-                                         static_cast<cudaStream_t>(stream)));
+                                         drift_rows, dev_status, g_wait_limit_ns,
+                                         num_sms_current(), static_cast<cudaStream_t>(stream)));
 }
 
 ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan, const void *part_O,
@@ -440,5 +485,6 @@ extern "C" ditango_status ditango_plan_noalloc(const ditango_geom *g, const floa
   const int target = plan_target(&dg, band_k, budget);
   return cuda_status(launch_plan(dg, cache_lse, cache_valid, band_k, target, anchor ? 1 : 0,
                                  reinterpret_cast<signed char *>(plan), fresh_list, counts,
-                                 score_out, scratch, static_cast<cudaStream_t>(stream)));
+                                 score_out, scratch, static_cast<cudaStream_t>(stream), nullptr,
+                                 nullptr, nullptr, nullptr, nullptr, 0));
 }

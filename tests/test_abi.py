@@ -122,3 +122,30 @@ def test_compose_rejects_bad_groupings_before_launching():
     with pytest.raises(dt.DitangoError):        # overlapping state buffers
         dt.ditango_cache_compose(fine, dt.Geometry(1, 2, 64, 64, po, group_off=[0, 4]),
                                  16, 16, None, 16, 16, None, stream=0)
+
+
+def test_error_plan_rejects_bad_arguments_before_launching():
+    g = dt.Geometry(1, 2, 64, 64, [0, 32, 64])
+    es = dt.error_state(16, 16, 16, 16, None)          # no drift rows
+    with pytest.raises(dt.DitangoError) as e:
+        dt.ditango_plan_error(g, 16, None, 0, 0.5, 0, 0, es, 16, 16, 16, None, 16, 10**6, stream=0)
+    assert e.value.status == 1
+    es2 = dt.error_state(None, 16, 16, 16, 16)         # no w buffer
+    with pytest.raises(dt.DitangoError):
+        dt.ditango_plan_error(g, 16, None, 0, 0.5, 1, 0, es2, 16, 16, 16, stream=0)
+    with pytest.raises(dt.DitangoError):               # drift rows need out_by_slot
+        dt.ditango_attn_partial(g, 16, 16, 16, 16, 16, 0.0, 16, 16, 0, drift_rows=16, stream=0)
+
+
+def test_size_one_dimensions_may_have_any_stride():
+    """B = 1 with a 0 batch stride (numpy/torch broadcast views) passes the
+    argument checks: only the CUDA stage can fail here (no GPU)."""
+    g = dt.Geometry(1, 2, 64, 64, [0, 32, 64], q_strides=(0, 4096, 64), k_strides=(0, 4096, 64),
+                    v_strides=(0, 4096, 64))
+    with pytest.raises(dt.DitangoError) as e:
+        dt.ditango_attn_partial(g, 4096, 4096, 4096, 4096, 4096, 0.0, 4096, 4096, 1, stream=0)
+    assert e.value.status != 1
+    g2 = dt.Geometry(2, 2, 64, 64, [0, 32, 64], q_strides=(0, 4096, 64))   # B = 2: a real stride
+    with pytest.raises(dt.DitangoError) as e:
+        dt.ditango_attn_partial(g2, 4096, 4096, 4096, 4096, 4096, 0.0, 4096, 4096, 1, stream=0)
+    assert e.value.status == 1

@@ -1,0 +1,104 @@
+"""GPU parity of the error-growth planner with anchor scheduling (DiTango,
+1. Anchor-Guided Selection Planner) against oracle.error_plan.Schedule over
+a drifting multi-step schedule.
+
+Per step: the plan equals the oracle's selection run on the GPU's own score
+array (bit for bit: the hard gate where floating point decides an integer);
+the local drift delta, the held importance w, the ages and the scores agree
+with the oracle's fp64 values within tolerances derived from fp32 log-sum-
+exps; the merged output agrees with the oracle (max-abs 2e-2, mean-abs 2e-3).
+The oracle follows the plan the GPU executed, so that both caches hold states
+of the same steps.  Whether the oracle, left alone, would pick the same units
+is reported (it may differ only where scores tie within fp32 resolution)."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import sparse_state_reuse_b200 as dt
+from oracle import error_plan as E
+from oracle import masks as OM
+from oracle.plan import PLAN_FRESH, select
+from workloads import configs, inputs
+
+import gpu_common as G
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+
+def to_dev(bits):
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+
+
+@pytest.mark.parametrize("gs,frames", [(0, False), (2, False), (0, True)], ids=["pairs", "groups2", "frame_tile"])
+def test_schedule_matches_oracle(gs, frames):
+    F = 6 if frames else 0
+    w = configs.scaled(configs.TINY, N=1536, P=6, d=64, H=2, drift_sigma=0.05, budget=0.5 if not frames else 0.7,
+                       band_k=0, group_size=gs, F=F, frame_component=0.5 if frames else 0.0,
+                       seed=31, drift_seed=131, name="error_schedule")
+    S, every = 8, 4
+    po, go = w.part_off(), w.group_off()
+    fo, fm = w.frame_off(), w.frame_mask()
+    q_bits = [inputs.slab(w, "q", 0, h) for h in range(w.H)]
+    k_steps = [inputs.step_slabs(w, "k", 0, h, S) for h in range(w.H)]
+    v_steps = [inputs.step_slabs(w, "v", 0, h, S) for h in range(w.H)]
+    f64 = lambda b: inputs.bf16_to_f32(b).astype(np.float64)  # noqa: E731
+    A = OM.pair_mask(po, fo, fm)
+    sch = E.Schedule([f64(x) for x in q_bits], po, go, A, w.band_k, w.budget, every, fo, fm)
+    Au, band = sch.Au, sch.band
+
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, po, fo, fm, group_off=go if gs else None)
+    ep = dt.ErrorPlanner(pa, w.band_k, w.budget, every)
+    Q = to_dev(np.stack(q_bits)[None])
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    out_lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
+    agree = 0
+    for s in range(S + 1):
+        K = to_dev(np.stack([k_steps[h][s] for h in range(w.H)])[None])
+        V = to_dev(np.stack([v_steps[h][s] for h in range(w.H)])[None])
+        ep.step(Q, K, V, out, out_lse)
+        torch.cuda.synchronize()
+        assert pa.status.item() == 0
+        plan_g = pa.plan.cpu().numpy().reshape(Au.shape)
+        score_g = pa.score.cpu().numpy().reshape(Au.shape)
+        plan_o, score_o, O_o, l_o = sch.step(s, [f64(k_steps[h][s]) for h in range(w.H)],
+                                             [f64(v_steps[h][s]) for h in range(w.H)], plan_override=plan_g)
+        if s % every == 0:
+            assert (plan_g[Au] == PLAN_FRESH).all()
+        else:
+            # hard gate: the selection rule on the GPU's own scores is the GPU plan
+            valid_pp = np.ones(Au.shape, dtype=bool)
+            sel, _ = select(score_g.astype(np.float64), Au, 0, w.budget, band=band, valid=valid_pp)
+            assert (sel == plan_g).all(), (s, sel, plan_g)
+            d_g = ep.delta.cpu().numpy()
+            np.testing.assert_allclose(d_g, sch.delta, rtol=2e-2, atol=1e-4, err_msg=f"delta step {s}")
+            if s > 1:
+                assert (d_g > 0).all()
+            np.testing.assert_allclose(ep.w.cpu().numpy().reshape(Au.shape), sch.w, rtol=1e-3, atol=1e-6,
+                                       err_msg=f"w step {s}")
+            np.testing.assert_allclose(ep.age.cpu().numpy()[:len(sch.age)], sch.age, rtol=3e-2, atol=3e-4,
+                                       err_msg=f"age step {s}")
+            np.testing.assert_allclose(score_g, score_o, rtol=3e-2, atol=1e-5, err_msg=f"score step {s}")
+            agree += int((plan_o == plan_g).all())
+        G.assert_close(out.cpu().numpy()[0], O_o, f"out step {s}")
+        G.assert_close(out_lse.cpu().numpy()[0], l_o, f"lse step {s}")
+    print(f"oracle's own plan equal to the GPU's on {agree} of {S - S // every} non-anchor steps")
+
+
+def test_anchor_every_step_is_all_fresh():
+    w = configs.TINY
+    Q, K, V = G.upload(w)
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    ep = dt.ErrorPlanner(pa, w.band_k, w.budget, 1)
+    o1 = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        ep.step(Q, K, V, o1)
+    ref = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    o2 = torch.empty_like(o1)
+    ref.step(Q, K, V, o2, anchor=True)
+    torch.cuda.synchronize()
+    assert (pa.plan.cpu().numpy() == PLAN_FRESH).all()
+    assert torch.equal(o1, o2)
