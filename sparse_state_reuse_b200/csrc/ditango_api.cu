@@ -174,14 +174,15 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 4-D map over a bf16 [B, H, N, d] tensor (d contiguous), box 64 x 128 rows,
-// 128-byte swizzle; columns past d and rows past N read as zero.
-bool make_qkv_map(CUtensorMap *m, const void *base, const DevGeom &g, const int64_t s[3]) {
+// 4-D map over a bf16 [B, H, N, d] tensor (d contiguous), box 64 columns x
+// box_rows rows, 128-byte swizzle; columns past d and rows past N read as zero.
+bool make_qkv_map(CUtensorMap *m, const void *base, const DevGeom &g, const int64_t s[3],
+                  unsigned box_rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[4] = {(cuuint64_t)g.d, (cuuint64_t)g.N, (cuuint64_t)g.H, (cuuint64_t)g.B};
   cuuint64_t strides[3] = {(cuuint64_t)(s[2] * 2), (cuuint64_t)(s[1] * 2), (cuuint64_t)(s[0] * 2)};
-  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t box[4] = {64, box_rows, 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -329,8 +330,9 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q, co
   if (!(scale >= 0.f) || !std::isfinite(scale)) return DITANGO_ERR_INVALID;
   if (scale == 0.f) scale = 1.f / std::sqrt((float)dg.d);
   CUtensorMap tq, tk, tv;
-  if (!make_qkv_map(&tq, Q, dg, qs) || !make_qkv_map(&tk, K, dg, ks) ||
-      !make_qkv_map(&tv, V, dg, vs))
+  // Q in 128-row tiles, K and V in 128-key tiles (the kernel's BM and BN)
+  if (!make_qkv_map(&tq, Q, dg, qs, 128) || !make_qkv_map(&tk, K, dg, ks, 128) ||
+      !make_qkv_map(&tv, V, dg, vs, 128))
     return DITANGO_ERR_CUDA;
   return cuda_status(launch_attn_partial(dg, tq, tk, tv, fresh_list, counts, scale, out_O, out_lse,
                                          out_by_slot ? 1 : 0, state_bf16 ? 1 : 0, out_valid,
