@@ -29,6 +29,10 @@
 // P V and next Q K^T.  One thread owns one query row, so row max and row sum
 // need no cross-thread reduction.  O is rescaled only when a row's running
 // maximum grows by more than 2^8 (exact: O and l share the stale maximum).
+#include <mutex>
+#include <set>
+#include <utility>
+
 #include "common.cuh"
 
 namespace ditango {
@@ -753,6 +757,28 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
 }  // namespace attn
 
+// Once per device and kernel: check the register count the setmaxnreg split
+// was written for, and opt in to the shared memory the kernel uses.  Done at
+// the first launch only, so that later launches (and CUDA graph captures)
+// make no attribute calls.
+static cudaError_t prepare_attn_kernel(const void *kfn, int smem) {
+  static std::mutex mu;
+  static std::set<std::pair<int, const void *>> ready;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ready.count({dev, kfn})) return cudaSuccess;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kfn);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != attn::kLaunchRegs) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  ready.insert({dev, kfn});
+  return cudaSuccess;
+}
+
 // Host launcher (called from the C ABI after validation).
 cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const CUtensorMap &tk,
                                 const CUtensorMap &tv, const int *fresh_list, const int *counts,
@@ -784,12 +810,7 @@ cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const C
                                          : attn::attn_partial_kernel<DD, true, false>)           \
                           : (g.multi_run ? attn::attn_partial_kernel<DD, false, true>            \
                                          : attn::attn_partial_kernel<DD, false, false>);         \
-    cudaFuncAttributes fa;                                                                       \
-    e = cudaFuncGetAttributes(&fa, kfn);                                                         \
-    if (e != cudaSuccess) return e;                                                              \
-    if (fa.numRegs != attn::kLaunchRegs) return cudaErrorInvalidConfiguration;                   \
-    e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,                   \
-                             attn::Cfg<DD>::SMEM);                                               \
+    e = prepare_attn_kernel(reinterpret_cast<const void *>(kfn), attn::Cfg<DD>::SMEM);          \
     if (e != cudaSuccess) return e;                                                              \
     kfn<<<grid, attn::kThreads, attn::Cfg<DD>::SMEM, stream>>>(tq, tk, tv, p);                    \
     return cudaGetLastError();                                                                   \

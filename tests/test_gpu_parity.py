@@ -232,3 +232,45 @@ def test_strided_qkv_inputs():
     pa.step(Qs, Ks, Vs, o2, anchor=True)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2)
+
+
+def test_step_captured_in_a_cuda_graph_replays_bit_identically():
+    """Every call is asynchronous, allocates nothing and never syncs the host,
+    so a whole step (plan -> partial -> merge) can be captured in a CUDA graph
+    and replayed; replays equal eager steps bit for bit."""
+    w = configs.TINY
+    Q, K, V = G.upload(w)
+    Kp, Vp = G.upload_prev(w)
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    build_cache(pa, Q, Kp, Vp)
+    cache0 = (pa.state_O.clone(), pa.state_lse.clone(), pa.valid.clone())
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    out_lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
+    pa.step(Q, K, V, out, out_lse, band_k=w.band_k, budget=w.budget)      # eager reference
+    torch.cuda.synchronize()
+    ref_out, ref_lse, ref_plan = out.clone(), out_lse.clone(), pa.plan.clone()
+
+    def restore():
+        pa.state_O.copy_(cache0[0]); pa.state_lse.copy_(cache0[1]); pa.valid.copy_(cache0[2])
+
+    restore()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):                  # warm-up on a side stream, as capture requires
+        pa.step(Q, K, V, out, out_lse, band_k=w.band_k, budget=w.budget)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    restore()
+    out.zero_(); out_lse.zero_()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        pa.step(Q, K, V, out, out_lse, band_k=w.band_k, budget=w.budget)
+    for _ in range(3):
+        restore()
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert pa.status.item() == 0
+        assert torch.equal(pa.plan, ref_plan)
+        assert torch.equal(out, ref_out) and torch.equal(out_lse, ref_lse)
