@@ -534,7 +534,8 @@ def blas_threads():
 
 
 def run_reference(args, w):
-    per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    # a bounded sample per step: the whole run stays within a few minutes
+    per_step = max(0.2, min(10.0, 150.0 / max(1, args.steps + args.warmup), args.cpu_baseline_seconds))
     for _ in range(args.warmup):
         oracle_sample(w, 7, 128, per_step / 4)
     tot_f, tot_s, desc = 0.0, 0.0, ""

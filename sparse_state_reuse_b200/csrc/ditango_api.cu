@@ -1,6 +1,7 @@
 // Host side of the C ABI declared in include/ditango.h: argument checks,
 // the kernels' geometry, TMA tensor maps and launches.  No device memory is
 // allocated here.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -42,7 +43,8 @@ using namespace ditango;
 
 namespace {
 
-long long g_wait_limit_ns = 1000000000LL;
+// Process-wide limit of every device wait; set from any host thread.
+std::atomic<long long> g_wait_limit_ns{1000000000LL};
 
 // Build the kernels' geometry; returns DITANGO_OK or the reason it cannot.
 ditango_status make_geom(const ditango_geom *in, DevGeom *out) {
@@ -336,7 +338,7 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q, co
     return DITANGO_ERR_CUDA;
   return cuda_status(launch_attn_partial(dg, tq, tk, tv, fresh_list, counts, scale, out_O, out_lse,
                                          out_by_slot ? 1 : 0, state_bf16 ? 1 : 0, out_valid,
-                                         drift_rows, dev_status, g_wait_limit_ns,
+                                         drift_rows, dev_status, g_wait_limit_ns.load(),
                                          num_sms_current(), static_cast<cudaStream_t>(stream)));
 }
 
@@ -425,7 +427,7 @@ ditango_status ditango_cache_compose(const ditango_geom *fine, const ditango_geo
                                           static_cast<cudaStream_t>(stream)));
 }
 
-void ditango_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns = ns > 0 ? ns : 1; }
+void ditango_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns.store(ns > 0 ? ns : 1); }
 
 ditango_status ditango_selftest_bounded_wait(int64_t limit_ns, int32_t *dev_status,
                                              ditango_stream stream) {
