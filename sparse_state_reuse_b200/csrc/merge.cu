@@ -24,6 +24,7 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowsPerBlock = 128;
 constexpr int kBatch = 4;    // O vectors per row in flight per lane
+constexpr int kSmallStates = 8;  // rows of at most this many states: per-lane weights
 
 struct Src {
   const char *O;     // [Lmax][d] block of this (index, b*h): float32, or bf16 (SB)
@@ -134,7 +135,12 @@ __device__ __forceinline__ void lse_weights(float l0, float l1, float &w0, float
   L = dead ? -INFINITY : Ms + logf(S);
 }
 
-template <int D, bool SB>
+// MS > 0: every row has at most MS states (frame-tile rows hold 2 to 4).
+// Then each lane loads all of a row's lse (one broadcast load each) and
+// computes the row's weights itself: no shuffles, and the weights overwrite
+// the loaded lse in place.  MS = 0: any number of states (up to 64), weights
+// by warp reductions over one state per lane.
+template <int D, bool SB, int MS>
 __global__ void __launch_bounds__(kThreads, SB ? 3 : 4)
 merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__restrict__ part_O,
              const float *__restrict__ part_lse, char *cache_O, float *cache_lse,
@@ -211,6 +217,85 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
   // keep the same bytes in flight); every load of a row -- its states' lse
   // and the first kBatch O vectors -- is issued before any of it is used.
   constexpr int R = SB ? 4 : 2;
+  if constexpr (MS > 0) {
+    constexpr int RS = 2;   // rows per warp iteration (the weights live in registers)
+    const bool act = lane < G4;
+    for (int r = r0 + RS * warp; r < rend; r += RS * kWarps) {
+      constexpr int R = RS;
+      float wt[R][MS];   // the states' lse, then their weights
+#pragma unroll
+      for (int q = 0; q < R; ++q)
+#pragma unroll
+        for (int a = 0; a < MS; ++a)
+          wt[q][a] = (a < nact && (r + q) < rend) ? __ldg(src[a].lse + r + q) : -INFINITY;
+      typename Raw4<SB>::T v[R][kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+        for (int q = 0; q < R; ++q) {
+          v[q][u] = zero_raw4<SB>();
+          if (act && u < nact && (r + q) < rend)
+            v[q][u] = load_raw4<SB>(src[u].O + (size_t)(r + q) * ROWB + lane * 4 * ES);
+        }
+      float L[R];
+#pragma unroll
+      for (int q = 0; q < R; ++q) {
+        // write back the lse of fresh states (lane a for state a)
+#pragma unroll
+        for (int a = 0; a < MS; ++a)
+          if (lane == a && a < nact && (r + q) < rend && src[a].wblse) src[a].wblse[r + q] = wt[q][a];
+        float M = wt[q][0];
+#pragma unroll
+        for (int a = 1; a < MS; ++a) M = fmaxf(M, wt[q][a]);
+        const bool dead = !(M > -INFINITY);
+        const float Ms = dead ? 0.f : M;
+        float S = 0.f;
+#pragma unroll
+        for (int a = 0; a < MS; ++a) {
+          wt[q][a] = expf(wt[q][a] - Ms);   // exp(-inf) = 0 for absent states
+          S += wt[q][a];
+        }
+        const float invS = dead ? 0.f : 1.f / S;
+#pragma unroll
+        for (int a = 0; a < MS; ++a) wt[q][a] *= invS;
+        L[q] = dead ? -INFINITY : Ms + logf(S);
+      }
+      float4 acc[R];
+#pragma unroll
+      for (int q = 0; q < R; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int a0 = 0; a0 < MS; a0 += kBatch) {
+        if (a0 >= nact) break;
+        if (a0 > 0) {
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+            for (int q = 0; q < R; ++q)
+              if (act && a0 + u < nact && (r + q) < rend)
+                v[q][u] = load_raw4<SB>(src[a0 + u].O + (size_t)(r + q) * ROWB + lane * 4 * ES);
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int a = a0 + u;
+          if (a >= nact) break;
+#pragma unroll
+          for (int q = 0; q < R; ++q) {
+            fma4(acc[q], wt[q][a], widen4<SB>(v[q][u]));
+            if (act && src[a].wbO && (r + q) < rend)
+              store_raw4<SB>(src[a].wbO + (size_t)(r + q) * ROWB + lane * 4 * ES, v[q][u]);
+          }
+        }
+      }
+      const int n = g.part_off[i] + r;
+      const size_t obase = (size_t)b * osb + (size_t)h * osh + lane * 4;
+#pragma unroll
+      for (int q = 0; q < R; ++q) {
+        if ((r + q) >= rend) continue;
+        if (act) store_out(out, out_is_fp32, obase + (size_t)(n + q) * osn, acc[q]);
+        if (out_lse && lane == 0) out_lse[((size_t)b * g.H + h) * g.N + n + q] = L[q];
+      }
+    }
+  } else {
   for (int r = r0 + R * warp; r < rend; r += R * kWarps) {
     float l0[R], l1[R];
 #pragma unroll
@@ -273,6 +358,7 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
       if (act) store_out(out, out_is_fp32, obase + (size_t)(n + q) * osn, acc[q]);
       if (out_lse && lane == 0) out_lse[((size_t)b * g.H + h) * g.N + n + q] = L[q];
     }
+  }
   }
 }
 
@@ -426,22 +512,39 @@ cudaError_t launch_merge(const DevGeom &g, const signed char *plan, const void *
                          long long osb, long long osh, long long osn, float *out_lse,
                          cudaStream_t stream) {
   dim3 grid((g.Lmax + merge::kRowsPerBlock - 1) / merge::kRowsPerBlock, g.P, g.BH);
+  int most = 0;   // most active units of any row: the states a row can merge
+  for (int i = 0; i < g.P; ++i) {
+    const int c = __builtin_popcountll(g.row_mask[i]);
+    most = c > most ? c : most;
+  }
+  const int ms = most <= 4 ? 4 : (most <= merge::kSmallStates ? merge::kSmallStates : 0);
   switch (g.d) {
+#define DITANGO_MERGE_MS(DD, SB, MS)                                                             \
+  merge::merge_kernel<DD, SB, MS><<<grid, merge::kThreads, 0, stream>>>(                         \
+      g, plan, static_cast<const char *>(part_O), part_lse, static_cast<char *>(cache_O),       \
+      cache_lse, cache_valid, writeback, out, out_is_fp32, osb, osh, osn, out_lse);
+#define DITANGO_MERGE_SB(DD, SB)                                                                 \
+  if (ms == 4) {                                                                                 \
+    DITANGO_MERGE_MS(DD, SB, 4)                                                                  \
+  } else if (ms == merge::kSmallStates) {                                                        \
+    DITANGO_MERGE_MS(DD, SB, merge::kSmallStates)                                                \
+  } else {                                                                                       \
+    DITANGO_MERGE_MS(DD, SB, 0)                                                                  \
+  }
 #define DITANGO_MERGE(DD)                                                                        \
   case DD:                                                                                       \
-    if (state_bf16)                                                                              \
-      merge::merge_kernel<DD, true><<<grid, merge::kThreads, 0, stream>>>(                       \
-          g, plan, static_cast<const char *>(part_O), part_lse, static_cast<char *>(cache_O),   \
-          cache_lse, cache_valid, writeback, out, out_is_fp32, osb, osh, osn, out_lse);          \
-    else                                                                                         \
-      merge::merge_kernel<DD, false><<<grid, merge::kThreads, 0, stream>>>(                      \
-          g, plan, static_cast<const char *>(part_O), part_lse, static_cast<char *>(cache_O),   \
-          cache_lse, cache_valid, writeback, out, out_is_fp32, osb, osh, osn, out_lse);          \
+    if (state_bf16) {                                                                            \
+      DITANGO_MERGE_SB(DD, true)                                                                 \
+    } else {                                                                                     \
+      DITANGO_MERGE_SB(DD, false)                                                                \
+    }                                                                                            \
     return cudaGetLastError();
     DITANGO_MERGE(64)
     DITANGO_MERGE(96)
     DITANGO_MERGE(128)
 #undef DITANGO_MERGE
+#undef DITANGO_MERGE_SB
+#undef DITANGO_MERGE_MS
     default:
       return cudaErrorInvalidValue;
   }
