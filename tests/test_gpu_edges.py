@@ -1,0 +1,116 @@
+"""Edge cases of the CUDA path against the fp64 oracle: the maximum number of
+partitions (P = 64) with ragged lengths down to one token, a single
+partition (P = 1), one KV group spanning every partition under the
+frame-tile mask (a unit of several runs), and an attention call with no
+fresh unit (a no-op that leaves the cache alone)."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import sparse_state_reuse_b200 as dt
+from oracle import groups as OG
+from oracle import masks as OM
+from oracle import step as OS
+from workloads import configs
+
+import gpu_common as G
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+
+def case(N, d, seed):
+    return configs.scaled(configs.TINY, N=N, d=d, B=1, H=2, P=1, seed=seed, name=f"edge_{N}_{d}")
+
+
+def all_fresh_states(w, part_off, fo=None, fm=None, go=None):
+    geom = dt.Geometry(w.B, w.H, w.N, w.d, part_off, fo, fm, group_off=go)
+    A = OM.pair_mask(part_off, fo, fm)
+    Au = OG.unit_mask(A, go) if go is not None else A
+    n, Lmax = int(Au.sum()), int(max(np.diff(part_off)))
+    Q, K, V = G.upload(w)
+    Gc = Au.shape[1]
+    plan = torch.zeros((len(part_off) - 1) * Gc, dtype=torch.int8, device="cuda")
+    fresh = torch.zeros(n, dtype=torch.int32, device="cuda")
+    counts = torch.zeros(2, dtype=torch.int32, device="cuda")
+    dt.ditango_plan(geom, None, None, 0, 1.0, True, plan, fresh, counts)
+    O = torch.full((n, w.BH, Lmax, w.d), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.full((n, w.BH, Lmax), float("nan"), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dt.ditango_attn_partial(geom, Q, K, V, fresh, counts, 0.0, O, lse, 0, None, st)
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    out_lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
+    dt.ditango_merge(geom, plan, O, lse, None, None, None, 0, out, 1, out_lse=out_lse)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    return Au, fresh.cpu().numpy()[:n], O.cpu().numpy(), lse.cpu().numpy(), out.cpu().numpy(), out_lse.cpu().numpy()
+
+
+def test_sixty_four_ragged_partitions_down_to_one_token():
+    rng = np.random.default_rng(9)
+    lens = rng.integers(1, 40, size=64)
+    lens[[0, 17, 63]] = 1
+    part_off = [0] + np.cumsum(lens).tolist()
+    w = case(part_off[-1], 64, 901)
+    Au, fresh, O, lse, out, out_lse = all_fresh_states(w, part_off)
+    assert len(fresh) == 64 * 64
+    for bh in range(w.BH):
+        q, k, v, _, _ = G.slabs(w, 0, bh, with_prev=False)
+        for f in (0, 1, 63, 64 * 17 + 5, 64 * 63, 64 * 64 - 1):
+            i, j = divmod(int(fresh[f]), 64)
+            rows = np.arange(part_off[i], part_off[i + 1])
+            Oo, lo = OS.pair_state(q[rows], rows, k, v, part_off, j)
+            G.assert_close(O[f, bh, :rows.size], Oo, f"O pair {(i, j)}")
+            G.assert_close(lse[f, bh, :rows.size], lo, f"lse pair {(i, j)}")
+        from oracle.attention import dense_attention
+        Od, ld = dense_attention(q, k, v)
+        G.assert_close(out[0, bh], Od, "64-way merge = dense")
+        G.assert_close(out_lse[0, bh], ld, "64-way merge lse")
+
+
+def test_single_partition_is_dense_attention():
+    w = case(1000, 128, 902)
+    Au, fresh, O, lse, out, out_lse = all_fresh_states(w, [0, 1000])
+    from oracle.attention import dense_attention
+    for bh in range(w.BH):
+        q, k, v, _, _ = G.slabs(w, 0, bh, with_prev=False)
+        Od, ld = dense_attention(q, k, v)
+        G.assert_close(out[0, bh], Od, "P = 1")
+        G.assert_close(out_lse[0, bh], ld, "P = 1 lse")
+
+
+def test_one_group_over_every_partition_with_the_frame_mask():
+    """Every row's unit holds frame 0 and its neighbours: up to two runs of
+    partitions with a gap between them."""
+    fo = [0, 70, 200, 260, 400, 530, 600, 700]
+    F = len(fo) - 1
+    fm = [[1 if (abs(f - g) <= 1 or g == 0) else 0 for g in range(F)] for f in range(F)]
+    w = case(fo[-1], 96, 903)
+    Au, fresh, O, lse, out, out_lse = all_fresh_states(w, fo, fo, fm, go=[0, F])
+    assert Au.shape == (F, 1) and len(fresh) == F
+    for bh in range(w.BH):
+        q, k, v, _, _ = G.slabs(w, 0, bh, with_prev=False)
+        for f, u in enumerate(fresh):
+            i = int(u)
+            rows = np.arange(fo[i], fo[i + 1])
+            Oo, lo = OG.unit_state(q[rows], rows, k, v, fo, [0, F], 0, fo, fm)
+            G.assert_close(O[f, bh, :rows.size], Oo, f"unit row {i}")
+            G.assert_close(out[0, bh, rows], Oo, f"merged row {i}")
+
+
+def test_attention_with_no_fresh_unit_is_a_no_op():
+    w = configs.TINY
+    Q, K, V = G.upload(w)
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    pa.plan_step(anchor=True)
+    pa.partial(Q, K, V)
+    torch.cuda.synchronize()
+    before = (pa.state_O.clone(), pa.state_lse.clone())
+    pa.counts.zero_()
+    pa.partial(Q, K, V)
+    torch.cuda.synchronize()
+    assert pa.status.item() == 0
+    assert torch.equal(pa.state_O, before[0]) and torch.equal(pa.state_lse, before[1])
