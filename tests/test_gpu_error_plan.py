@@ -33,8 +33,10 @@ def to_dev(bits):
     return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
 
 
-@pytest.mark.parametrize("gs,frames", [(0, False), (2, False), (0, True)], ids=["pairs", "groups2", "frame_tile"])
-def test_schedule_matches_oracle(gs, frames):
+@pytest.mark.parametrize("gs,frames,sb", [(0, False, False), (2, False, False), (0, True, False),
+                                           (3, True, False), (0, False, True)],
+                         ids=["pairs", "groups2", "frame_tile", "groups3_frame_tile", "pairs_bf16_cache"])
+def test_schedule_matches_oracle(gs, frames, sb):
     F = 6 if frames else 0
     w = configs.scaled(configs.TINY, N=1536, P=6, d=64, H=2, drift_sigma=0.05, budget=0.5 if not frames else 0.7,
                        band_k=0, group_size=gs, F=F, frame_component=0.5 if frames else 0.0,
@@ -50,7 +52,8 @@ def test_schedule_matches_oracle(gs, frames):
     sch = E.Schedule([f64(x) for x in q_bits], po, go, A, w.band_k, w.budget, every, fo, fm)
     Au, band = sch.Au, sch.band
 
-    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, po, fo, fm, group_off=go if gs else None)
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, po, fo, fm, group_off=go if gs else None,
+                                 state_bf16=sb)
     ep = dt.ErrorPlanner(pa, w.band_k, w.budget, every)
     Q = to_dev(np.stack(q_bits)[None])
     out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")

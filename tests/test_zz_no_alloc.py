@@ -16,6 +16,7 @@ import pytest
 torch = pytest.importorskip("torch")
 
 import sparse_state_reuse_b200 as dt
+from oracle import groups as OG
 from oracle import masks as OM
 from workloads import configs, inputs
 
@@ -25,20 +26,25 @@ if not torch.cuda.is_available():
     pytest.skip("no CUDA device", allow_module_level=True)
 
 
-def _buffers(P, n):
+def _buffers(P, n, G=None):
     dev = "cuda"
-    return (torch.full((P * P,), -7, dtype=torch.int8, device=dev),
+    G = P if G is None else G
+    return (torch.full((P * G,), -7, dtype=torch.int8, device=dev),
             torch.full((n,), -7, dtype=torch.int32, device=dev),
             torch.full((2,), -7, dtype=torch.int32, device=dev),
-            torch.full((P * P,), -7.0, dtype=torch.float32, device=dev))
+            torch.full((P * G,), -7.0, dtype=torch.float32, device=dev))
 
 
-@pytest.mark.parametrize("w", [configs.DITANGO_REUSE, configs.LONG_VIDEO], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [configs.DITANGO_REUSE, configs.LONG_VIDEO, configs.DITANGO_GROUPS],
+                         ids=lambda w: w.name)
 def test_noalloc_plan_equals_plan_on_two_calls(w):
     lib = ctypes.CDLL(dt.LIB_PATH)
     assert hasattr(lib, "ditango_plan_noalloc")
-    g = dt.Geometry(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask())
+    go = w.group_off() if w.grouped else None
+    g = dt.Geometry(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask(), group_off=go)
     A = OM.pair_mask(w.part_off(), w.frame_off(), w.frame_mask())
+    if go is not None:
+        A = OG.unit_mask(A, go)
     pairs = OM.slot_pairs(A)
     n = len(pairs)
     nws = dt.ditango_plan_workspace_size(g)
@@ -48,9 +54,9 @@ def test_noalloc_plan_equals_plan_on_two_calls(w):
         lse = torch.from_numpy(inputs.synthetic_cache_lse(w, n, pairs, seed=seed + w.seed)).cuda()
         if call == 1:
             valid[3] = 0                      # a different cache state on the second call
-        ref = _buffers(w.P, n)
+        ref = _buffers(w.P, n, g.G)
         dt.ditango_plan(g, lse, valid, w.band_k, w.budget, 0, *ref, ws, nws)
-        got = _buffers(w.P, n)
+        got = _buffers(w.P, n, g.G)
         dt.ditango_plan_noalloc(g, lse, valid, w.band_k, w.budget, 0, *got)
         torch.cuda.synchronize()
         assert torch.equal(ref[0], got[0]), f"plan differs on call {call}"
