@@ -212,10 +212,13 @@ def run_ours(args, w, rank, world, local_rank):
     n_ev = args.steps
     e_part0, e_part1 = [ev() for _ in range(n_ev)], [ev() for _ in range(n_ev)]
     e_merge1 = [ev() for _ in range(n_ev)]
+    e_plan0 = [ev() for _ in range(n_ev)]
     e_start, e_end = ev(), ev()
 
     def one_step(t=None):
         with torch.cuda.stream(stream):
+            if t is not None:
+                e_plan0[t].record(stream)
             pa.plan_step(w.band_k, w.budget, w.anchor, stream=stream)
             if t is not None:
                 e_part0[t].record(stream)
@@ -247,6 +250,7 @@ def run_ours(args, w, rank, world, local_rank):
     ms = e_start.elapsed_time(e_end)
     part_ms = float(np.mean([e_part0[t].elapsed_time(e_part1[t]) for t in range(n_ev)]))
     merge_ms = float(np.mean([e_part1[t].elapsed_time(e_merge1[t]) for t in range(n_ev)]))
+    plan_us = 1e3 * float(np.mean([e_plan0[t].elapsed_time(e_part0[t]) for t in range(n_ev)]))
     ms = max_over_ranks(ms, dev, dist)
     if world > 1:
         dist.barrier()
@@ -351,6 +355,9 @@ def run_ours(args, w, rank, world, local_rank):
                            "kernel_ms": round(merge_ms, 4),
                            "algorithmic_bytes_per_launch": mbytes,
                            "traffic": recorded_traffic("merge.cu", w.name)},
+        "plan": {"us": round(plan_us, 2), "launches": 1 if w.anchor else 2,
+                 "note": "selection alone on anchor steps; mass score over the cached lse + "
+                         "selection otherwise"},
         "e2e": {"value": round(aggregate_tflops(world, flops, e2e_ms), 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
