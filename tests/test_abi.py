@@ -149,3 +149,25 @@ def test_size_one_dimensions_may_have_any_stride():
     with pytest.raises(dt.DitangoError) as e:
         dt.ditango_attn_partial(g2, 4096, 4096, 4096, 4096, 4096, 0.0, 4096, 4096, 1, stream=0)
     assert e.value.status == 1
+
+
+def test_plain_c_program_uses_the_abi(tmp_path):
+    """The boundary is a C ABI: a C program built with gcc against
+    include/ditango.h and linked to libditango.so runs its host-side calls."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc") or shutil.which("cc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(__file__))
+    exe = str(tmp_path / "abi_host")
+    libdir = os.path.dirname(dt.LIB_PATH)
+    r = subprocess.run([gcc, "-std=c99", "-O1", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
+                        os.path.join(root, "tests", "c", "abi_host.c"), "-L", libdir, "-lditango",
+                        "-Wl,-rpath," + libdir, "-o", exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stdout + run.stderr
+    out = dict(line.split() for line in run.stdout.splitlines())
+    assert out["fails"] == "0" and out["active_pairs"] == "28"
+    assert int(out["version"]) == dt.ditango_version()
