@@ -1,0 +1,384 @@
+"""CPU model of the synchronisation inside the persistent attention kernel
+(sparse_state_reuse_b200/csrc/attn_partial.cu), checked on random
+interleavings.
+
+The kernel's roles talk only through mbarriers in shared memory:
+  * the producer warp arms a full barrier (arrive + expect_tx) and issues TMA
+    loads of the Q tiles and of the two K and V stages;
+  * the MMA warp issues tcgen05.mma (S = Q K^T into TMEM, O += P V with P
+    read from the S columns) and tcgen05.commit arrivals;
+  * eight softmax warps, four per 128-row Q tile, each own 32 TMEM lanes:
+    they read S, write P in place, sometimes rescale O, and read O in the
+    epilogue.
+Each role below yields the same waits, arrivals and asynchronous operations
+as the kernel, in the kernel's program order, with the kernel's own parity
+expressions.  A scheduler interleaves them at random: a TMA load lands at
+any later moment; MMAs complete in issue order at any later moment; a
+commit arrives once every MMA issued before it has completed.
+
+Checked on every interleaving:
+  * progress: every wait ends (no interleaving stalls every role);
+  * no phase aliasing: a parity wait can tell phase n from phase n + 1 only,
+    so while a role waits for phase n its barrier never completes phase
+    n + 1; and each parity the kernel computes is that of the phase it means;
+  * no arrival beyond a barrier's count within one phase;
+  * no data race on TMEM (S/P and O of each Q tile) or on the shared-memory
+    tiles (Q0, Q1, K and V stages): a softmax access never overlaps an
+    asynchronous operation in flight that writes the region (or reads it,
+    when the access writes), and a load never overlaps an MMA that reads its
+    region.  MMA after MMA is ordered by the tensor pipe and not checked;
+  * at the end no operation is in flight and no barrier holds a half
+    complete phase.
+Planted mistakes (a dropped wait, an early release) must be caught, so that
+a checker that passes everything would fail here.
+"""
+import random
+
+import pytest
+
+STAGES = 2
+WARPS_PER_TILE = 4
+
+
+class Violation(AssertionError):
+    pass
+
+
+class Bar:
+    def __init__(self, name, count):
+        self.name = name
+        self.count = count
+        self.pending = count
+        self.tx = 0                    # loads armed but not landed
+        self.phase = 0                 # phases completed
+
+    def arrive(self):
+        if self.pending == 0:
+            raise Violation(f"arrival beyond the count of {self.name}")
+        self.pending -= 1
+        self._complete()
+
+    def arm(self, loads):
+        self.tx += loads
+        self.arrive()
+
+    def land(self):
+        self.tx -= 1
+        self._complete()
+
+    def _complete(self):
+        if self.pending == 0 and self.tx == 0:
+            self.phase += 1
+            self.pending = self.count
+
+
+def barriers():
+    b = {"q_full": 1, "q_empty": 1, "drain": 1}
+    for s in range(STAGES):
+        for n in ("k_full", "k_empty", "v_full", "v_empty"):
+            b[f"{n}{s}"] = 1
+    for k in range(2):
+        b[f"s_full{k}"] = 1
+        b[f"p_full{k}"] = WARPS_PER_TILE      # one arrival per softmax warp
+        b[f"o_full{k}"] = 1
+        b[f"o_empty{k}"] = WARPS_PER_TILE
+    return {n: Bar(n, c) for n, c in b.items()}
+
+
+# ---------------------------------------------------------------- the roles
+# An item is one (query partition, batch-head, pair of Q tiles) of a CTA:
+# (has1, [key tiles of each fresh unit of the partition]).
+
+def producer(items, mut):
+    kc = vc = uc = 0
+    for has1, Ts in items:
+        yield ("wait", "q_empty", (uc & 1) ^ 1, uc - 1)
+        yield ("arm", "q_full", 2 if has1 else 1)
+        yield ("load", "Q0", "q_full")
+        if has1:
+            yield ("load", "Q1", "q_full")
+        for T in Ts:
+            for _ in range(T):
+                s = kc % STAGES
+                if mut != "producer_skips_k_empty":
+                    yield ("wait", f"k_empty{s}", ((kc // STAGES) & 1) ^ 1, kc // STAGES - 1)
+                yield ("arm", f"k_full{s}", 1)
+                yield ("load", f"K{s}", f"k_full{s}")
+                kc += 1
+                s = vc % STAGES
+                yield ("wait", f"v_empty{s}", ((vc // STAGES) & 1) ^ 1, vc // STAGES - 1)
+                yield ("arm", f"v_full{s}", 1)
+                yield ("load", f"V{s}", f"v_full{s}")
+                vc += 1
+        uc += 1
+
+
+def mma(items, mut):
+    kc = vc = uc = 0
+    pc = [0, 0]
+    oc = [0, 0]
+
+    def qk(k, ks):
+        return ("mma", {f"Q{k}", f"K{ks}"}, {f"S{k}"})
+
+    def pv(k, vs, acc):
+        return ("mma", {f"S{k}", f"V{vs}"} | ({f"O{k}"} if acc else set()), {f"O{k}"})
+
+    for has1, Ts in items:
+        yield ("wait", "q_full", uc & 1, uc)
+        for fi, T in enumerate(Ts):
+            last_pair = fi + 1 == len(Ts)
+            ks = kc % STAGES
+            yield ("wait", f"k_full{ks}", (kc // STAGES) & 1, kc // STAGES)
+            if mut == "k_released_before_qk":
+                yield ("commit", f"k_empty{ks}")
+            yield qk(0, ks)
+            yield ("commit", "s_full0")
+            if has1:
+                yield qk(1, ks)
+                yield ("commit", "s_full1")
+            if mut != "k_released_before_qk":
+                yield ("commit", f"k_empty{ks}")
+            kc += 1
+            if T == 1 and last_pair:
+                yield ("commit", "q_empty")
+            for t in range(T):
+                vs = vc % STAGES
+                yield ("wait", f"v_full{vs}", (vc // STAGES) & 1, vc // STAGES)
+                more = t + 1 < T
+                for k in range(2):
+                    if k == 1 and not has1:
+                        break
+                    if not (mut == "mma_skips_p_full" and k == 0):
+                        yield ("wait", f"p_full{k}", pc[k] & 1, pc[k])
+                    pc[k] += 1
+                    if t == 0:
+                        if mut != "mma_skips_o_empty":
+                            yield ("wait", f"o_empty{k}", (oc[k] & 1) ^ 1, oc[k] - 1)
+                        oc[k] += 1
+                    yield pv(k, vs, t > 0)
+                    if not more:
+                        yield ("commit", f"o_full{k}")
+                    if more:
+                        ks2 = kc % STAGES
+                        if k == 0:
+                            yield ("wait", f"k_full{ks2}", (kc // STAGES) & 1, kc // STAGES)
+                        yield qk(k, ks2)
+                        yield ("commit", f"s_full{k}")
+                yield ("commit", f"v_empty{vs}")
+                vc += 1
+                if more:
+                    yield ("commit", f"k_empty{kc % STAGES}")
+                    kc += 1
+                    if t + 2 == T and last_pair:
+                        yield ("commit", "q_empty")
+        uc += 1
+    # drain: every MMA issued must finish before TMEM is released
+    yield ("commit", "drain")
+    yield ("wait", "drain", 0, 0)
+
+
+def softmax_warp(k, items, rng, rescale_p, mut):
+    sc = ofc = 0
+    S, O = f"S{k}", f"O{k}"
+    for has1, Ts in items:
+        if k == 1 and not has1:
+            continue
+        for T in Ts:
+            for t in range(T):
+                yield ("wait", f"s_full{k}", sc & 1, sc)
+                sc += 1
+                yield ("hold", S, "w")                 # read S, write P over it
+                if t > 0 and rng.random() < rescale_p:
+                    yield ("hold", O, "w")             # O *= alpha
+                    yield ("release", O)
+                if mut == "p_full_before_p_written":
+                    yield ("arrive", f"p_full{k}")
+                    yield ("release", S)
+                else:
+                    yield ("release", S)
+                    yield ("arrive", f"p_full{k}")
+            if mut != "softmax_skips_o_full":
+                yield ("wait", f"o_full{k}", ofc & 1, ofc)
+            ofc += 1
+            yield ("hold", O, "r")                     # O into registers
+            yield ("release", O)
+            yield ("arrive", f"o_empty{k}")
+
+
+# ---------------------------------------------------------------- scheduler
+
+def conflicts(reads_a, writes_a, reads_b, writes_b):
+    return bool(writes_a & (reads_b | writes_b)) or bool(reads_a & writes_b)
+
+
+def run(items, seed, rescale_p=0.5, mut=None, max_steps=2_000_000):
+    """Interleave the roles at random; raise Violation on any broken rule."""
+    rng = random.Random(seed)
+    B = barriers()
+    roles = {"producer": producer(items, mut), "mma": mma(items, mut)}
+    for k in range(2):
+        for w in range(WARPS_PER_TILE):
+            roles[f"softmax{k}.{w}"] = softmax_warp(k, items, random.Random(rng.random()),
+                                                    rescale_p, mut)
+    nxt = {r: next(g, None) for r, g in roles.items()}
+    loads = []                 # in flight: (region, barrier)
+    mma_q = []                 # in issue order: ("mma", reads, writes) | ("commit", barrier)
+    holds = {}                 # role -> {region: mode}
+
+    def check_wait(role, op):
+        _, name, parity, n = op
+        if parity != (n & 1):
+            raise Violation(f"{role}: parity {parity} for phase {n} of {name}")
+        if B[name].phase > n + 1:
+            raise Violation(f"{role}: {name} completed phase {n + 1} while it waits for phase {n}")
+
+    def mma_in_flight():
+        return [op for op in mma_q if op[0] == "mma"]
+
+    for _ in range(max_steps):
+        choices = []
+        for r, op in nxt.items():
+            if op is None:
+                continue
+            if op[0] == "wait":
+                check_wait(r, op)
+                if B[op[1]].phase >= op[3] + 1:
+                    choices.append(("role", r))
+            else:
+                choices.append(("role", r))
+        if mma_q:
+            choices.append(("mma", None))
+        choices.extend(("land", i) for i in range(len(loads)))
+        if not choices:
+            if all(op is None for op in nxt.values()):
+                break
+            blocked = {r: op for r, op in nxt.items() if op is not None}
+            raise Violation(f"no role can proceed: {blocked}")
+        kind, x = rng.choice(choices)
+        if kind == "mma":
+            op = mma_q.pop(0)
+            if op[0] == "commit":
+                B[op[1]].arrive()
+            continue
+        if kind == "land":
+            region, name = loads.pop(x)
+            B[name].land()
+            continue
+        role, op = x, nxt[x]
+        what = op[0]
+        if what == "arrive":
+            B[op[1]].arrive()
+        elif what == "arm":
+            B[op[1]].arm(op[2])
+        elif what == "load":
+            region = op[1]
+            for m in mma_in_flight():
+                if conflicts(set(), {region}, m[1], m[2]):
+                    raise Violation(f"load of {region} while an MMA on it is in flight")
+            if any(r == region for r, _ in loads):
+                raise Violation(f"two loads of {region} in flight")
+            for h in holds.values():
+                if region in h:
+                    raise Violation(f"load of {region} while a softmax warp holds it")
+            loads.append((region, op[2]))
+        elif what == "mma":
+            _, reads, writes = op
+            for region, _ in loads:
+                if region in reads | writes:
+                    raise Violation(f"MMA on {region} before its load landed")
+            for h in holds.values():
+                for region, mode in h.items():
+                    if conflicts(reads, writes, {region} if mode == "r" else set(),
+                                 {region} if mode == "w" else set()):
+                        raise Violation(f"MMA on {region} while a softmax warp holds it ({mode})")
+            mma_q.append(op)
+        elif what == "commit":
+            mma_q.append(op)
+        elif what == "hold":
+            region, mode = op[1], op[2]
+            r_set = {region}
+            w_set = {region} if mode == "w" else set()
+            for m in mma_in_flight():
+                if conflicts(r_set, w_set, m[1], m[2]):
+                    raise Violation(f"{role} touches {region} ({mode}) under an MMA in flight")
+            holds.setdefault(role, {})[region] = mode
+        elif what == "release":
+            del holds[role][op[1]]
+        elif what == "wait":
+            pass
+        nxt[role] = next(roles[role], None)
+    else:
+        raise Violation("step limit reached")
+    if mma_q or loads:
+        raise Violation("operations still in flight at the end")
+    for b in B.values():
+        if b.pending != b.count or b.tx != 0:
+            raise Violation(f"{b.name} ends inside a phase")
+    if any(holds.values()):
+        raise Violation("a region is still held at the end")
+    return B
+
+
+def random_items(rng):
+    items = []
+    for _ in range(rng.randint(1, 5)):
+        has1 = rng.random() < 0.7
+        items.append((has1, [rng.choice([1, 1, 2, 3, 5]) for _ in range(rng.randint(1, 4))]))
+    return items
+
+
+@pytest.mark.parametrize("seed", range(60))
+def test_protocol_on_random_items_and_interleavings(seed):
+    rng = random.Random(1000 + seed)
+    items = random_items(rng)
+    B = run(items, seed, rescale_p=rng.choice([0.0, 0.3, 1.0]))
+    # every barrier completed exactly the phases its traffic implies
+    n_units = sum(len(Ts) for _, Ts in items)
+    n_tiles = sum(sum(Ts) for _, Ts in items)
+    n_units1 = sum(len(Ts) for has1, Ts in items if has1)
+    n_tiles1 = sum(sum(Ts) for has1, Ts in items if has1)
+    assert B["q_full"].phase == B["q_empty"].phase == len(items)
+    assert sum(B[f"k_full{s}"].phase for s in range(STAGES)) == n_tiles
+    assert sum(B[f"v_empty{s}"].phase for s in range(STAGES)) == n_tiles
+    assert B["s_full0"].phase == B["p_full0"].phase == n_tiles
+    assert B["s_full1"].phase == B["p_full1"].phase == n_tiles1
+    assert B["o_full0"].phase == B["o_empty0"].phase == n_units
+    assert B["o_full1"].phase == B["o_empty1"].phase == n_units1
+    assert B["drain"].phase == 1
+
+
+@pytest.mark.parametrize("items", [
+    [(False, [1])],                       # one tile, one Q tile
+    [(True, [1])],
+    [(True, [1] * 7)],                    # many one-tile units: q_empty on the first QK
+    [(False, [2]), (True, [1]), (False, [3, 1])],
+    [(True, [9])],                        # a long unit: both stages cycle many times
+], ids=["T1_tile0", "T1_both", "units_of_one_tile", "mixed", "long_unit"])
+def test_protocol_edge_items(items):
+    for seed in range(20):
+        run(items, seed)
+
+
+@pytest.mark.parametrize("mut", ["mma_skips_p_full", "softmax_skips_o_full", "k_released_before_qk",
+                                 "p_full_before_p_written", "producer_skips_k_empty"])
+def test_planted_mistakes_are_caught(mut):
+    items = [(True, [3, 2]), (True, [1, 4]), (False, [2])]
+    caught = 0
+    for seed in range(40):
+        try:
+            run(items, seed, mut=mut)
+        except Violation:
+            caught += 1
+    assert caught > 0, mut
+
+
+def test_o_empty_wait_is_implied_by_p_full():
+    """The MMA warp's o_empty wait before the first P V of a unit never
+    blocks: each softmax warp arrives on o_empty before it reaches the next
+    unit's first tile, and that P V already waits for all four warps' p_full
+    arrivals.  The wait stays in the kernel as a guard; the model shows it is
+    not what orders the epilogue's O reads before the next unit's P V."""
+    items = [(True, [3, 2]), (True, [1, 4]), (False, [2])]
+    for seed in range(40):
+        run(items, seed, mut="mma_skips_o_empty")
