@@ -27,6 +27,26 @@ from ._abi import (  # noqa: F401
 )
 
 
+def check_tensor(t, name, shape, dtypes, contiguous=False):
+    """Raise unless t is a tensor of one of `dtypes` with this shape, on a
+    CUDA device, its last dimension contiguous (the whole tensor when
+    `contiguous`).  The kernels see raw addresses and strides only, so these
+    are checked here, before anything is launched."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: a torch.Tensor is required, got {type(t).__name__}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {' or '.join(str(d) for d in dtypes)}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.shape[-1] > 1 and t.stride(-1) != 1:
+        raise ValueError(f"{name}: the last dimension must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be on a CUDA device, is on {t.device}")
+
+
 class PartitionedAttention:
     """Device buffers for one geometry and the three-call step.
 
@@ -48,6 +68,8 @@ class PartitionedAttention:
         self.frame_mask = frame_mask
         self.group_off = None if group_off is None else list(group_off)
         self.device = torch.device(device)
+        if self.device.type != "cuda":
+            raise ValueError(f"the state cache lives on a CUDA device, not {self.device}")
         self.geom = self._geometry(strides)
         self.P = self.geom.P
         self.G = self.geom.G
@@ -75,6 +97,18 @@ class PartitionedAttention:
                         self.frame_mask, q_strides=s[0], k_strides=s[1], v_strides=s[2],
                         group_off=self.group_off)
 
+    def check_inputs(self, Q, K, V, out=None, out_lse=None):
+        """Shapes, dtypes and devices of a step's tensors (raises on a mismatch)."""
+        import torch
+        qkv = (self.B, self.H, self.N, self.d)
+        for name, t in (("Q", Q), ("K", K), ("V", V)):
+            check_tensor(t, name, qkv, (torch.bfloat16,))
+        if out is not None:
+            check_tensor(out, "out", qkv, (torch.float32, torch.bfloat16))
+        if out_lse is not None:
+            check_tensor(out_lse, "out_lse", (self.B, self.H, self.N), (torch.float32,),
+                         contiguous=True)
+
     def _bind(self, Q, K, V):
         want = tuple(tuple(t.stride()[:3]) for t in (Q, K, V))
         have = (tuple(self.geom.g.q_strides), tuple(self.geom.g.k_strides), tuple(self.geom.g.v_strides))
@@ -87,6 +121,11 @@ class PartitionedAttention:
                      self.ws_bytes, stream)
 
     def partial(self, Q, K, V, scale=0.0, stream=None, drift_rows=None):
+        import torch
+        self.check_inputs(Q, K, V)
+        if drift_rows is not None:
+            check_tensor(drift_rows, "drift_rows", (self.P, self.B * self.H, self.Lmax),
+                         (torch.float32,), contiguous=True)
         self._bind(Q, K, V)
         ditango_attn_partial(self.geom, Q, K, V, self.fresh_list, self.counts, scale,
                              self.state_O, self.state_lse, 1, self.valid, self.status, stream,
@@ -94,6 +133,11 @@ class PartitionedAttention:
 
     def merge(self, out, out_lse=None, stream=None):
         import torch
+        qkv = (self.B, self.H, self.N, self.d)
+        check_tensor(out, "out", qkv, (torch.float32, torch.bfloat16))
+        if out_lse is not None:
+            check_tensor(out_lse, "out_lse", (self.B, self.H, self.N), (torch.float32,),
+                         contiguous=True)
         ditango_merge(self.geom, self.plan, None, None, self.state_O, self.state_lse, self.valid, 0,
                       out, out.dtype == torch.float32, tuple(out.stride()[:3]), out_lse, stream,
                       state_bf16=self.state_bf16)
@@ -101,6 +145,7 @@ class PartitionedAttention:
     def step(self, Q, K, V, out, out_lse=None, band_k=0, budget=1.0, anchor=False, scale=0.0,
              stream=None):
         """plan -> partial attention of the fresh units -> merge, on one stream."""
+        self.check_inputs(Q, K, V, out, out_lse)
         self.plan_step(band_k, budget, anchor, stream)
         self.partial(Q, K, V, scale, stream)
         self.merge(out, out_lse, stream)
@@ -160,6 +205,7 @@ class ErrorPlanner:
     def step(self, Q, K, V, out, out_lse=None, scale=0.0, stream=None):
         """plan by predicted error -> attention of the fresh units (measuring the
         local drift) -> merge."""
+        self.pa.check_inputs(Q, K, V, out, out_lse)    # before the plan advances the ages
         self.plan(stream)
         self.pa.partial(Q, K, V, scale, stream, drift_rows=self.drift_rows)
         self.pa.merge(out, out_lse, stream)

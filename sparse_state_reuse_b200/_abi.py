@@ -94,10 +94,14 @@ def status_string(s: int) -> str:
 
 
 def _ptr(x):
+    """Device address of a tensor (or an address given as an int)."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
+    if getattr(x, "is_cuda", True) is False:
+        # a host tensor's address would be dereferenced by a kernel
+        raise ValueError(f"a CUDA tensor is required here, got one on {x.device}")
     return x.data_ptr()
 
 

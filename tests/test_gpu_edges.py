@@ -114,3 +114,20 @@ def test_attention_with_no_fresh_unit_is_a_no_op():
     torch.cuda.synchronize()
     assert pa.status.item() == 0
     assert torch.equal(pa.state_O, before[0]) and torch.equal(pa.state_lse, before[1])
+
+
+def test_mismatched_tensors_are_refused_before_any_launch():
+    w = configs.TINY
+    Q, K, V = G.upload(w)
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    with pytest.raises(ValueError, match="shape"):
+        pa.step(Q[:, :, : w.N // 2], K, V, out, anchor=True)
+    with pytest.raises(TypeError, match="dtype"):
+        pa.step(Q.float(), K, V, out, anchor=True)
+    with pytest.raises(ValueError, match="CUDA device"):
+        pa.step(Q, K.cpu(), V, out, anchor=True)
+    with pytest.raises(TypeError, match="dtype"):
+        pa.merge(out.half())
+    torch.cuda.synchronize()
+    assert pa.status.item() == 0
