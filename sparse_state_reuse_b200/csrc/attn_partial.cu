@@ -359,7 +359,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     {
       const bool leader = elect_one();
       uint32_t kc = 0, vc = 0, uc = 0;
-      // last armed phase per full barrier (for a clean stop on abort)
+      // last armed phase per full barrier (drained before the warp exits)
       // bit 2s: stage s armed at least once; bit 2s+1: parity of its last arming
       int q_armed = -1;
       uint32_t k_armed = 0, v_armed = 0;
@@ -407,8 +407,13 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         ++uc;
       }
-      if (!ok) {
-        // stop cleanly: let every load already issued land before exiting
+      // Every load issued lands before the warp exits, on both paths.  When
+      // another role gave up, this warp can still finish its loop with
+      // ok == true (each wait of its last tiles completed at once and never
+      // looked at the abort flag) while nothing consumes its last loads.  On
+      // the normal path these waits pass at once or as the loads land: only
+      // this warp arms the full barriers, so none runs past its last arming.
+      {
         WaitCtl drain_ctl{nullptr, nullptr, 100000000LL};
         volatile int never = 0;
         drain_ctl.abort_flag = &never;

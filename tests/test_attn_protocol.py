@@ -88,12 +88,28 @@ def barriers():
 # ---------------------------------------------------------------- the roles
 # An item is one (query partition, batch-head, pair of Q tiles) of a CTA:
 # (has1, [key tiles of each fresh unit of the partition]).
+#
+# A wait is ("wait", barrier, parity, phase index[, abortable]); the role gets
+# back True when the phase completed, False when it gave up (its time limit
+# ran out, or another role set the CTA's abort flag), as the kernel's bounded
+# waits return.  Waits that are not abortable are the drains of the stop
+# path, which wait for work already issued and ignore the abort flag.
+
+def W(bar, parity, n, abortable=True):
+    return ("wait", bar, parity, n, abortable)
+
 
 def producer(items, mut):
     kc = vc = uc = 0
+    q_armed = None              # phase index of the last arming, per barrier
+    k_armed, v_armed = {}, {}
+    ok = True
     for has1, Ts in items:
-        yield ("wait", "q_empty", (uc & 1) ^ 1, uc - 1)
+        ok = yield W("q_empty", (uc & 1) ^ 1, uc - 1)
+        if not ok:
+            break
         yield ("arm", "q_full", 2 if has1 else 1)
+        q_armed = uc
         yield ("load", "Q0", "q_full")
         if has1:
             yield ("load", "Q1", "q_full")
@@ -101,22 +117,47 @@ def producer(items, mut):
             for _ in range(T):
                 s = kc % STAGES
                 if mut != "producer_skips_k_empty":
-                    yield ("wait", f"k_empty{s}", ((kc // STAGES) & 1) ^ 1, kc // STAGES - 1)
+                    ok = yield W(f"k_empty{s}", ((kc // STAGES) & 1) ^ 1, kc // STAGES - 1)
+                    if not ok:
+                        break
                 yield ("arm", f"k_full{s}", 1)
+                k_armed[s] = kc // STAGES
                 yield ("load", f"K{s}", f"k_full{s}")
                 kc += 1
                 s = vc % STAGES
-                yield ("wait", f"v_empty{s}", ((vc // STAGES) & 1) ^ 1, vc // STAGES - 1)
+                ok = yield W(f"v_empty{s}", ((vc // STAGES) & 1) ^ 1, vc // STAGES - 1)
+                if not ok:
+                    break
                 yield ("arm", f"v_full{s}", 1)
+                v_armed[s] = vc // STAGES
                 yield ("load", f"V{s}", f"v_full{s}")
                 vc += 1
+            if not ok:
+                break
+        if not ok:
+            break
         uc += 1
+    # every load issued lands before the warp exits, on both paths: when
+    # another role gave up, this warp may still end its loop with ok (each
+    # of its last waits completed at once) while nothing consumes its loads
+    drain = mut != "producer_stops_without_drain"
+    if mut == "producer_drains_only_after_giving_up":
+        drain = not ok
+    if drain:
+        if q_armed is not None:
+            yield W("q_full", q_armed & 1, q_armed, False)
+        for s in range(STAGES):
+            if s in k_armed:
+                yield W(f"k_full{s}", k_armed[s] & 1, k_armed[s], False)
+            if s in v_armed:
+                yield W(f"v_full{s}", v_armed[s] & 1, v_armed[s], False)
 
 
 def mma(items, mut):
     kc = vc = uc = 0
     pc = [0, 0]
     oc = [0, 0]
+    ok = True
 
     def qk(k, ks):
         return ("mma", {f"Q{k}", f"K{ks}"}, {f"S{k}"})
@@ -125,11 +166,15 @@ def mma(items, mut):
         return ("mma", {f"S{k}", f"V{vs}"} | ({f"O{k}"} if acc else set()), {f"O{k}"})
 
     for has1, Ts in items:
-        yield ("wait", "q_full", uc & 1, uc)
+        ok = yield W("q_full", uc & 1, uc)
+        if not ok:
+            break
         for fi, T in enumerate(Ts):
             last_pair = fi + 1 == len(Ts)
             ks = kc % STAGES
-            yield ("wait", f"k_full{ks}", (kc // STAGES) & 1, kc // STAGES)
+            ok = yield W(f"k_full{ks}", (kc // STAGES) & 1, kc // STAGES)
+            if not ok:
+                break
             if mut == "k_released_before_qk":
                 yield ("commit", f"k_empty{ks}")
             yield qk(0, ks)
@@ -144,17 +189,23 @@ def mma(items, mut):
                 yield ("commit", "q_empty")
             for t in range(T):
                 vs = vc % STAGES
-                yield ("wait", f"v_full{vs}", (vc // STAGES) & 1, vc // STAGES)
+                ok = yield W(f"v_full{vs}", (vc // STAGES) & 1, vc // STAGES)
+                if not ok:
+                    break
                 more = t + 1 < T
                 for k in range(2):
                     if k == 1 and not has1:
                         break
                     if not (mut == "mma_skips_p_full" and k == 0):
-                        yield ("wait", f"p_full{k}", pc[k] & 1, pc[k])
+                        ok = yield W(f"p_full{k}", pc[k] & 1, pc[k])
+                        if not ok:
+                            break
                     pc[k] += 1
                     if t == 0:
                         if mut != "mma_skips_o_empty":
-                            yield ("wait", f"o_empty{k}", (oc[k] & 1) ^ 1, oc[k] - 1)
+                            ok = yield W(f"o_empty{k}", (oc[k] & 1) ^ 1, oc[k] - 1)
+                            if not ok:
+                                break
                         oc[k] += 1
                     yield pv(k, vs, t > 0)
                     if not more:
@@ -162,9 +213,13 @@ def mma(items, mut):
                     if more:
                         ks2 = kc % STAGES
                         if k == 0:
-                            yield ("wait", f"k_full{ks2}", (kc // STAGES) & 1, kc // STAGES)
+                            ok = yield W(f"k_full{ks2}", (kc // STAGES) & 1, kc // STAGES)
+                            if not ok:
+                                break
                         yield qk(k, ks2)
                         yield ("commit", f"s_full{k}")
+                if not ok:
+                    break
                 yield ("commit", f"v_empty{vs}")
                 vc += 1
                 if more:
@@ -172,21 +227,29 @@ def mma(items, mut):
                     kc += 1
                     if t + 2 == T and last_pair:
                         yield ("commit", "q_empty")
+            if not ok:
+                break
+        if not ok:
+            break
         uc += 1
     # drain: every MMA issued must finish before TMEM is released
-    yield ("commit", "drain")
-    yield ("wait", "drain", 0, 0)
+    if mut != "mma_stops_without_drain":
+        yield ("commit", "drain")
+        yield W("drain", 0, 0, False)
 
 
 def softmax_warp(k, items, rng, rescale_p, mut):
     sc = ofc = 0
     S, O = f"S{k}", f"O{k}"
+    ok = True
     for has1, Ts in items:
         if k == 1 and not has1:
             continue
         for T in Ts:
             for t in range(T):
-                yield ("wait", f"s_full{k}", sc & 1, sc)
+                ok = yield W(f"s_full{k}", sc & 1, sc)
+                if not ok:
+                    break
                 sc += 1
                 yield ("hold", S, "w")                 # read S, write P over it
                 if t > 0 and rng.random() < rescale_p:
@@ -198,12 +261,18 @@ def softmax_warp(k, items, rng, rescale_p, mut):
                 else:
                     yield ("release", S)
                     yield ("arrive", f"p_full{k}")
+            if not ok:
+                break
             if mut != "softmax_skips_o_full":
-                yield ("wait", f"o_full{k}", ofc & 1, ofc)
+                ok = yield W(f"o_full{k}", ofc & 1, ofc)
+                if not ok:
+                    break
             ofc += 1
             yield ("hold", O, "r")                     # O into registers
             yield ("release", O)
             yield ("arrive", f"o_empty{k}")
+        if not ok:
+            break
 
 
 # ---------------------------------------------------------------- scheduler
@@ -212,8 +281,13 @@ def conflicts(reads_a, writes_a, reads_b, writes_b):
     return bool(writes_a & (reads_b | writes_b)) or bool(reads_a & writes_b)
 
 
-def run(items, seed, rescale_p=0.5, mut=None, max_steps=2_000_000):
-    """Interleave the roles at random; raise Violation on any broken rule."""
+def run(items, seed, rescale_p=0.5, mut=None, timeout_p=0.0, max_steps=2_000_000):
+    """Interleave the roles at random; raise Violation on any broken rule.
+
+    timeout_p: per scheduling step, the chance that one role blocked on an
+    abortable wait runs out of time (which sets the abort flag; from then on
+    every role blocked on an abortable wait may give up).  Returns the
+    barriers and whether the run aborted."""
     rng = random.Random(seed)
     B = barriers()
     roles = {"producer": producer(items, mut), "mma": mma(items, mut)}
@@ -225,9 +299,10 @@ def run(items, seed, rescale_p=0.5, mut=None, max_steps=2_000_000):
     loads = []                 # in flight: (region, barrier)
     mma_q = []                 # in issue order: ("mma", reads, writes) | ("commit", barrier)
     holds = {}                 # role -> {region: mode}
+    aborted = False
 
     def check_wait(role, op):
-        _, name, parity, n = op
+        _, name, parity, n, _ = op
         if parity != (n & 1):
             raise Violation(f"{role}: parity {parity} for phase {n} of {name}")
         if B[name].phase > n + 1:
@@ -236,8 +311,21 @@ def run(items, seed, rescale_p=0.5, mut=None, max_steps=2_000_000):
     def mma_in_flight():
         return [op for op in mma_q if op[0] == "mma"]
 
+    def advance(role, value=None):
+        try:
+            nxt[role] = roles[role].send(value)
+        except StopIteration:
+            nxt[role] = None
+        if all(op is None for op in nxt.values()):
+            # the CTA exits (TMEM is freed): nothing of it may still be in flight
+            if mma_in_flight() or any(op[0] == "commit" for op in mma_q):
+                raise Violation("MMAs in flight when the CTA exits")
+            if loads:
+                raise Violation("loads in flight when the CTA exits")
+
     for _ in range(max_steps):
         choices = []
+        blocked = []
         for r, op in nxt.items():
             if op is None:
                 continue
@@ -245,16 +333,22 @@ def run(items, seed, rescale_p=0.5, mut=None, max_steps=2_000_000):
                 check_wait(r, op)
                 if B[op[1]].phase >= op[3] + 1:
                     choices.append(("role", r))
+                elif op[4]:
+                    blocked.append(r)
+                    if aborted:
+                        choices.append(("give_up", r))
             else:
                 choices.append(("role", r))
+        if blocked and not aborted and timeout_p and rng.random() < timeout_p:
+            choices = [("give_up", rng.choice(blocked))]
         if mma_q:
             choices.append(("mma", None))
         choices.extend(("land", i) for i in range(len(loads)))
         if not choices:
             if all(op is None for op in nxt.values()):
                 break
-            blocked = {r: op for r, op in nxt.items() if op is not None}
-            raise Violation(f"no role can proceed: {blocked}")
+            waiting = {r: op for r, op in nxt.items() if op is not None}
+            raise Violation(f"no role can proceed: {waiting}")
         kind, x = rng.choice(choices)
         if kind == "mma":
             op = mma_q.pop(0)
@@ -264,6 +358,10 @@ def run(items, seed, rescale_p=0.5, mut=None, max_steps=2_000_000):
         if kind == "land":
             region, name = loads.pop(x)
             B[name].land()
+            continue
+        if kind == "give_up":
+            aborted = True
+            advance(x, False)
             continue
         role, op = x, nxt[x]
         what = op[0]
@@ -305,19 +403,16 @@ def run(items, seed, rescale_p=0.5, mut=None, max_steps=2_000_000):
             holds.setdefault(role, {})[region] = mode
         elif what == "release":
             del holds[role][op[1]]
-        elif what == "wait":
-            pass
-        nxt[role] = next(roles[role], None)
+        advance(role, True if what == "wait" else None)
     else:
         raise Violation("step limit reached")
-    if mma_q or loads:
-        raise Violation("operations still in flight at the end")
-    for b in B.values():
-        if b.pending != b.count or b.tx != 0:
-            raise Violation(f"{b.name} ends inside a phase")
     if any(holds.values()):
         raise Violation("a region is still held at the end")
-    return B
+    if not aborted:
+        for b in B.values():
+            if b.pending != b.count or b.tx != 0:
+                raise Violation(f"{b.name} ends inside a phase")
+    return B, aborted
 
 
 def random_items(rng):
@@ -332,7 +427,8 @@ def random_items(rng):
 def test_protocol_on_random_items_and_interleavings(seed):
     rng = random.Random(1000 + seed)
     items = random_items(rng)
-    B = run(items, seed, rescale_p=rng.choice([0.0, 0.3, 1.0]))
+    B, aborted = run(items, seed, rescale_p=rng.choice([0.0, 0.3, 1.0]))
+    assert not aborted
     # every barrier completed exactly the phases its traffic implies
     n_units = sum(len(Ts) for _, Ts in items)
     n_tiles = sum(sum(Ts) for _, Ts in items)
@@ -382,3 +478,34 @@ def test_o_empty_wait_is_implied_by_p_full():
     items = [(True, [3, 2]), (True, [1, 4]), (False, [2])]
     for seed in range(40):
         run(items, seed, mut="mma_skips_o_empty")
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_stop_path_after_a_timeout(seed):
+    """A wait that runs out of time sets the CTA's abort flag; every role then
+    leaves at its next wait that has not completed.  The stop path must end
+    (its drains wait only for work already issued) and leave no TMA load or
+    MMA in flight when the CTA exits and frees its TMEM.  A producer that
+    drained only after giving up itself fails this (its last loads can be
+    in flight when the CTA exits after the MMA warp gave up)."""
+    rng = random.Random(5000 + seed)
+    items = random_items(rng)
+    aborted_runs = 0
+    for timeout_p in (0.002, 0.02, 0.2):
+        _, aborted = run(items, seed, timeout_p=timeout_p)
+        aborted_runs += aborted
+    assert aborted_runs > 0
+
+
+@pytest.mark.parametrize("mut", ["producer_stops_without_drain",
+                                 "producer_drains_only_after_giving_up",
+                                 "mma_stops_without_drain"])
+def test_stop_path_without_its_drain_is_caught(mut):
+    caught = 0
+    for items in ([(True, [2])], [(True, [3, 2]), (True, [1, 4]), (False, [2])]):
+        for seed in range(60):
+            try:
+                run(items, seed, mut=mut, timeout_p=0.05)
+            except Violation:
+                caught += 1
+    assert caught > 0, mut
