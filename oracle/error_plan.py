@@ -43,7 +43,7 @@ import numpy as np
 from .attention import merge_states
 from .groups import unit_band, unit_mask, unit_state
 from .masks import slot_pairs, slot_table
-from .plan import PLAN_FRESH, PLAN_REUSE, mass_scores, select
+from .plan import PLAN_FRESH, mass_scores, select
 
 
 def local_unit(i, group_off):

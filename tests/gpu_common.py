@@ -4,11 +4,10 @@ from __future__ import annotations
 
 import numpy as np
 
-from oracle import attention as OA
 from oracle import groups as OG
 from oracle import masks as OM
 from oracle import step as OS
-from oracle.plan import PLAN_FRESH, PLAN_REUSE
+from oracle.plan import PLAN_FRESH
 from workloads import inputs
 
 # spec tolerance against fp64 for bf16 inputs with fp32 accumulation

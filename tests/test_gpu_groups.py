@@ -13,7 +13,7 @@ torch = pytest.importorskip("torch")
 import sparse_state_reuse_b200 as dt
 from oracle import groups as OG
 from oracle import masks as OM
-from oracle.plan import PLAN_FRESH, PLAN_REUSE, mass_scores, select
+from oracle.plan import PLAN_FRESH, mass_scores, select
 from workloads import configs, inputs
 
 import gpu_common as G

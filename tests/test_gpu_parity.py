@@ -13,9 +13,8 @@ torch = pytest.importorskip("torch")
 
 import sparse_state_reuse_b200 as dt
 from sparse_state_reuse_b200 import _abi
-from oracle import attention as OA
 from oracle import masks as OM
-from oracle.plan import PLAN_FRESH, PLAN_REUSE, mass_scores, select
+from oracle.plan import PLAN_REUSE, mass_scores, select
 from oracle import step as OS
 from workloads import configs, inputs
 

@@ -18,7 +18,7 @@ import pytest
 
 from oracle import error_plan as E
 from oracle import groups, masks
-from oracle.plan import PLAN_FRESH, PLAN_REUSE, budget_target, select
+from oracle.plan import PLAN_FRESH, budget_target, select
 from workloads import configs, inputs
 
 

@@ -19,7 +19,7 @@ import torch
 
 from oracle import groups, masks, step
 from oracle.attention import merge_states
-from oracle.plan import PLAN_FRESH, PLAN_REUSE, budget_target, mass_scores, select
+from oracle.plan import PLAN_FRESH, budget_target, mass_scores, select
 
 
 def sdpa(q, k, v, mask=None):

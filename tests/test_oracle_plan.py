@@ -14,7 +14,6 @@ import os
 import numpy as np
 import pytest
 
-import oracle
 from oracle import groups, masks
 from oracle.plan import PLAN_FRESH, PLAN_REUSE, PLAN_SKIP, budget_target, mass_scores, select
 from workloads import configs

@@ -9,10 +9,8 @@
   reused pairs (reported, not gated: the pages print no error values).
 """
 import numpy as np
-import pytest
 import torch
 
-import oracle
 from oracle import masks, step
 from oracle.plan import PLAN_FRESH, PLAN_REUSE, mass_scores, select
 from workloads import configs, inputs

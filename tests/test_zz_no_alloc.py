@@ -10,7 +10,6 @@ geometry whose scratch would not fit.  This file is collected last.
 """
 import ctypes
 
-import numpy as np
 import pytest
 
 torch = pytest.importorskip("torch")

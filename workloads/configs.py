@@ -11,7 +11,7 @@ This module holds geometry and seeds only; none of the method's arithmetic.
 """
 from __future__ import annotations
 
-from dataclasses import dataclass, field
+from dataclasses import dataclass
 from typing import List, Optional
 
 
