@@ -509,3 +509,39 @@ def test_stop_path_without_its_drain_is_caught(mut):
             except Violation:
                 caught += 1
     assert caught > 0, mut
+
+
+def cta_items(part_off, fresh_rows, BH, cta, grid, BM=128, BN=128):
+    """The item list one CTA of the persistent grid walks: items are
+    (partition, batch-head, pair of 128-row Q tiles) in the kernel's order,
+    taken round-robin with stride `grid`; fresh_rows[i] lists the key counts
+    of the fresh units of partition i."""
+    P = len(part_off) - 1
+    Lmax = max(part_off[i + 1] - part_off[i] for i in range(P))
+    nqt2 = -(-Lmax // (2 * BM))
+    items = []
+    for it in range(cta, P * BH * nqt2, grid):
+        qt2, rest = it % nqt2, it // nqt2
+        i = rest // BH
+        rem = part_off[i + 1] - part_off[i] - qt2 * 2 * BM
+        if rem <= 0 or not fresh_rows[i]:
+            continue                     # not live: no role touches it
+        items.append((rem > BM, [-(-Lk // BN) for Lk in fresh_rows[i]]))
+    return items
+
+
+@pytest.mark.parametrize("cta", [0, 147])
+def test_protocol_on_a_frame_tile_cta(cta):
+    """One CTA of the 148-CTA grid on 8 frames of 3600 tokens, 24 heads, every
+    active pair fresh: about 20 items of 2 to 4 units of 29 key tiles, the
+    last Q-tile pair of each partition with a single tile of 16 rows."""
+    F, L = 8, 3600
+    part_off = [f * L for f in range(F + 1)]
+    fresh_rows = [[L] * len({0, f - 1, f, f + 1} & set(range(F))) for f in range(F)]
+    items = cta_items(part_off, fresh_rows, 24, cta, 148)
+    assert 15 <= len(items) <= 25 and any(not has1 for has1, _ in items)
+    assert {T for _, Ts in items for T in Ts} == {29}
+    for seed in range(2):
+        B, aborted = run(items, seed, rescale_p=0.05)
+        assert not aborted
+        assert B["o_full0"].phase == sum(len(Ts) for _, Ts in items)
