@@ -78,6 +78,21 @@ int main(void) {
             DITANGO_ERR_INVALID, "plan without buffers");
   CHECK(ditango_merge(&geo, NULL, NULL, NULL, NULL, NULL, NULL, 0, 0, NULL, 1, NULL, NULL, NULL) ==
             DITANGO_ERR_INVALID, "merge without buffers");
+  CHECK(ditango_plan_error(&geo, NULL, NULL, 1, 0.5, 1, 0, NULL, NULL, NULL, NULL, NULL, NULL, 0,
+                           NULL) == DITANGO_ERR_INVALID, "error plan without its state");
+  {
+    /* composing into groups that are not a coarsening of the fine ones */
+    ditango_geom fine = geo, coarse = geo;
+    int32_t fine_groups[3] = {0, 4, 8}, coarse_groups[3] = {0, 2, 8};
+    fine.G = 2;
+    fine.group_off = fine_groups;
+    coarse.G = 2;
+    coarse.group_off = coarse_groups;
+    void *fake = (void *)(uintptr_t)4096;   /* never dereferenced: refused first */
+    CHECK(ditango_cache_compose(&fine, &coarse, fake, (const float *)fake, NULL, fake,
+                                (float *)fake, NULL, 0, NULL) == DITANGO_ERR_INVALID,
+          "compose into a grouping that is not coarser");
+  }
   CHECK(ditango_selftest_bounded_wait(0, NULL, NULL) == DITANGO_ERR_INVALID, "selftest limit 0");
   CHECK(strcmp(ditango_status_string(DITANGO_ERR_TIMEOUT), "device wait timed out") == 0, "status string");
   ditango_set_wait_limit_ns(2000000);
