@@ -1,4 +1,5 @@
 import os
+import subprocess
 import sys
 
 import pytest
@@ -11,6 +12,11 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running full-size case")
+    # a fresh checkout has no library yet: build it in-tree (nvcc, sm_100a)
+    lib = os.path.join(ROOT, "sparse_state_reuse_b200", "libditango.so")
+    if not os.path.exists(lib):
+        subprocess.run([sys.executable, os.path.join(ROOT, "sparse_state_reuse_b200", "build.py")],
+                       check=True)
 
 
 @pytest.fixture(scope="session")
