@@ -547,7 +547,7 @@ def blas_threads():
         return cpu_cores()
 
 
-def run_reference(args, w):
+def run_reference(args, w, world=1):
     # a bounded sample per step: the whole run stays within a few minutes
     per_step = max(0.2, min(10.0, 150.0 / max(1, args.steps + args.warmup), args.cpu_baseline_seconds))
     for _ in range(args.warmup):
@@ -561,7 +561,7 @@ def run_reference(args, w):
     return {
         "impl": "reference",
         "metric": "effective attention TFLOP/s (fresh blocks only) at 1 B200; tokens/s",
-        "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16 values)",
@@ -601,8 +601,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
+        # the oracle runs on rank 0's host cores only; the line names the
+        # launch's GPU count so that it pairs with this arm's own line
         if rank == 0:
-            print(json.dumps(run_reference(args, w)), flush=True)
+            print(json.dumps(run_reference(args, w, max(world, args.gpus))), flush=True)
         return
 
     if world > 1:

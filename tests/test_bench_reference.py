@@ -31,3 +31,18 @@ def test_warmup_below_three_is_refused():
                         "--steps", "1", "--warmup", "2"], capture_output=True, text=True,
                        timeout=120, cwd=ROOT)
     assert r.returncode != 0 and "warmup" in r.stderr
+
+
+def test_reference_arm_under_a_launcher():
+    """Launched with N ranks, rank 0 alone times the oracle and prints the
+    line (naming N GPUs); every other rank exits 0 without work."""
+    base = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+            "--steps", "1", "--warmup", "3", "--cpu-baseline-seconds", "0.2"]
+    other = subprocess.run(base, capture_output=True, text=True, timeout=120, cwd=ROOT,
+                           env={**os.environ, "RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert other.returncode == 0 and other.stdout.strip() == ""
+    first = subprocess.run(base, capture_output=True, text=True, timeout=300, cwd=ROOT,
+                           env={**os.environ, "RANK": "0", "WORLD_SIZE": "2", "LOCAL_RANK": "0"})
+    assert first.returncode == 0, first.stderr[-2000:]
+    d = json.loads(first.stdout.strip())
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
