@@ -301,10 +301,17 @@ ditango_status ditango_plan_error(const ditango_geom *g, const float *cache_lse,
  * the library (held by every GPU that loads the library until the process
  * exits).  Returns DITANGO_ERR_UNSUPPORTED when ditango_plan_workspace_size
  * exceeds 4 MiB (anchor plans need no scratch and are never rejected).
- * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
- * The first call on a device looks up the array's device address (one
- * cudaGetSymbolAddress with that device current); make that first call
- * before any stream capture.  Every call shares the one array per device and
+ * Allocates nothing itself: no cudaMalloc, cudaFree or allocating library
+ * call.  But the CUDA runtime loads the library's device code lazily by
+ * default, so the first call on a device (in a context) is what makes the
+ * driver load the module and reserve the 4 MiB array; that first load can
+ * fail under memory pressure.  A caller whose allocator is frozen should
+ * make one call per device at start-up (it must anyway come before any
+ * stream capture), or run with CUDA_MODULE_LOADING=EAGER.
+ * The array's device address is looked up with cudaGetSymbolAddress, with
+ * the device current, on the first call in each context and cached with the
+ * context's unique ID; after cudaDeviceReset (a new context) the next call
+ * looks it up again.  Every call shares the one array per device and
  * overwrites all of the scratch it reads, so nothing carries over between
  * calls; but calls that overlap on the GPU (other streams, concurrent graph
  * branches) race on it -- order them. */

@@ -157,8 +157,10 @@ class Schedule:
         plan_override: execute this plan instead of the one planned (the
         planner state still advances from the planned scores and the
         executed plan), so that a run of another implementation can be
-        followed step by step."""
+        followed step by step; the plan the oracle made itself is kept in
+        self.planned."""
         plan, score = self.plan(s)
+        self.planned = plan          # the oracle's own plan, before any override
         if plan_override is not None:
             plan = np.asarray(plan_override, dtype=np.int8).reshape(self.Au.shape)
         N, d = self.q[0].shape

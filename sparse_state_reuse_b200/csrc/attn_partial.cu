@@ -198,14 +198,18 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // 2^x on the FMA/ALU pipes, to take part of the exponentials off the
-// special-function unit.  Range reduction to the nearest integer with the
-// 1.5 * 2^23 rounding constant (x = n + f, f in [-1/2, 1/2]); 2^f by a
-// degree-3 polynomial fitted here for minimum relative error on [-1/2, 1/2]
-// (max relative error 1.0e-4, far below the bf16 rounding P gets next);
-// 2^n by adding n to the exponent field.  Inputs below -126 give ~0.
+// special-function unit.  Range reduction in the style of Cody and Waite, to
+// the nearest integer with the 1.5 * 2^23 rounding constant (x = n + f,
+// f in [-1/2, 1/2]); 2^f by a cubic whose constant term is fixed at 1 (so
+// integer inputs are exact) and whose other coefficients are the minimax
+// (Chebyshev) fit of the relative error on [-1/2, 1/2], computed as a linear
+// program over a dense grid -- the optimum the Remez exchange algorithm
+// converges to; max relative error 1.013e-4, far below the bf16 rounding P
+// gets next; 2^n by adding n to the exponent field.  Inputs below -126
+// give ~0.
 constexpr float kExpC1 = 0.6932829022f;
-constexpr float kExpC2 = 0.2422106713f;
-constexpr float kExpC3 = 0.0550087579f;
+constexpr float kExpC2 = 0.2422109693f;
+constexpr float kExpC3 = 0.0550090596f;
 __device__ __forceinline__ float exp2_poly(float x) {
   x = fmaxf(x, -126.0f);
   const float kRound = 12582912.0f;  // 1.5 * 2^23

@@ -447,12 +447,49 @@ ditango_status ditango_selftest_bounded_wait(int64_t limit_ns, int32_t *dev_stat
 // denoising steps.  They still pass their own inputs and outputs, but the
 // plan's scratch (the per-chunk mass sums) lives here, in a fixed device
 // array of this library of kNoAllocPlanScratchBytes.  Every GPU that loads
-// the library holds that array until the process exits.
+// the library holds that array until the process exits (or until its context
+// is destroyed).
+//
+// The array's host-side name is not a device address: its address is asked
+// of the runtime with the device current, and cached per device together
+// with the unique ID of the context it belongs to.  A new context on the
+// device (after cudaDeviceReset, say) has a new ID, and the address is then
+// looked up again instead of reusing one that points into freed memory.
 namespace {
 constexpr size_t kNoAllocPlanScratchBytes = size_t(4) << 20;  // 4 MiB
 constexpr int kNoAllocMaxDevices = 64;
+
+struct NoAllocScratch {
+  unsigned long long ctx_id;  // context the address belongs to
+  void *ptr;                  // null: not looked up in that context yet
+};
 std::mutex g_noalloc_mu;
-void *g_noalloc_scratch[kNoAllocMaxDevices] = {};
+NoAllocScratch g_noalloc_scratch[kNoAllocMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// Unique ID (for the life of the process) of the calling thread's current
+// context; false when no context is current or the driver has no such call.
+bool current_context_id(unsigned long long *id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
 }  // namespace
 
 static __device__ __align__(256) unsigned char g_plan_scratch[kNoAllocPlanScratchBytes];
@@ -475,16 +512,25 @@ extern "C" ditango_status ditango_plan_noalloc(const ditango_geom *g, const floa
   if (dev < 0 || dev >= kNoAllocMaxDevices) return DITANGO_ERR_UNSUPPORTED;
   void *scratch = nullptr;
   {
-    // once per device, with that device current: the host-side name of the
-    // array is not a device address; ask the runtime for the real one.
+    // with this device current: the cached address if it belongs to the
+    // current context, else ask the runtime for it (the first ask in a
+    // context also makes the primary context current on this thread)
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_scratch[dev]) {
+    NoAllocScratch &e = g_noalloc_scratch[dev];
+    unsigned long long id = 0;
+    bool have_id = current_context_id(&id);
+    if (have_id && e.ptr != nullptr && e.ctx_id == id) {
+      scratch = e.ptr;
+    } else {
       void *p = nullptr;
-      cudaError_t e = cudaGetSymbolAddress(&p, g_plan_scratch);
-      if (e != cudaSuccess || p == nullptr) return cuda_status(e == cudaSuccess ? cudaErrorUnknown : e);
-      g_noalloc_scratch[dev] = p;
+      cudaError_t err = cudaGetSymbolAddress(&p, g_plan_scratch);
+      if (err != cudaSuccess || p == nullptr)
+        return cuda_status(err == cudaSuccess ? cudaErrorUnknown : err);
+      if (!have_id) have_id = current_context_id(&id);
+      e.ptr = have_id ? p : nullptr;   // without a context ID: look it up every call
+      e.ctx_id = have_id ? id : 0;
+      scratch = p;
     }
-    scratch = g_noalloc_scratch[dev];
   }
   const int target = plan_target(&dg, band_k, budget);
   return cuda_status(launch_plan(dg, cache_lse, cache_valid, band_k, target, anchor ? 1 : 0,

@@ -21,7 +21,7 @@ def test_reference_arm_prints_one_json_line():
                 "cpu_baseline", "e2e"):
         assert key in d, key
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s"
-    assert d["config"]["workload"] == "frame_tile_8x3600"
+    assert d["config"]["workload"] == "dense_p16"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
 

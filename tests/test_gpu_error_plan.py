@@ -4,12 +4,15 @@ a drifting multi-step schedule.
 
 Per step: the plan equals the oracle's selection run on the GPU's own score
 array (bit for bit: the hard gate where floating point decides an integer);
-the local drift delta, the held importance w, the ages and the scores agree
-with the oracle's fp64 values within tolerances derived from fp32 log-sum-
-exps; the merged output agrees with the oracle (max-abs 2e-2, mean-abs 2e-3).
-The oracle follows the plan the GPU executed, so that both caches hold states
-of the same steps.  Whether the oracle, left alone, would pick the same units
-is reported (it may differ only where scores tie within fp32 resolution)."""
+the oracle's own plan -- its selection on its own fp64 scores -- equals the
+GPU's, except units whose oracle score lies within 1e-5 relative of the cut
+(each listed); the local drift delta, the held importance w, the ages and
+the scores agree with the oracle's fp64 values within tolerances set by the
+fp32 log-sum-exps they are made of; the merged output agrees with the oracle
+(max-abs 2e-2, mean-abs 2e-3).  The oracle executes the GPU's plan, which by
+the check above differs from its own only on such ties, so that both caches
+hold states of the same steps.
+"""
 import numpy as np
 import pytest
 
@@ -58,7 +61,11 @@ def test_schedule_matches_oracle(gs, frames, sb):
     Q = to_dev(np.stack(q_bits)[None])
     out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
     out_lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
-    agree = 0
+    ties, worst = [], {"delta": 0.0, "w": 0.0, "age": 0.0, "score": 0.0}
+
+    def rel(got, want, floor):
+        return float((np.abs(got - want) / np.maximum(np.abs(want), floor)).max())
+
     for s in range(S + 1):
         K = to_dev(np.stack([k_steps[h][s] for h in range(w.H)])[None])
         V = to_dev(np.stack([v_steps[h][s] for h in range(w.H)])[None])
@@ -67,28 +74,45 @@ def test_schedule_matches_oracle(gs, frames, sb):
         assert pa.status.item() == 0
         plan_g = pa.plan.cpu().numpy().reshape(Au.shape)
         score_g = pa.score.cpu().numpy().reshape(Au.shape)
-        plan_o, score_o, O_o, l_o = sch.step(s, [f64(k_steps[h][s]) for h in range(w.H)],
-                                             [f64(v_steps[h][s]) for h in range(w.H)], plan_override=plan_g)
+        _, score_o, O_o, l_o = sch.step(s, [f64(k_steps[h][s]) for h in range(w.H)],
+                                        [f64(v_steps[h][s]) for h in range(w.H)], plan_override=plan_g)
+        own = sch.planned
         if s % every == 0:
-            assert (plan_g[Au] == PLAN_FRESH).all()
+            assert (plan_g[Au] == PLAN_FRESH).all() and (own == plan_g).all()
         else:
             # hard gate: the selection rule on the GPU's own scores is the GPU plan
             valid_pp = np.ones(Au.shape, dtype=bool)
             sel, _ = select(score_g.astype(np.float64), Au, 0, w.budget, band=band, valid=valid_pp)
             assert (sel == plan_g).all(), (s, sel, plan_g)
+            # the oracle's own plan: equal, but for units tied at the cut
+            cand = Au & ~band
+            chosen = cand & (own == PLAN_FRESH)
+            if chosen.any() and (cand & ~chosen).any():
+                cut = score_o[chosen].min()
+                for i, c in zip(*np.nonzero(own != plan_g)):
+                    assert abs(score_o[i, c] - cut) <= 1e-5 * cut, \
+                        f"step {s}: the oracle would plan unit {(i, c)} differently " \
+                        f"(score {score_o[i, c]:.6e}, cut {cut:.6e})"
+                    ties.append((s, int(i), int(c)))
+            else:
+                assert (own == plan_g).all(), (s, own, plan_g)
             d_g = ep.delta.cpu().numpy()
-            np.testing.assert_allclose(d_g, sch.delta, rtol=2e-2, atol=1e-4, err_msg=f"delta step {s}")
+            worst["delta"] = max(worst["delta"], rel(d_g, sch.delta, 1e-3))
+            np.testing.assert_allclose(d_g, sch.delta, rtol=5e-3, atol=1e-5, err_msg=f"delta step {s}")
             if s > 1:
                 assert (d_g > 0).all()
-            np.testing.assert_allclose(ep.w.cpu().numpy().reshape(Au.shape), sch.w, rtol=1e-3, atol=1e-6,
-                                       err_msg=f"w step {s}")
-            np.testing.assert_allclose(ep.age.cpu().numpy()[:len(sch.age)], sch.age, rtol=3e-2, atol=3e-4,
-                                       err_msg=f"age step {s}")
-            np.testing.assert_allclose(score_g, score_o, rtol=3e-2, atol=1e-5, err_msg=f"score step {s}")
-            agree += int((plan_o == plan_g).all())
+            w_g = ep.w.cpu().numpy().reshape(Au.shape)
+            worst["w"] = max(worst["w"], rel(w_g[Au], sch.w[Au], 1e-3))
+            np.testing.assert_allclose(w_g, sch.w, rtol=1e-4, atol=1e-7, err_msg=f"w step {s}")
+            a_g = ep.age.cpu().numpy()[:len(sch.age)]
+            worst["age"] = max(worst["age"], rel(a_g, sch.age, 1e-3))
+            np.testing.assert_allclose(a_g, sch.age, rtol=5e-3, atol=1e-5, err_msg=f"age step {s}")
+            worst["score"] = max(worst["score"], rel(score_g[Au], score_o[Au], 1e-4))
+            np.testing.assert_allclose(score_g, score_o, rtol=5e-3, atol=1e-6, err_msg=f"score step {s}")
         G.assert_close(out.cpu().numpy()[0], O_o, f"out step {s}")
         G.assert_close(out_lse.cpu().numpy()[0], l_o, f"lse step {s}")
-    print(f"oracle's own plan equal to the GPU's on {agree} of {S - S // every} non-anchor steps")
+    print(f"oracle's own plan equal to the GPU's on every non-anchor step but for ties at the cut: "
+          f"{ties}; largest relative differences {worst}")
 
 
 def test_anchor_every_step_is_all_fresh():

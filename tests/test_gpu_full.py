@@ -10,7 +10,7 @@ torch = pytest.importorskip("torch")
 import sparse_state_reuse_b200 as dt
 from oracle import groups as OG
 from oracle import masks as OM
-from oracle.plan import PLAN_FRESH, mass_scores, select
+from oracle.plan import PLAN_FRESH, PLAN_REUSE, mass_scores, select
 from workloads import configs, inputs
 
 import gpu_common as G
@@ -31,6 +31,9 @@ def sample_rows(w, i, n=24):
 
 
 def run_workload(w, out_dtype=torch.float32, state_bf16=False):
+    """The benchmark's step on the full-size workload.  Returns the
+    PartitionedAttention, the output, its lse and, for a reuse workload, a
+    host copy of the cache (lse, valid bits) the plan was computed from."""
     Q, K, V = G.upload(w)
     pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask(),
                                  state_bf16=state_bf16,
@@ -42,10 +45,78 @@ def run_workload(w, out_dtype=torch.float32, state_bf16=False):
         del Kp, Vp
     out = torch.empty((w.B, w.H, w.N, w.d), dtype=out_dtype, device="cuda")
     out_lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
-    pa.step(Q, K, V, out, out_lse, band_k=w.band_k, budget=w.budget, anchor=w.anchor)
+    pa.check_inputs(Q, K, V, out, out_lse)
+    pa.plan_step(w.band_k, w.budget, w.anchor)
+    snap = None
+    if w.reuses:
+        torch.cuda.synchronize()
+        snap = (pa.state_lse.cpu().numpy(), pa.valid.cpu().numpy().astype(bool))
+    pa.partial(Q, K, V)
+    pa.merge(out, out_lse)
     torch.cuda.synchronize()
     assert pa.status.item() == 0
-    return pa, out, out_lse
+    return pa, out, out_lse, snap
+
+
+def check_plan_hard_gate(w, pa, snap):
+    """The plan on the workload's real cache (the anchor step's states on the
+    previous K/V):
+      * the oracle's selection run on the GPU's own float32 scores equals
+        the GPU plan and fresh list bit for bit;
+      * the GPU scores equal the oracle's fp64 mass scores of the same cached
+        lse within 1e-5 relative;
+      * the oracle's selection on its own fp64 scores equals the GPU plan,
+        except units within 1e-5 relative of the cut (listed; none expected).
+    Returns the relative margin at the cut (None when nothing is ranked)."""
+    lse, valid = snap
+    A, band = G.unit_masks(w)
+    C = A.shape[1]
+    plan = pa.plan.cpu().numpy().reshape(w.P, C)
+    n_fresh = int(pa.counts[0].item())
+    fl = pa.fresh_list.cpu().numpy()[:n_fresh]
+    score = pa.score.cpu().numpy().reshape(w.P, C)
+    valid_pc = np.ones((w.P, C), dtype=bool)
+    valid_pc[A] = valid
+    plan_s, fl_s = select(score.astype(np.float64), A, w.band_k, w.budget, valid=valid_pc, band=band)
+    assert (plan_s == plan).all(), "selection on the GPU's scores differs from the GPU plan"
+    assert (fl_s == fl).all(), "fresh list differs"
+    w_o = mass_scores(lse, A, w.part_off(), valid=valid)
+    np.testing.assert_allclose(score[A], w_o[A], rtol=1e-5, atol=0)
+    plan_o, _ = select(w_o, A, w.band_k, w.budget, valid=valid_pc, band=band)
+    cand = A & ~band & valid_pc
+    sel = cand & (plan_o == PLAN_FRESH)
+    rest = cand & (plan_o == PLAN_REUSE)
+    if not sel.any() or not rest.any():
+        assert (plan_o == plan).all()
+        return None
+    cut_in, cut_out = w_o[sel].min(), w_o[rest].max()
+    margin = (cut_in - cut_out) / cut_in
+    near = [(int(i), int(c)) for i, c in zip(*np.nonzero(cand))
+            if abs(w_o[i, c] - cut_in) <= 1e-5 * cut_in]
+    print(f"{w.name}: {int(sel.sum())} units chosen by mass, relative margin at the cut "
+          f"{margin:.3e}, units within 1e-5 of the cut (the cut unit included): {near}")
+    diff = plan_o != plan
+    for i, c in zip(*np.nonzero(diff)):
+        assert abs(w_o[i, c] - cut_in) <= 1e-5 * cut_in, (i, c, w_o[i, c], cut_in)
+    return margin
+
+
+def check_cached_states(w, pa, states, b, h, i, rows):
+    """Every active pair's state of these rows as the cache holds it after the
+    step -- this step's fresh states and the reused ones -- against the
+    oracle's state of the same pair (current K/V when fresh, previous K/V
+    when reused).  A wrong state of small weight can hide in the merged
+    output; here each is compared on its own."""
+    slot = OM.slot_table(OM.pair_mask(w.part_off(), w.frame_off(), w.frame_mask()))
+    bh = b * w.H + h
+    loc = torch.as_tensor(rows - w.part_off()[i], device="cuda")
+    for j, (Oj, lj, code) in states.items():
+        s = int(slot[i, j])
+        got_O = pa.state_O[s, bh].index_select(0, loc).float().cpu().numpy()
+        got_l = pa.state_lse[s, bh].index_select(0, loc).cpu().numpy()
+        kind = "fresh" if code == PLAN_FRESH else "reused"
+        G.assert_close(got_O, Oj, f"{w.name} cached O of {kind} pair {(i, j)} bh{bh}")
+        G.assert_close(got_l, lj, f"{w.name} cached lse of {kind} pair {(i, j)} bh{bh}")
 
 
 @pytest.mark.parametrize("w,sb", [(configs.FRAME_TILE, False), (configs.DITANGO_REUSE, False),
@@ -55,21 +126,25 @@ def run_workload(w, out_dtype=torch.float32, state_bf16=False):
                          ids=["frame_tile", "reuse_p32", "long_video", "dense",
                               "reuse_p32_bf16_cache", "long_video_bf16_cache", "groups_p32_g4"])
 def test_full_size_sampled_rows(w, sb):
-    pa, out, out_lse = run_workload(w, state_bf16=sb)
+    pa, out, out_lse, snap = run_workload(w, state_bf16=sb)
     plan = pa.plan.cpu().numpy().reshape(w.P, w.G)
     G.check_plan_valid(w, plan)
     counts = pa.counts.cpu().numpy()
     assert counts[0] == int((plan == PLAN_FRESH).sum())
+    if snap is not None:
+        check_plan_hard_gate(w, pa, snap)
     bhs = sorted({0, w.BH - 1, w.BH // 2})
     parts = sorted({0, w.P // 2, w.P - 1})
     for bh in bhs:
         b, h = divmod(bh, w.H)
         for i in parts:
             rows = sample_rows(w, i)
-            Oo, lo, _ = G.oracle_rows(w, plan, b, h, i, rows)
+            Oo, lo, states = G.oracle_rows(w, plan, b, h, i, rows)
             rt = torch.as_tensor(rows, device="cuda")
             G.assert_close(out[b, h].index_select(0, rt).cpu().numpy(), Oo, f"{w.name} out bh{bh} p{i}")
             G.assert_close(out_lse[b, h].index_select(0, rt).cpu().numpy(), lo, f"{w.name} lse bh{bh} p{i}")
+            if states is not None:
+                check_cached_states(w, pa, states, b, h, i, rows)
     if w.anchor and w.F == 0:
         # all fresh, unmasked: the merged output is unpartitioned attention
         from oracle.attention import dense_attention

@@ -9,6 +9,9 @@ call's contents, which must not leak into the next), and it must refuse a
 geometry whose scratch would not fit.  This file is collected last.
 """
 import ctypes
+import os
+import shutil
+import subprocess
 
 import pytest
 
@@ -20,6 +23,8 @@ from oracle import masks as OM
 from workloads import configs, inputs
 
 pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 if not torch.cuda.is_available():
     pytest.skip("no CUDA device", allow_module_level=True)
@@ -80,3 +85,38 @@ def test_noalloc_anchor_plan_and_size_limit():
     with pytest.raises(dt.DitangoError) as e:
         dt.ditango_plan_noalloc(big, lse, None, 1, 0.5, 0, *bufs)
     assert e.value.status == 2
+
+
+def test_noalloc_call_takes_no_device_memory():
+    """After a first call on the device (which loads the library's device
+    code, the array included), further calls change no free-memory count."""
+    w = configs.DITANGO_REUSE
+    g = dt.Geometry(w.B, w.H, w.N, w.d, w.part_off())
+    pairs = OM.slot_pairs(OM.pair_mask(w.part_off()))
+    n = len(pairs)
+    lse = torch.from_numpy(inputs.synthetic_cache_lse(w, n, pairs, seed=w.seed + 31)).cuda()
+    bufs = _buffers(w.P, n)
+    dt.ditango_plan_noalloc(g, lse, None, w.band_k, w.budget, 0, *bufs)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        dt.ditango_plan_noalloc(g, lse, None, w.band_k, w.budget, 0, *bufs)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
+
+
+def test_noalloc_after_device_reset(tmp_path):
+    """A plain C program plans with both entry points, resets the device and
+    plans again, three times: the allocation-free plan must look its array
+    up again in every new context and keep matching ditango_plan."""
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    exe = str(tmp_path / "noalloc_reset")
+    libdir = os.path.dirname(dt.LIB_PATH)
+    r = subprocess.run([nvcc, "-O1", "-Wno-deprecated-gpu-targets", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c", "noalloc_reset.c"), "-L", libdir, "-lditango",
+                        "-Xlinker", "-rpath=" + libdir, "-o", exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stdout + run.stderr
+    assert run.stdout.count("equal") == 3, run.stdout
