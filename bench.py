@@ -60,16 +60,20 @@ def fresh_pairs_of_units(w, plan_units, A_pairs):
     return A_pairs & (plan_units[:, col] == 1)
 
 
-def merge_bytes(w, A, fresh_mask, out_bytes_per_elem=2, writeback=False, state_o_bytes=4):
+def merge_bytes(w, A, fresh_mask, out_bytes_per_elem=2, writeback=False, state_o_bytes=4,
+                mass_partials=True):
     """Algorithmic HBM bytes of the merge: every active state read once
     (d O values of state_o_bytes each + an fp32 lse per row), the output
-    written once (d elements + fp32 lse), plus the write-back of fresh states
-    when they are copied."""
+    written once (d elements + fp32 lse), the mass partials (one float per
+    KV column per block of 128 rows of each (b*h, partition)), plus the
+    write-back of fresh states when they are copied."""
     po = np.array(w.part_off())
     L = np.diff(po)
     rows_states = (A.sum(axis=1) * L).sum() * w.BH
     row_state = w.d * state_o_bytes + 4
     b = rows_states * row_state + w.BH * w.N * (w.d * out_bytes_per_elem + 4)
+    if mass_partials:
+        b += float(np.ceil(L / 128.0).sum()) * w.BH * A.shape[1] * 4
     if writeback:
         b += (fresh_mask.sum(axis=1) * L).sum() * w.BH * row_state
     return float(b)
@@ -84,10 +88,11 @@ def load_peaks():
 
 
 def kernel_source_hash(name):
-    src = os.path.join(ROOT, "sparse_state_reuse_b200", "csrc", name)
+    csrc = os.path.join(ROOT, "sparse_state_reuse_b200", "csrc")
+    files = [name, "common.cuh"] + (["weights.cuh"] if name in ("merge.cu", "plan.cu") else [])
     h = hashlib.sha256()
-    for f in (src, os.path.join(ROOT, "sparse_state_reuse_b200", "csrc", "common.cuh")):
-        h.update(open(f, "rb").read())
+    for f in files:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -213,7 +218,8 @@ def run_ours(args, w, rank, world, local_rank):
     fresh = plan == 1
     flops = effective_flops(w, fresh_pairs_of_units(w, plan, pair_mask(w)))
     mbytes = merge_bytes(w, A, fresh, state_o_bytes=2 if args.state_bf16 else 4)
-    launches_per_step = (1 if w.anchor else 2) + 1 + 1
+    # plan (selection alone: the merge before it left the mass score), attention, merge
+    launches_per_step = 3
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     n_ev = args.steps
@@ -362,9 +368,9 @@ def run_ours(args, w, rank, world, local_rank):
                            "kernel_ms": round(merge_ms, 4),
                            "algorithmic_bytes_per_launch": mbytes,
                            "traffic": recorded_traffic("merge.cu", w.name)},
-        "plan": {"us": round(plan_us, 2), "launches": 1 if w.anchor else 2,
-                 "note": "selection alone on anchor steps; mass score over the cached lse + "
-                         "selection otherwise"},
+        "plan": {"us": round(plan_us, 2), "launches": 1,
+                 "note": "selection alone: anchor steps need no mass score, and reuse steps take "
+                         "it from the previous step's merge (mass partials)"},
         "e2e": {"value": round(aggregate_tflops(world, flops, e2e_ms), 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

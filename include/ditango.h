@@ -126,7 +126,9 @@ int64_t ditango_state_rows(const ditango_geom *g);
  * -1 for masked units (row-major rank of the active units). */
 ditango_status ditango_slot_table(const ditango_geom *g, int32_t *slot_out);
 
-/* Bytes of device scratch ditango_plan needs. */
+/* Bytes of device scratch ditango_plan needs; also the size of the mass
+ * partials ditango_merge can emit (the same layout: float32 block sums
+ * [P][B*H][ceil(Lmax / 128)][G + 1], see ditango_merge). */
 size_t ditango_plan_workspace_size(const ditango_geom *g);
 
 /* Plan: per unit, fresh or reuse (DiTango, 1. Anchor-Guided Selection
@@ -155,6 +157,26 @@ ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
                             int32_t anchor, int8_t *plan, int32_t *fresh_list,
                             int32_t *counts, float *score_out, void *workspace,
                             size_t workspace_bytes, ditango_stream stream);
+
+/* Plan from mass partials: ditango_plan with its first stage (the mass
+ * score read from the cache) replaced by the block sums a ditango_merge
+ * call emitted (its mass_partials argument) -- DiTango, "Anchor Steps":
+ * the importance w is refreshed from the states just composed, without
+ * reading the cache again.  The partials describe the cache as that merge
+ * left it (every state it composed counts as valid); after anything else
+ * has changed the cache (states invalidated or written by another call, a
+ * composition), plan with ditango_plan instead.  The same selection,
+ * outputs and determinism as ditango_plan; given the partials of a merge
+ * whose composed states are the cache's valid states, the plan and scores
+ * are bit-identical to ditango_plan's on that cache.
+ *   mass_partials  dev, written by ditango_merge, mass_bytes >=
+ *                  ditango_plan_workspace_size (else INVALID).
+ *   cache_valid    as for ditango_plan (invalid slots are forced fresh). */
+ditango_status ditango_plan_from_mass(const ditango_geom *g, const float *mass_partials,
+                                     size_t mass_bytes, const uint8_t *cache_valid,
+                                     int32_t band_k, double budget, int8_t *plan,
+                                     int32_t *fresh_list, int32_t *counts, float *score_out,
+                                     ditango_stream stream);
 
 /* Partial attention states of the fresh units (tcgen05 tensor cores, TMA).
  * For each fresh unit (i, c) = fresh_list[f], f < counts[0] (read on the
@@ -199,7 +221,10 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q,
  * fresh states read from part_O/part_lse (indexed by fresh-list position)
  * and reused ones from cache_O/cache_lse (indexed by slot).  part_O = NULL
  * means the fresh states were already written into the cache slots
- * (ditango_attn_partial with out_by_slot = 1).
+ * (ditango_attn_partial with out_by_slot = 1).  The weights
+ * exp(lse_c - L) of a row are computed in a fixed order (largest lse first
+ * subtracted, a fixed summation tree), shared with ditango_plan's mass
+ * score.
  *   plan          dev int8 [P*G] from ditango_plan.
  *   writeback     nonzero: also copy each fresh state into its cache slot
  *                 and mark cache_valid (ignored when part_O is NULL).
@@ -207,13 +232,20 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q,
  *   out           dev [B, H, N, d] (element strides out_strides for b, h, n;
  *                 NULL = contiguous), bf16 bits (out_is_fp32 = 0) or float32.
  *   out_lse       dev float32 [B, H, N] or NULL.
+ *   mass_partials dev float32 of ditango_plan_workspace_size bytes, or NULL:
+ *                 receives, per (query partition i, b*h, block of 128 rows),
+ *                 every active unit's sum of its weights over the block's
+ *                 rows (0 for a unit the plan skipped) -- the next step's
+ *                 importance w before averaging (DiTango, "Anchor Steps":
+ *                 refreshed from the states just composed); pass it to
+ *                 ditango_plan_from_mass.  Column G is not written.
  * A token whose partition has no active pair gets O = 0, lse = -inf. */
 ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan,
                              const void *part_O, const float *part_lse,
                              void *cache_O, float *cache_lse, uint8_t *cache_valid,
                              int32_t writeback, int32_t state_bf16, void *out,
                              int32_t out_is_fp32, const int64_t *out_strides,
-                             float *out_lse, ditango_stream stream);
+                             float *out_lse, float *mass_partials, ditango_stream stream);
 
 /* Cache update: copy the fresh states (indexed by fresh position) into their
  * cache slots and mark them valid -- the write half of an anchor step

@@ -23,7 +23,7 @@ from ._abi import (  # noqa: F401
     ditango_slot_table, ditango_plan_workspace_size, ditango_plan, ditango_attn_partial,
     ditango_merge, ditango_cache_update, ditango_set_wait_limit_ns,
     ditango_selftest_bounded_wait, ditango_plan_noalloc, ditango_cache_compose, status_string,
-    ditango_plan_error, error_state,
+    ditango_plan_error, error_state, ditango_plan_from_mass,
 )
 
 
@@ -90,6 +90,9 @@ class PartitionedAttention:
         self.ws_bytes = ditango_plan_workspace_size(self.geom)
         self.workspace = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        # the workspace holds the mass partials of the last merge, and the
+        # cache has not changed since: the next plan need not read the cache
+        self.mass_from_merge = False
 
     def _geometry(self, strides):
         s = strides or (None, None, None)
@@ -116,9 +119,18 @@ class PartitionedAttention:
             self.geom = self._geometry(want)
 
     def plan_step(self, band_k=0, budget=1.0, anchor=False, stream=None):
-        ditango_plan(self.geom, None if anchor else self.state_lse, self.valid, band_k, budget,
-                     anchor, self.plan, self.fresh_list, self.counts, self.score, self.workspace,
-                     self.ws_bytes, stream)
+        """The plan of the next attention call.  After a merge (which left the
+        mass score of the states it composed in the workspace) the selection
+        runs alone; otherwise the mass score is read from the cache."""
+        if not anchor and self.mass_from_merge:
+            ditango_plan_from_mass(self.geom, self.workspace, self.ws_bytes, self.valid, band_k,
+                                   budget, self.plan, self.fresh_list, self.counts, self.score,
+                                   stream)
+        else:
+            ditango_plan(self.geom, None if anchor else self.state_lse, self.valid, band_k, budget,
+                         anchor, self.plan, self.fresh_list, self.counts, self.score,
+                         self.workspace, self.ws_bytes, stream)
+        self.mass_from_merge = False
 
     def partial(self, Q, K, V, scale=0.0, stream=None, drift_rows=None):
         import torch
@@ -127,6 +139,7 @@ class PartitionedAttention:
             check_tensor(drift_rows, "drift_rows", (self.P, self.B * self.H, self.Lmax),
                          (torch.float32,), contiguous=True)
         self._bind(Q, K, V)
+        self.mass_from_merge = False
         ditango_attn_partial(self.geom, Q, K, V, self.fresh_list, self.counts, scale,
                              self.state_O, self.state_lse, 1, self.valid, self.status, stream,
                              state_bf16=self.state_bf16, drift_rows=drift_rows)
@@ -140,7 +153,8 @@ class PartitionedAttention:
                          contiguous=True)
         ditango_merge(self.geom, self.plan, None, None, self.state_O, self.state_lse, self.valid, 0,
                       out, out.dtype == torch.float32, tuple(out.stride()[:3]), out_lse, stream,
-                      state_bf16=self.state_bf16)
+                      state_bf16=self.state_bf16, mass_partials=self.workspace)
+        self.mass_from_merge = True
 
     def step(self, Q, K, V, out, out_lse=None, band_k=0, budget=1.0, anchor=False, scale=0.0,
              stream=None):

@@ -72,8 +72,10 @@ _SIGS = {
     "ditango_plan_error": (C.c_int, [_G, _P, _P, C.c_int32, C.c_double, C.c_int32, C.c_int32,
                                      C.POINTER(ditango_error_state), _P, _P, _P, _P, _P,
                                      C.c_size_t, _P]),
+    "ditango_plan_from_mass": (C.c_int, [_G, _P, C.c_size_t, _P, C.c_int32, C.c_double, _P, _P,
+                                         _P, _P, _P]),
     "ditango_merge": (C.c_int, [_G, _P, _P, _P, _P, _P, _P, C.c_int32, C.c_int32, _P, C.c_int32,
-                                _P, _P, _P]),
+                                _P, _P, _P, _P]),
     "ditango_cache_update": (C.c_int, [_G, _P, _P, _P, _P, _P, _P, C.c_int32, _P]),
     "ditango_plan_noalloc": (C.c_int, [_G, _P, _P, C.c_int32, C.c_double, C.c_int32, _P, _P, _P,
                                        _P, _P]),
@@ -227,8 +229,18 @@ def ditango_plan_error(geom, cache_lse, cache_valid, band_k, budget, anchor, ref
         _ptr(counts), _ptr(score_out), _ptr(workspace), int(workspace_bytes), _stream(stream)))
 
 
+def ditango_plan_from_mass(geom, mass_partials, mass_bytes, cache_valid, band_k, budget, plan,
+                           fresh_list, counts, score_out=None, stream=None):
+    """ditango_plan with the mass score taken from a merge's mass partials."""
+    _check("ditango_plan_from_mass", _lib.ditango_plan_from_mass(
+        geom.ref, _ptr(mass_partials), int(mass_bytes), _ptr(cache_valid), int(band_k),
+        float(budget), _ptr(plan), _ptr(fresh_list), _ptr(counts), _ptr(score_out),
+        _stream(stream)))
+
+
 def ditango_merge(geom, plan, part_O, part_lse, cache_O, cache_lse, cache_valid, writeback,
-                  out, out_is_fp32, out_strides=None, out_lse=None, stream=None, state_bf16=0):
+                  out, out_is_fp32, out_strides=None, out_lse=None, stream=None, state_bf16=0,
+                  mass_partials=None):
     strides = None
     if out_strides is not None:
         strides = (C.c_int64 * 3)(*[int(s) for s in out_strides])
@@ -237,7 +249,7 @@ def ditango_merge(geom, plan, part_O, part_lse, cache_O, cache_lse, cache_valid,
         _ptr(cache_valid), int(bool(writeback)), int(bool(state_bf16)), _ptr(out),
         int(bool(out_is_fp32)),
         C.cast(strides, C.c_void_p) if strides is not None else None, _ptr(out_lse),
-        _stream(stream)))
+        _ptr(mass_partials), _stream(stream)))
 
 
 def ditango_cache_update(geom, plan, part_O, part_lse, cache_O, cache_lse, cache_valid,

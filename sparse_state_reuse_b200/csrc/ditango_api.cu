@@ -21,12 +21,12 @@ cudaError_t launch_plan(const DevGeom &g, const float *cache_lse, const unsigned
                         int band_k, int target, int anchor, signed char *plan_out, int *fresh_list,
                         int *counts, float *score_out, void *workspace, cudaStream_t stream,
                         const float *drift_rows, float *w_hold, float *age, float *delta,
-                        unsigned char *local_ok, int refresh_w);
+                        unsigned char *local_ok, int refresh_w, int mass_given);
 cudaError_t launch_merge(const DevGeom &g, const signed char *plan, const void *part_O,
                          const float *part_lse, void *cache_O, float *cache_lse,
                          unsigned char *cache_valid, int writeback, int state_bf16, void *out,
                          int out_is_fp32, long long osb, long long osh, long long osn,
-                         float *out_lse, cudaStream_t stream);
+                         float *out_lse, float *mass_partials, cudaStream_t stream);
 cudaError_t launch_cache_update(const DevGeom &g, const signed char *plan, const void *part_O,
                                 const float *part_lse, void *cache_O, float *cache_lse,
                                 unsigned char *cache_valid, int state_bf16, int num_sms,
@@ -209,7 +209,7 @@ ditango_status cuda_status(cudaError_t e) {
 
 extern "C" {
 
-int32_t ditango_version(void) { return 10100; }
+int32_t ditango_version(void) { return 10200; }
 
 const char *ditango_status_string(int32_t s) {
   switch (s) {
@@ -273,7 +273,26 @@ ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
   return cuda_status(launch_plan(dg, cache_lse, cache_valid, band_k, target, anchor ? 1 : 0,
                                  reinterpret_cast<signed char *>(plan), fresh_list, counts,
                                  score_out, workspace, static_cast<cudaStream_t>(stream), nullptr,
-                                 nullptr, nullptr, nullptr, nullptr, 0));
+                                 nullptr, nullptr, nullptr, nullptr, 0, 0));
+}
+
+ditango_status ditango_plan_from_mass(const ditango_geom *g, const float *mass_partials,
+                                     size_t mass_bytes, const uint8_t *cache_valid,
+                                     int32_t band_k, double budget, int8_t *plan,
+                                     int32_t *fresh_list, int32_t *counts, float *score_out,
+                                     ditango_stream stream) {
+  DevGeom dg;
+  ditango_status st = make_geom(g, &dg);
+  if (st != DITANGO_OK) return st;
+  if (!plan || !fresh_list || !counts || !mass_partials) return DITANGO_ERR_INVALID;
+  if (band_k < 0 || !(budget >= 0.0 && budget <= 1.0)) return DITANGO_ERR_INVALID;
+  if (mass_bytes < plan_workspace_bytes(dg)) return DITANGO_ERR_INVALID;
+  const int target = plan_target(&dg, band_k, budget);
+  return cuda_status(launch_plan(dg, nullptr, cache_valid, band_k, target, 0,
+                                 reinterpret_cast<signed char *>(plan), fresh_list, counts,
+                                 score_out, const_cast<float *>(mass_partials),
+                                 static_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr,
+                                 nullptr, nullptr, 0, 1));
 }
 
 ditango_status ditango_plan_error(const ditango_geom *g, const float *cache_lse,
@@ -299,7 +318,7 @@ ditango_status ditango_plan_error(const ditango_geom *g, const float *cache_lse,
                                  reinterpret_cast<signed char *>(plan), fresh_list, counts,
                                  score_out, workspace, static_cast<cudaStream_t>(stream),
                                  es->drift_rows, es->w, es->age, es->delta, es->local_ok,
-                                 refresh_w ? 1 : 0));
+                                 refresh_w ? 1 : 0, 0));
 }
 
 ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q, const uint16_t *K,
@@ -346,7 +365,7 @@ ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan, const vo
                              const float *part_lse, void *cache_O, float *cache_lse,
                              uint8_t *cache_valid, int32_t writeback, int32_t state_bf16,
                              void *out, int32_t out_is_fp32, const int64_t *out_strides,
-                             float *out_lse, ditango_stream stream) {
+                             float *out_lse, float *mass_partials, ditango_stream stream) {
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
   if (st != DITANGO_OK) return st;
@@ -369,7 +388,7 @@ ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan, const vo
   return cuda_status(launch_merge(dg, reinterpret_cast<const signed char *>(plan), part_O,
                                   part_lse, cache_O, cache_lse, cache_valid,
                                   (writeback && part_O) ? 1 : 0, state_bf16 ? 1 : 0, out,
-                                  out_is_fp32 ? 1 : 0, osb, osh, osn, out_lse,
+                                  out_is_fp32 ? 1 : 0, osb, osh, osn, out_lse, mass_partials,
                                   static_cast<cudaStream_t>(stream)));
 }
 
@@ -536,5 +555,5 @@ extern "C" ditango_status ditango_plan_noalloc(const ditango_geom *g, const floa
   return cuda_status(launch_plan(dg, cache_lse, cache_valid, band_k, target, anchor ? 1 : 0,
                                  reinterpret_cast<signed char *>(plan), fresh_list, counts,
                                  score_out, scratch, static_cast<cudaStream_t>(stream), nullptr,
-                                 nullptr, nullptr, nullptr, nullptr, 0));
+                                 nullptr, nullptr, nullptr, nullptr, 0, 0));
 }

@@ -8,14 +8,20 @@
 // fresh states coming from this step's partial buffer and reused ones from
 // the cache.  "Anchor Steps": the states computed fresh refresh the cache.
 //
-// The merge is HBM bound: one warp per token row, d/4 lanes each holding a
-// float4 of d; the loads of up to 8 states are issued before they are
-// consumed so that enough bytes are in flight.  The per-block table of
-// source pointers (fresh -> partial buffer at its fresh-list position,
-// reuse -> cache slot) is built once per (b*h, partition) in shared memory.
+// The merge is HBM bound.  A block takes 128 rows of one (b*h, query
+// partition).  Phase 1: one thread per row reads the row's lse of every
+// state and writes the weights to shared memory (weights.cuh, the same
+// arithmetic as the plan's mass score).  Phase 2: the block's rows of each
+// state are one contiguous run of memory, streamed as a flat array of 4-value
+// groups by all threads -- coalesced whatever d is, no idle lanes -- with
+// several states' loads of several groups in flight per thread.  Optionally
+// the block also writes its sums of the weights ("mass partials"): the
+// importance w of the next step's plan, so that the plan need not read the
+// cache again.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "weights.cuh"
 
 namespace ditango {
 namespace merge {
@@ -24,7 +30,6 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowsPerBlock = 128;
 constexpr int kBatch = 4;    // O vectors per row in flight per lane
-constexpr int kSmallStates = 4;  // rows of at most this many states: per-lane weights
 
 struct Src {
   const char *O;     // [Lmax][d] block of this (index, b*h): float32, or bf16 (SB)
@@ -135,32 +140,35 @@ __device__ __forceinline__ void lse_weights(float l0, float l1, float &w0, float
   L = dead ? -INFINITY : Ms + logf(S);
 }
 
-// MS > 0: every row has at most MS states (frame-tile rows hold 2 to 4;
-// measured on B200, rows of 8 states merge faster on the general path).
-// Then each lane loads all of a row's lse (one broadcast load each) and
-// computes the row's weights itself: no shuffles, and the weights overwrite
-// the loaded lse in place.  MS = 0: any number of states (up to 64), weights
-// by warp reductions over one state per lane.
-template <int D, bool SB, int MS>
-__global__ void __launch_bounds__(kThreads, SB ? 3 : 4)
+// Merge of one block of rows (see the file comment).  Dynamic shared memory:
+// the weights, [states][kWRows] floats.
+template <int D, bool SB>
+__global__ void __launch_bounds__(kThreads, 2)
 merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__restrict__ part_O,
              const float *__restrict__ part_lse, char *cache_O, float *cache_lse,
              unsigned char *cache_valid, int writeback, void *out, int out_is_fp32, long long osb,
-             long long osh, long long osn, float *__restrict__ out_lse) {
-  constexpr int G4 = D / 4;  // lanes carrying one row
+             long long osh, long long osn, float *__restrict__ out_lse, float *__restrict__ mass) {
+  constexpr int Q4 = D / 4;                 // 4-value groups per row
   constexpr int ES = SB ? 2 : 4;            // bytes per stored O element
   constexpr size_t ROWB = (size_t)D * ES;   // bytes per state row
+  constexpr int U = SB ? 8 : 4;             // groups per thread per pass
+  constexpr int SBATCH = 4;                 // states per batch of loads
+  using weights::kWRows;
   const int i = blockIdx.y;
   const int bh = blockIdx.z;
   const int Li = g.part_off[i + 1] - g.part_off[i];
-  const int r0 = blockIdx.x * kRowsPerBlock;
+  const int r0 = blockIdx.x * kWRows;
   if (r0 >= Li) return;
+  const int nrows = (Li - r0 < kWRows) ? Li - r0 : kWRows;
   const int G = g.G;
-  __shared__ Src src[kMaxP];
-  __shared__ int s_nact, s_fresh_before;
+  extern __shared__ float sh[];             // weights [n][kWRows]
+  __shared__ const char *s_O[kMaxP];        // state rows of this block
+  __shared__ const float *s_lse[kMaxP];
+  __shared__ char *s_wbO[kMaxP];            // write-back targets (fresh states) or null
+  __shared__ float *s_wblse[kMaxP];
+  __shared__ signed char s_state_of[kMaxP]; // column -> state index, -1: none
+  __shared__ int s_n;
   __shared__ int warp_cnt[kWarps];
-  __shared__ signed char s_plan[kMaxP];
-  if (threadIdx.x < G) s_plan[threadIdx.x] = plan[i * G + threadIdx.x];
 
   // fresh units before row i (row-major), for fresh-list positions
   int cnt = 0;
@@ -170,196 +178,116 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
   if ((threadIdx.x & 31) == 0) warp_cnt[threadIdx.x >> 5] = cnt;
   __syncthreads();
   if (threadIdx.x == 0) {
-    int fb = 0;
-    for (int w = 0; w < kWarps; ++w) fb += warp_cnt[w];
-    s_fresh_before = fb;
+    int fpos = 0;
+    for (int w = 0; w < kWarps; ++w) fpos += warp_cnt[w];
     const size_t blk = (size_t)g.BH * g.Lmax;
+    const size_t row0 = (size_t)bh * g.Lmax + r0;   // this block's first row in a state block
     int a = 0;
-    const int slot0 = g.row_start[i];
-    int fpos = fb;
     for (int c = 0; c < G; ++c) {
+      s_state_of[c] = -1;
       if (!((g.row_mask[i] >> c) & 1ull)) continue;
-      const int code = s_plan[c];
-      const int slot = slot0 + __popcll(g.row_mask[i] & ((c == 0) ? 0ull : (~0ull >> (64 - c))));
-      Src s;
-      s.wbO = nullptr;
-      s.wblse = nullptr;
-      if (code == DITANGO_PLAN_FRESH) {
-        if (part_O != nullptr) {
-          s.O = part_O + ((size_t)fpos * blk + (size_t)bh * g.Lmax) * ROWB;
-          s.lse = part_lse + (size_t)fpos * blk + (size_t)bh * g.Lmax;
-          if (writeback) {
-            s.wbO = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * ROWB;
-            s.wblse = cache_lse + (size_t)slot * blk + (size_t)bh * g.Lmax;
-            if (cache_valid && bh == 0 && blockIdx.x == 0) cache_valid[slot] = 1;
-          }
-        } else {
-          s.O = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * ROWB;
-          s.lse = cache_lse + (size_t)slot * blk + (size_t)bh * g.Lmax;
+      const int code = plan[i * G + c];
+      const int slot = slot_of(g, i, c);
+      char *wbO = nullptr;
+      float *wblse = nullptr;
+      const char *O;
+      const float *lse;
+      if (code == DITANGO_PLAN_FRESH && part_O != nullptr) {
+        O = part_O + ((size_t)fpos * blk + row0) * ROWB;
+        lse = part_lse + (size_t)fpos * blk + row0;
+        if (writeback) {
+          wbO = cache_O + ((size_t)slot * blk + row0) * ROWB;
+          wblse = cache_lse + (size_t)slot * blk + row0;
+          if (cache_valid && bh == 0 && blockIdx.x == 0) cache_valid[slot] = 1;
         }
-        ++fpos;
-      } else if (code == DITANGO_PLAN_REUSE) {
-        s.O = cache_O + ((size_t)slot * blk + (size_t)bh * g.Lmax) * ROWB;
-        s.lse = cache_lse + (size_t)slot * blk + (size_t)bh * g.Lmax;
+      } else if (code == DITANGO_PLAN_FRESH || code == DITANGO_PLAN_REUSE) {
+        O = cache_O + ((size_t)slot * blk + row0) * ROWB;
+        lse = cache_lse + (size_t)slot * blk + row0;
       } else {
         continue;  // active unit the plan skipped: contributes nothing
       }
-      src[a++] = s;
+      if (code == DITANGO_PLAN_FRESH) ++fpos;
+      s_O[a] = O;
+      s_lse[a] = lse;
+      s_wbO[a] = wbO;
+      s_wblse[a] = wblse;
+      s_state_of[c] = (signed char)a;
+      ++a;
     }
-    s_nact = a;
+    s_n = a;
   }
   __syncthreads();
-  const int nact = s_nact;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = s_n;
   const int b = bh / g.H, h = bh - (bh / g.H) * g.H;
-  const int rend = (r0 + kRowsPerBlock < Li) ? r0 + kRowsPerBlock : Li;
+  const int tok0 = g.part_off[i] + r0;
 
-  // R rows per warp iteration (2 for fp32 states, 4 for bf16 states, so both
-  // keep the same bytes in flight); every load of a row -- its states' lse
-  // and the first kBatch O vectors -- is issued before any of it is used.
-  constexpr int R = SB ? 4 : 2;
-  if constexpr (MS > 0) {
-    constexpr int RS = 2;   // rows per warp iteration (the weights live in registers)
-    const bool act = lane < G4;
-    for (int r = r0 + RS * warp; r < rend; r += RS * kWarps) {
-      constexpr int R = RS;
-      float wt[R][MS];   // the states' lse, then their weights
-#pragma unroll
-      for (int q = 0; q < R; ++q)
-#pragma unroll
-        for (int a = 0; a < MS; ++a)
-          wt[q][a] = (a < nact && (r + q) < rend) ? __ldg(src[a].lse + r + q) : -INFINITY;
-      typename Raw4<SB>::T v[R][kBatch];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u)
-#pragma unroll
-        for (int q = 0; q < R; ++q) {
-          v[q][u] = zero_raw4<SB>();
-          if (act && u < nact && (r + q) < rend)
-            v[q][u] = load_raw4<SB>(src[u].O + (size_t)(r + q) * ROWB + lane * 4 * ES);
-        }
-      float L[R];
-#pragma unroll
-      for (int q = 0; q < R; ++q) {
-        // write back the lse of fresh states (lane a for state a)
-#pragma unroll
-        for (int a = 0; a < MS; ++a)
-          if (lane == a && a < nact && (r + q) < rend && src[a].wblse) src[a].wblse[r + q] = wt[q][a];
-        float M = wt[q][0];
-#pragma unroll
-        for (int a = 1; a < MS; ++a) M = fmaxf(M, wt[q][a]);
-        const bool dead = !(M > -INFINITY);
-        const float Ms = dead ? 0.f : M;
-        float S = 0.f;
-#pragma unroll
-        for (int a = 0; a < MS; ++a) {
-          wt[q][a] = expf(wt[q][a] - Ms);   // exp(-inf) = 0 for absent states
-          S += wt[q][a];
-        }
-        const float invS = dead ? 0.f : 1.f / S;
-#pragma unroll
-        for (int a = 0; a < MS; ++a) wt[q][a] *= invS;
-        L[q] = dead ? -INFINITY : Ms + logf(S);
-      }
-      float4 acc[R];
-#pragma unroll
-      for (int q = 0; q < R; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int a0 = 0; a0 < MS; a0 += kBatch) {
-        if (a0 >= nact) break;
-        if (a0 > 0) {
-#pragma unroll
-          for (int u = 0; u < kBatch; ++u)
-#pragma unroll
-            for (int q = 0; q < R; ++q)
-              if (act && a0 + u < nact && (r + q) < rend)
-                v[q][u] = load_raw4<SB>(src[a0 + u].O + (size_t)(r + q) * ROWB + lane * 4 * ES);
-        }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-          const int a = a0 + u;
-          if (a >= nact) break;
-#pragma unroll
-          for (int q = 0; q < R; ++q) {
-            fma4(acc[q], wt[q][a], widen4<SB>(v[q][u]));
-            if (act && src[a].wbO && (r + q) < rend)
-              store_raw4<SB>(src[a].wbO + (size_t)(r + q) * ROWB + lane * 4 * ES, v[q][u]);
-          }
-        }
-      }
-      const int n = g.part_off[i] + r;
-      const size_t obase = (size_t)b * osb + (size_t)h * osh + lane * 4;
-#pragma unroll
-      for (int q = 0; q < R; ++q) {
-        if ((r + q) >= rend) continue;
-        if (act) store_out(out, out_is_fp32, obase + (size_t)(n + q) * osn, acc[q]);
-        if (out_lse && lane == 0) out_lse[((size_t)b * g.H + h) * g.N + n + q] = L[q];
-      }
-    }
-  } else {
-  for (int r = r0 + R * warp; r < rend; r += R * kWarps) {
-    float l0[R], l1[R];
-#pragma unroll
-    for (int q = 0; q < R; ++q) {
-      const bool ok = (r + q) < rend;
-      l0[q] = (ok && lane < nact) ? __ldg(src[lane].lse + r + q) : -INFINITY;
-      l1[q] = (ok && lane + 32 < nact) ? __ldg(src[lane + 32].lse + r + q) : -INFINITY;
-    }
-    const bool act = lane < G4;
-    typename Raw4<SB>::T v[R][kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u)
-#pragma unroll
-      for (int q = 0; q < R; ++q) {
-        v[q][u] = zero_raw4<SB>();
-        if (act && u < nact && (r + q) < rend)
-          v[q][u] = load_raw4<SB>(src[u].O + (size_t)(r + q) * ROWB + lane * 4 * ES);
-      }
-    float w0[R], w1[R], L[R];
-#pragma unroll
-    for (int q = 0; q < R; ++q) lse_weights(l0[q], l1[q], w0[q], w1[q], L[q]);
-    float4 acc[R];
-#pragma unroll
-    for (int q = 0; q < R; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int a0 = 0; a0 < nact; a0 += kBatch) {
-      if (a0 > 0) {
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-#pragma unroll
-          for (int q = 0; q < R; ++q)
-            if (act && a0 + u < nact && (r + q) < rend)
-              v[q][u] = load_raw4<SB>(src[a0 + u].O + (size_t)(r + q) * ROWB + lane * 4 * ES);
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int a = a0 + u;
-#pragma unroll
-        for (int q = 0; q < R; ++q) {
-          const float wq = __shfl_sync(0xffffffffu, (a < 32) ? w0[q] : w1[q], a & 31);
-          if (a < nact) {
-            fma4(acc[q], wq, widen4<SB>(v[q][u]));
-            if (act && src[a].wbO && (r + q) < rend)
-              store_raw4<SB>(src[a].wbO + (size_t)(r + q) * ROWB + lane * 4 * ES, v[q][u]);
-          }
-        }
-      }
-    }
-    // write back the lse of fresh states
-#pragma unroll
-    for (int q = 0; q < R; ++q) {
-      if ((r + q) >= rend) continue;
-      if (lane < nact && src[lane].wblse) src[lane].wblse[r + q] = l0[q];
-      if (lane + 32 < nact && src[lane + 32].wblse) src[lane + 32].wblse[r + q] = l1[q];
-    }
-    const int n = g.part_off[i] + r;
-    const size_t obase = (size_t)b * osb + (size_t)h * osh + lane * 4;
-#pragma unroll
-    for (int q = 0; q < R; ++q) {
-      if ((r + q) >= rend) continue;
-      if (act) store_out(out, out_is_fp32, obase + (size_t)(n + q) * osn, acc[q]);
-      if (out_lse && lane == 0) out_lse[((size_t)b * g.H + h) * g.N + n + q] = L[q];
+  // ---- phase 1: weights of every row (one thread per row)
+  if (threadIdx.x < kWRows) {
+    const int t = threadIdx.x;
+    const float L = weights::row_shares(s_lse, n, t, t < nrows, sh, t);
+    if (t < nrows) {
+      if (out_lse) out_lse[(size_t)bh * g.N + tok0 + t] = L;
+      for (int a = 0; a < n; ++a)
+        if (s_wblse[a]) s_wblse[a][t] = __ldg(s_lse[a] + t);
     }
   }
+  __syncthreads();
+
+  // the block's sums of the weights: the next plan's importance w
+  if (mass != nullptr) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int c = warp; c < G; c += kWarps) {
+      const int a = s_state_of[c];
+      const float v = (a >= 0) ? weights::block_sum(sh + a * kWRows, lane) : 0.f;
+      if (lane == 0) mass[weights::partial_index(g, i, bh, blockIdx.x, c)] = v;
+    }
+  }
+
+  // ---- phase 2: stream the states' rows as one flat array of 4-value groups
+  const int n4 = nrows * Q4;
+  const size_t obase = (size_t)b * osb + (size_t)h * osh;
+  for (int f0 = threadIdx.x; f0 < n4; f0 += kThreads * U) {
+    float4 acc[U];
+    int row[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      row[u] = (f0 + u * kThreads) / Q4;
+    }
+    for (int a0 = 0; a0 < n; a0 += SBATCH) {
+      typename Raw4<SB>::T v[SBATCH][U];
+#pragma unroll
+      for (int q = 0; q < SBATCH; ++q) {
+        const char *src = (a0 + q < n) ? s_O[a0 + q] : nullptr;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int f = f0 + u * kThreads;
+          v[q][u] = zero_raw4<SB>();
+          if (src != nullptr && f < n4) v[q][u] = load_raw4<SB>(src + (size_t)f * 4 * ES);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < SBATCH; ++q) {
+        if (a0 + q >= n) break;
+        const float *wq = sh + (a0 + q) * kWRows;
+        char *wb = s_wbO[a0 + q];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int f = f0 + u * kThreads;
+          if (f < n4) {
+            fma4(acc[u], wq[row[u]], widen4<SB>(v[q][u]));
+            if (wb != nullptr) store_raw4<SB>(wb + (size_t)f * 4 * ES, v[q][u]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int f = f0 + u * kThreads;
+      if (f < n4)
+        store_out(out, out_is_fp32, obase + (size_t)(tok0 + row[u]) * osn + (f - row[u] * Q4) * 4,
+                  acc[u]);
+    }
   }
 }
 
@@ -511,39 +439,32 @@ cudaError_t launch_merge(const DevGeom &g, const signed char *plan, const void *
                          unsigned char *cache_valid, int writeback, int state_bf16, void *out,
                          int out_is_fp32,
                          long long osb, long long osh, long long osn, float *out_lse,
-                         cudaStream_t stream) {
-  dim3 grid((g.Lmax + merge::kRowsPerBlock - 1) / merge::kRowsPerBlock, g.P, g.BH);
-  int most = 0;   // most active units of any row: the states a row can merge
+                         float *mass_partials, cudaStream_t stream) {
+  dim3 grid(weights::n_row_blocks(g.Lmax), g.P, g.BH);
+  int most = 1;   // most active units of any row: the states a row can merge
   for (int i = 0; i < g.P; ++i) {
     const int c = __builtin_popcountll(g.row_mask[i]);
     most = c > most ? c : most;
   }
-  const int ms = most <= merge::kSmallStates ? merge::kSmallStates : 0;
+  const size_t smem = (size_t)most * weights::kWRows * sizeof(float);
   switch (g.d) {
-#define DITANGO_MERGE_MS(DD, SB, MS)                                                             \
-  merge::merge_kernel<DD, SB, MS><<<grid, merge::kThreads, 0, stream>>>(                         \
-      g, plan, static_cast<const char *>(part_O), part_lse, static_cast<char *>(cache_O),       \
-      cache_lse, cache_valid, writeback, out, out_is_fp32, osb, osh, osn, out_lse);
-#define DITANGO_MERGE_SB(DD, SB)                                                                 \
-  if (ms == merge::kSmallStates) {                                                               \
-    DITANGO_MERGE_MS(DD, SB, merge::kSmallStates)                                                \
-  } else {                                                                                       \
-    DITANGO_MERGE_MS(DD, SB, 0)                                                                  \
-  }
 #define DITANGO_MERGE(DD)                                                                        \
   case DD:                                                                                       \
-    if (state_bf16) {                                                                            \
-      DITANGO_MERGE_SB(DD, true)                                                                 \
-    } else {                                                                                     \
-      DITANGO_MERGE_SB(DD, false)                                                                \
-    }                                                                                            \
+    if (state_bf16)                                                                              \
+      merge::merge_kernel<DD, true><<<grid, merge::kThreads, smem, stream>>>(                    \
+          g, plan, static_cast<const char *>(part_O), part_lse, static_cast<char *>(cache_O),   \
+          cache_lse, cache_valid, writeback, out, out_is_fp32, osb, osh, osn, out_lse,           \
+          mass_partials);                                                                        \
+    else                                                                                         \
+      merge::merge_kernel<DD, false><<<grid, merge::kThreads, smem, stream>>>(                   \
+          g, plan, static_cast<const char *>(part_O), part_lse, static_cast<char *>(cache_O),   \
+          cache_lse, cache_valid, writeback, out, out_is_fp32, osb, osh, osn, out_lse,           \
+          mass_partials);                                                                        \
     return cudaGetLastError();
     DITANGO_MERGE(64)
     DITANGO_MERGE(96)
     DITANGO_MERGE(128)
 #undef DITANGO_MERGE
-#undef DITANGO_MERGE_SB
-#undef DITANGO_MERGE_MS
     default:
       return cudaErrorInvalidValue;
   }

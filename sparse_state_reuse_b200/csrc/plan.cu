@@ -4,40 +4,35 @@
 // The candidates are units (query partition i, KV group c); without KV
 // groups a unit is the pair (i, j) ("Strategia per Gruppi": decisions per
 // group of adjacent partitions).
-// Stage 1 (mass_partial_kernel): importance of each active unit from the
-// cached log-sum-exps.  For every cached row r of query partition i the
-// share of unit (i, c) in that row's softmax denominator is
-//   e_c / sum_c' e_c',  e_c = exp(lse_ic[r] - max_c' lse_ic'[r]),
-// and each block sums these shares over a fixed chunk of (b*h, r) rows with
-// a fixed-order tree (warp shuffles, then warps in index order).  Invalid
-// (never written) slots hold no mass.
-// Stage 2 (plan_select_kernel, one block): chunk sums are added in chunk
-// order in double precision and divided by the row count (w = mean share),
-// then the band, the invalid slots and the top-w units up to the budget are
-// marked fresh.  Ranking sorts 64-bit keys (~bits(w) << 32 | i*G + c) with a
-// bitonic network: larger w first, ties to the lower linear index.
+// Stage 1 (mass_kernel): importance of each active unit from the cached
+// log-sum-exps.  For every cached row r of query partition i the share of
+// unit (i, c) in that row's softmax denominator is e_c / sum_c' e_c',
+// e_c = exp(lse_ic[r] - max_c' lse_ic'[r]); each block of 128 rows of one
+// (b*h, i) sums these shares in a fixed order (weights.cuh -- the same
+// arithmetic, and the same blocks, as the merge's mass partials, so the
+// merge of the previous step can stand in for this stage).  Invalid (never
+// written) slots hold no mass.
+// Stage 2 (plan_select_kernel, one block): the block sums are added in
+// (b*h, block) order in double precision and divided by the row count
+// (w = mean share), then the band, the invalid slots and the top-w units up
+// to the budget are marked fresh.  Ranking sorts 64-bit keys
+// (~bits(w) << 32 | i*G + c) with a bitonic network: larger w first, ties to
+// the lower linear index.
 // Error mode (DiTango, "Modellazione dell'Errore", "Predizione Online"):
 // stage 1 also sums each partition's local drift rows (written by the
-// attention kernel) into the extra column G of the chunk sums; stage 2 turns
+// attention kernel) into the extra column G of the block sums; stage 2 turns
 // them into delta_i, ages every cached state (0 if the previous plan made it
 // fresh, + delta_i if it reused it) and ranks by w * (age + delta_i), with w
 // recomputed only on the step after an anchor and held otherwise.
 // Everything is deterministic; no floating-point atomics.
 #include "common.cuh"
+#include "weights.cuh"
 
 namespace ditango {
 namespace plan {
 
-constexpr int kMassThreads = 256;
-constexpr int kRowsPerThread = 4;
-constexpr int kRowsPerBlock = kMassThreads * kRowsPerThread;
 constexpr int kSelThreads = 1024;
-
-__device__ __forceinline__ float warp_sum_fixed(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
+using weights::kWRows;
 
 // Error-mode arguments of the plan (all null in the plain mode).
 struct ErrorArgs {
@@ -49,107 +44,77 @@ struct ErrorArgs {
   int refresh_w;
 };
 
-__global__ void __launch_bounds__(kMassThreads)
-mass_partial_kernel(DevGeom g, const float *__restrict__ cache_lse,
-                    const unsigned char *__restrict__ cache_valid, float *__restrict__ partial,
-                    int nchunks_max, int do_mass, const float *__restrict__ drift_rows,
-                    const unsigned char *__restrict__ local_ok) {
+// Block sums of one (row block, query partition, b*h): the shares of the
+// valid active units of each row (do_mass), and the rows' local drift
+// (drift_rows non-null).  One thread per row; dynamic shared memory holds the
+// shares [units][kWRows] and the drift [kWRows].
+__global__ void __launch_bounds__(kWRows)
+mass_kernel(DevGeom g, const float *__restrict__ cache_lse,
+            const unsigned char *__restrict__ cache_valid, float *__restrict__ partial, int do_mass,
+            const float *__restrict__ drift_rows, const unsigned char *__restrict__ local_ok) {
   const int i = blockIdx.y;
-  const int chunk = blockIdx.x;
+  const int bh = blockIdx.z;
   const int Li = g.part_off[i + 1] - g.part_off[i];
-  const long long nrows = (long long)g.BH * Li;
-  const long long row0 = (long long)chunk * kRowsPerBlock;
-  if (row0 >= nrows) return;  // uniform per block
-  const unsigned long long mask = g.row_mask[i];
-  const int nact = __popcll(mask);
-  if (nact == 0) return;
-  const int s0 = g.row_start[i];
-  const int GC = g.G + 1;       // columns of the chunk sums: G units + the drift
+  const int r0 = blockIdx.x * kWRows;
+  if (r0 >= Li) return;   // uniform per block
+  const int nrows = (Li - r0 < kWRows) ? Li - r0 : kWRows;
+  const int G = g.G;
+  extern __shared__ float sh[];
+  __shared__ const float *s_lse[kMaxP];
+  __shared__ signed char s_state_of[kMaxP];
+  __shared__ int s_n;
   const size_t slot_stride = (size_t)g.BH * g.Lmax;
-
-  // per-thread rows: row0 + threadIdx.x + t * kMassThreads
-  long long roff[kRowsPerThread];
-  bool rok[kRowsPerThread];
-  float rmax[kRowsPerThread], rinv[kRowsPerThread];
-#pragma unroll
-  for (int t = 0; t < kRowsPerThread; ++t) {
-    long long q = row0 + threadIdx.x + (long long)t * kMassThreads;
-    rok[t] = q < nrows;
-    long long bh = rok[t] ? q / Li : 0;
-    long long r = rok[t] ? q - bh * Li : 0;
-    roff[t] = bh * g.Lmax + r;
-    rmax[t] = -INFINITY;
-    rinv[t] = 0.f;
+  if (threadIdx.x == 0) {
+    int a = 0;
+    for (int c = 0; c < G; ++c) {
+      s_state_of[c] = -1;
+      if (!do_mass || !((g.row_mask[i] >> c) & 1ull)) continue;
+      const int slot = slot_of(g, i, c);
+      if (cache_valid != nullptr && cache_valid[slot] == 0) continue;   // no state, no mass
+      s_lse[a] = cache_lse + (size_t)slot * slot_stride + (size_t)bh * g.Lmax + r0;
+      s_state_of[c] = (signed char)a;
+      ++a;
+    }
+    s_n = a;
   }
-  // pass 1: per-row maximum and denominator over the valid active slots
-  const int nact_m = do_mass ? nact : 0;
-  for (int a = 0; a < nact_m; ++a) {
-    const bool valid = cache_valid == nullptr || cache_valid[s0 + a] != 0;
-    if (!valid) continue;
-    const float *src = cache_lse + (size_t)(s0 + a) * slot_stride;
-#pragma unroll
-    for (int t = 0; t < kRowsPerThread; ++t)
-      if (rok[t]) rmax[t] = fmaxf(rmax[t], __ldg(src + roff[t]));
-  }
-  for (int a = 0; a < nact_m; ++a) {
-    const bool valid = cache_valid == nullptr || cache_valid[s0 + a] != 0;
-    if (!valid) continue;
-    const float *src = cache_lse + (size_t)(s0 + a) * slot_stride;
-#pragma unroll
-    for (int t = 0; t < kRowsPerThread; ++t)
-      if (rok[t] && rmax[t] > -INFINITY) rinv[t] += expf(__ldg(src + roff[t]) - rmax[t]);
-  }
-#pragma unroll
-  for (int t = 0; t < kRowsPerThread; ++t) rinv[t] = (rinv[t] > 0.f) ? 1.f / rinv[t] : 0.f;
-
-  // pass 2: per active unit, the block's sum of shares
-  __shared__ float warp_part[kMassThreads / 32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  const int n = s_n;
+  const int t = threadIdx.x;
+  float *drift_sh = sh + (size_t)n * kWRows;
+  weights::row_shares(s_lse, n, t, t < nrows, sh, t);
   if (drift_rows != nullptr) {
-    // the block's sum of the local drift rows of partition i
-    float v = 0.f;
-    if (local_ok == nullptr || local_ok[i]) {
-      const float *src = drift_rows + (size_t)i * g.BH * g.Lmax;
-#pragma unroll
-      for (int t = 0; t < kRowsPerThread; ++t)
-        if (rok[t]) v += __ldg(src + roff[t]);
-    }
-    v = warp_sum_fixed(v);
-    if (lane == 0) warp_part[warp] = v;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float s = 0.f;
-      for (int w = 0; w < kMassThreads / 32; ++w) s += warp_part[w];
-      partial[((size_t)i * nchunks_max + chunk) * GC + g.G] = s;
-    }
-    __syncthreads();
+    const bool use = (local_ok == nullptr || local_ok[i]) && t < nrows;
+    drift_sh[t] = use ? __ldg(drift_rows + ((size_t)i * g.BH + bh) * g.Lmax + r0 + t) : 0.f;
   }
-  unsigned long long m = mask;
-  for (int a = 0; a < nact_m; ++a) {
-    const int j = __ffsll((long long)m) - 1;
-    m &= m - 1;
-    const bool valid = cache_valid == nullptr || cache_valid[s0 + a] != 0;
-    float v = 0.f;
-    if (valid) {
-      const float *src = cache_lse + (size_t)(s0 + a) * slot_stride;
-#pragma unroll
-      for (int t = 0; t < kRowsPerThread; ++t)
-        if (rok[t] && rmax[t] > -INFINITY) v += expf(__ldg(src + roff[t]) - rmax[t]) * rinv[t];
+  __syncthreads();
+  const int warp = t >> 5, lane = t & 31;
+  for (int c = warp; c <= G; c += kWRows / 32) {
+    float v;
+    if (c < G) {
+      if (!((g.row_mask[i] >> c) & 1ull)) continue;
+      const int a = s_state_of[c];
+      v = (a >= 0) ? weights::block_sum(sh + a * kWRows, lane) : 0.f;
+    } else {
+      if (drift_rows == nullptr) continue;
+      v = weights::block_sum(drift_sh, lane);
     }
-    v = warp_sum_fixed(v);
-    if (lane == 0) warp_part[warp] = v;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float s = 0.f;
-      for (int w = 0; w < kMassThreads / 32; ++w) s += warp_part[w];
-      partial[((size_t)i * nchunks_max + chunk) * GC + j] = s;
-    }
-    __syncthreads();
+    if (lane == 0) partial[weights::partial_index(g, i, bh, blockIdx.x, c)] = v;
   }
 }
 
+// Sum of a unit's (or the drift column's) block sums over every (b*h, row
+// block) of query partition i, in that order, in double precision.
+__device__ __forceinline__ double sum_blocks(const DevGeom &g, const float *partial, int i, int col) {
+  const int Li = g.part_off[i + 1] - g.part_off[i];
+  const int nrb_i = weights::n_row_blocks(Li);
+  double acc = 0.0;
+  for (int bh = 0; bh < g.BH; ++bh)
+    for (int rb = 0; rb < nrb_i; ++rb) acc += (double)partial[weights::partial_index(g, i, bh, rb, col)];
+  return acc;
+}
+
 __global__ void __launch_bounds__(kSelThreads)
-plan_select_kernel(DevGeom g, const float *__restrict__ partial, int nchunks_max,
+plan_select_kernel(DevGeom g, const float *__restrict__ partial,
                    const unsigned char *__restrict__ cache_valid, int band_k, int target,
                    int anchor, signed char *__restrict__ plan_out, int *__restrict__ fresh_list,
                    int *__restrict__ counts, float *__restrict__ score_out, ErrorArgs ea) {
@@ -159,7 +124,6 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial, int nchunks_max
   __shared__ int n_forced;
   __shared__ float s_delta[kMaxP];
   const int G = g.G;
-  const int GC = G + 1;
   const int PP = g.P * G;
   const bool err = ea.age != nullptr;
   int n = 1;
@@ -171,10 +135,7 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial, int nchunks_max
     float d = 0.f;
     if (ea.local_ok[i]) {
       const int Li = g.part_off[i + 1] - g.part_off[i];
-      const int nch = (int)(((long long)g.BH * Li + kRowsPerBlock - 1) / kRowsPerBlock);
-      double acc = 0.0;
-      for (int ch = 0; ch < nch; ++ch) acc += (double)partial[((size_t)i * nchunks_max + ch) * GC + G];
-      d = (float)(acc / ((double)g.BH * Li));
+      d = (float)(sum_blocks(g, partial, i, G) / ((double)g.BH * Li));
     }
     s_delta[i] = d;
     ea.delta[i] = d;
@@ -195,11 +156,7 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial, int nchunks_max
         if (!anchor) {
           if (!err || ea.refresh_w) {
             const int Li = g.part_off[i + 1] - g.part_off[i];
-            const int nch = (int)(((long long)g.BH * Li + kRowsPerBlock - 1) / kRowsPerBlock);
-            double acc = 0.0;
-            for (int ch = 0; ch < nch; ++ch)
-              acc += (double)partial[((size_t)i * nchunks_max + ch) * GC + c];
-            w = (float)(acc / ((double)g.BH * Li));
+            w = (float)(sum_blocks(g, partial, i, c) / ((double)g.BH * Li));
             if (err) ea.w[p] = w;
           } else {
             w = ea.w[p];
@@ -297,33 +254,35 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial, int nchunks_max
 }  // namespace plan
 
 size_t plan_workspace_bytes(const DevGeom &g) {
-  const int nchunks_max =
-      (int)(((long long)g.BH * g.Lmax + plan::kRowsPerBlock - 1) / plan::kRowsPerBlock);
-  return (size_t)g.P * nchunks_max * (g.G + 1) * sizeof(float);
+  return (size_t)g.P * g.BH * weights::n_row_blocks(g.Lmax) * (g.G + 1) * sizeof(float);
 }
 
+// mass_source: the block sums are already in `workspace` (written by the
+// merge of the previous step), so stage 1 is skipped.
 cudaError_t launch_plan(const DevGeom &g, const float *cache_lse, const unsigned char *cache_valid,
                         int band_k, int target, int anchor, signed char *plan_out, int *fresh_list,
                         int *counts, float *score_out, void *workspace, cudaStream_t stream,
                         const float *drift_rows, float *w_hold, float *age, float *delta,
-                        unsigned char *local_ok, int refresh_w) {
-  const int nchunks_max =
-      (int)(((long long)g.BH * g.Lmax + plan::kRowsPerBlock - 1) / plan::kRowsPerBlock);
+                        unsigned char *local_ok, int refresh_w, int mass_given) {
   float *partial = static_cast<float *>(workspace);
   plan::ErrorArgs ea{drift_rows, w_hold, age, delta, local_ok, refresh_w};
   const bool err = age != nullptr;
   const int do_mass = err ? refresh_w : 1;
-  if (!anchor && (do_mass || err)) {
-    dim3 grid(nchunks_max, g.P);
-    plan::mass_partial_kernel<<<grid, plan::kMassThreads, 0, stream>>>(
-        g, cache_lse, cache_valid, partial, nchunks_max, do_mass, err ? drift_rows : nullptr,
-        local_ok);
+  if (!anchor && !mass_given && (do_mass || err)) {
+    int most = 0;
+    for (int i = 0; i < g.P; ++i) {
+      const int c = __builtin_popcountll(g.row_mask[i]);
+      most = c > most ? c : most;
+    }
+    const size_t smem = ((size_t)(do_mass ? most : 0) + 1) * weights::kWRows * sizeof(float);
+    dim3 grid(weights::n_row_blocks(g.Lmax), g.P, g.BH);
+    plan::mass_kernel<<<grid, weights::kWRows, smem, stream>>>(
+        g, cache_lse, cache_valid, partial, do_mass, err ? drift_rows : nullptr, local_ok);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   plan::plan_select_kernel<<<1, plan::kSelThreads, 0, stream>>>(
-      g, partial, nchunks_max, cache_valid, band_k, target, anchor, plan_out, fresh_list, counts,
-      score_out, ea);
+      g, partial, cache_valid, band_k, target, anchor, plan_out, fresh_list, counts, score_out, ea);
   return cudaGetLastError();
 }
 

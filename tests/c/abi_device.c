@@ -94,7 +94,7 @@ int main(int argc, char **argv) {
   /* an anchor step: every pair fresh, states written into the cache slots */
   DK(ditango_plan(&g, NULL, valid, 0, 1.0, 1, plan, fresh, counts, NULL, NULL, 0, st));
   DK(ditango_attn_partial(&g, q, k, v, fresh, counts, 0.0f, sO, slse, 1, 0, valid, NULL, status, st));
-  DK(ditango_merge(&g, plan, NULL, NULL, sO, slse, valid, 0, 0, out, 1, NULL, olse, st));
+  DK(ditango_merge(&g, plan, NULL, NULL, sO, slse, valid, 0, 0, out, 1, NULL, olse, NULL, st));
   CK(cudaStreamSynchronize(st));
   int32_t hstatus = -1;
   CK(cudaMemcpy(&hstatus, status, 4, cudaMemcpyDeviceToHost));

@@ -76,10 +76,21 @@ int main(void) {
   /* launching calls validate their arguments first (no GPU needed to fail) */
   CHECK(ditango_plan(&geo, NULL, NULL, 1, 0.5, 0, NULL, NULL, NULL, NULL, NULL, 0, NULL) ==
             DITANGO_ERR_INVALID, "plan without buffers");
-  CHECK(ditango_merge(&geo, NULL, NULL, NULL, NULL, NULL, NULL, 0, 0, NULL, 1, NULL, NULL, NULL) ==
+  CHECK(ditango_merge(&geo, NULL, NULL, NULL, NULL, NULL, NULL, 0, 0, NULL, 1, NULL, NULL, NULL, NULL) ==
             DITANGO_ERR_INVALID, "merge without buffers");
   CHECK(ditango_plan_error(&geo, NULL, NULL, 1, 0.5, 1, 0, NULL, NULL, NULL, NULL, NULL, NULL, 0,
                            NULL) == DITANGO_ERR_INVALID, "error plan without its state");
+  {
+    /* a plan from mass partials needs the partials, of the plan workspace's size */
+    void *fake = (void *)(uintptr_t)4096;   /* never dereferenced: refused first */
+    CHECK(ditango_plan_from_mass(&geo, NULL, 0, NULL, 1, 0.5, (int8_t *)fake, (int32_t *)fake,
+                                 (int32_t *)fake, NULL, NULL) == DITANGO_ERR_INVALID,
+          "plan from mass without partials");
+    CHECK(ditango_plan_from_mass(&geo, (const float *)fake, ditango_plan_workspace_size(&geo) - 4,
+                                 NULL, 1, 0.5, (int8_t *)fake, (int32_t *)fake, (int32_t *)fake,
+                                 NULL, NULL) == DITANGO_ERR_INVALID,
+          "plan from mass partials that are too small");
+  }
   {
     /* composing into groups that are not a coarsening of the fine ones */
     ditango_geom fine = geo, coarse = geo;

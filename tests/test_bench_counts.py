@@ -50,9 +50,13 @@ def test_published_flop_figures_of_the_workloads():
 def test_merge_bytes(w, per_row_states, fresh, sob):
     plan = plan_of(w, fresh)
     A = plan != 0
-    got = bench.merge_bytes(w, A, plan == 1, state_o_bytes=sob)
+    got = bench.merge_bytes(w, A, plan == 1, state_o_bytes=sob, mass_partials=False)
     states = int(A.sum()) if per_row_states is None else per_row_states * w.P
     want = states * w.Lp * w.BH * (w.d * sob + 4) + w.BH * w.N * (w.d * 2 + 4)
     assert got == want
     if w is configs.FRAME_TILE:
         assert got / 1e9 == pytest.approx(1.074, abs=1e-3)   # 28 states of 3600 rows, 24 heads
+    # the mass partials: one float per KV column per block of 128 rows of each
+    # (b*h, partition): ceil(Lp / 128) blocks
+    with_mass = bench.merge_bytes(w, A, plan == 1, state_o_bytes=sob)
+    assert with_mass - got == w.P * -(-w.Lp // 128) * w.BH * A.shape[1] * 4

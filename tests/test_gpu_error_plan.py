@@ -98,17 +98,19 @@ def test_schedule_matches_oracle(gs, frames, sb):
                 assert (own == plan_g).all(), (s, own, plan_g)
             d_g = ep.delta.cpu().numpy()
             worst["delta"] = max(worst["delta"], rel(d_g, sch.delta, 1e-3))
-            np.testing.assert_allclose(d_g, sch.delta, rtol=5e-3, atol=1e-5, err_msg=f"delta step {s}")
+            # delta and the ages are means of |lse differences| between steps
+            # (~1e-2 each) of fp32 lse whose error is ~1e-6: 1e-4 relative
+            np.testing.assert_allclose(d_g, sch.delta, rtol=1e-4, atol=1e-7, err_msg=f"delta step {s}")
             if s > 1:
                 assert (d_g > 0).all()
             w_g = ep.w.cpu().numpy().reshape(Au.shape)
             worst["w"] = max(worst["w"], rel(w_g[Au], sch.w[Au], 1e-3))
-            np.testing.assert_allclose(w_g, sch.w, rtol=1e-4, atol=1e-7, err_msg=f"w step {s}")
+            np.testing.assert_allclose(w_g, sch.w, rtol=1e-5, atol=1e-8, err_msg=f"w step {s}")
             a_g = ep.age.cpu().numpy()[:len(sch.age)]
             worst["age"] = max(worst["age"], rel(a_g, sch.age, 1e-3))
-            np.testing.assert_allclose(a_g, sch.age, rtol=5e-3, atol=1e-5, err_msg=f"age step {s}")
+            np.testing.assert_allclose(a_g, sch.age, rtol=1e-4, atol=1e-7, err_msg=f"age step {s}")
             worst["score"] = max(worst["score"], rel(score_g[Au], score_o[Au], 1e-4))
-            np.testing.assert_allclose(score_g, score_o, rtol=5e-3, atol=1e-6, err_msg=f"score step {s}")
+            np.testing.assert_allclose(score_g, score_o, rtol=1e-4, atol=1e-9, err_msg=f"score step {s}")
         G.assert_close(out.cpu().numpy()[0], O_o, f"out step {s}")
         G.assert_close(out_lse.cpu().numpy()[0], l_o, f"lse step {s}")
     print(f"oracle's own plan equal to the GPU's on every non-anchor step but for ties at the cut: "
