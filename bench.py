@@ -209,11 +209,15 @@ def run_ours(args, w, rank, world, local_rank):
     out_lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
     kw = dict(band_k=w.band_k, budget=w.budget, anchor=w.anchor)
 
-    # one step to learn the plan (the fresh set is the same every step here)
+    # one step to learn the plan (the fresh count, and so the work, is the
+    # same every step here); its output rows are kept for the error check
     with torch.cuda.stream(stream):
         pa.step(Q, K, V, out, out_lse, stream=stream, **kw)
     stream.synchronize()
     plan = pa.plan.cpu().numpy().reshape(w.P, pa.G)
+    check_rows = sample_check_rows(w)
+    first_out = {(b, h, i): out[b, h].index_select(0, torch.as_tensor(rows, device=dev)).float().cpu().numpy()
+                 for (b, h, i, rows) in check_rows}
     A = plan != 0
     fresh = plan == 1
     flops = effective_flops(w, fresh_pairs_of_units(w, plan, pair_mask(w)))
@@ -376,7 +380,9 @@ def run_ours(args, w, rank, world, local_rank):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
+        "plan_sha16": hashlib.sha256(plan.astype(np.int8).tobytes()).hexdigest()[:16],
     }
+    res["_check"] = (plan, first_out, check_rows)
     if compose is not None:
         res["compose"] = compose
     if args.schedule > 0:
@@ -486,6 +492,7 @@ def measure_compose(w, pa, Q, K, V, dev, stream, args, peaks):
                                  pa.state_O, pa.state_lse, pa.valid, args.state_bf16, stream)
     b.record(stream)
     stream.synchronize()
+    pa.mass_from_merge = False      # its cache was rewritten by the composition
     ms = a.elapsed_time(b) / reps
     gbs = nbytes / (ms * 1e-3) / 1e9
     out = {"from_slots": int(fine.n_slots), "to_slots": int(pa.n_slots),
@@ -502,6 +509,49 @@ def measure_compose(w, pa, Q, K, V, dev, stream, args, peaks):
 
 
 # ------------------------------------------------------------------ CPU oracle
+def sample_check_rows(w, n_rows=32):
+    """(b, h, partition, token rows) whose output the benchmark checks against
+    the oracle: the first and last rows of the first and last partitions of
+    the first and last (b, h)."""
+    po = w.part_off()
+    out = []
+    for bh in sorted({0, w.BH - 1}):
+        b, h = divmod(bh, w.H)
+        for i in sorted({0, w.P - 1}):
+            lo, hi = po[i], po[i + 1]
+            rows = np.unique(np.concatenate([np.arange(lo, min(hi, lo + n_rows // 2)),
+                                             np.arange(max(lo, hi - n_rows // 2), hi)]))
+            out.append((b, h, i, rows))
+    return out
+
+
+def error_vs_oracle(w, check):
+    """Max and mean |GPU - oracle| of the first step's sampled output rows:
+    the oracle composes the same plan's states in fp64 (fresh states from the
+    current K/V, reused ones from the previous step's)."""
+    from oracle import groups as OG, step as OS
+    plan, first_out, rows_list = check
+    errs = []
+    for (b, h, i, rows) in rows_list:
+        q = inputs.slab_f64(w, "q", b, h)
+        k = inputs.slab_f64(w, "k", b, h)
+        v = inputs.slab_f64(w, "v", b, h)
+        kp, vp = (inputs.slab_f64(w, "k", b, h, prev=True), inputs.slab_f64(w, "v", b, h, prev=True)) \
+            if w.reuses else (k, v)
+        if w.grouped:
+            O, _ = OG.step_rows_units(q, k, v, kp, vp, plan, w.part_off(), w.group_off(), i, rows,
+                                      w.frame_off(), w.frame_mask())
+        else:
+            O, _, _ = OS.step_rows(q, k, v, kp, vp, plan, w.part_off(), i, rows, w.frame_off(),
+                                   w.frame_mask())
+        errs.append(np.abs(first_out[(b, h, i)] - O).ravel())
+    e = np.concatenate(errs)
+    return {"max_abs": float(e.max()), "mean_abs": float(e.mean()),
+            "rows": int(sum(r.size for (_, _, _, r) in rows_list)),
+            "output": "bf16", "tolerance": {"max_abs": 2e-2, "mean_abs": 2e-3}}
+
+
+
 def oracle_sample(w, rng_seed, rows_per_sample, deadline_s, n_slabs=4):
     """Time the fp64 oracle on seeded (b, h, partition, row-block) samples of
     the workload until deadline_s of CPU work; returns (flops, seconds, desc).
@@ -628,8 +678,10 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     try:
         res = run_ours(args, w, rank, world, local_rank)
+        check = res.pop("_check")
         if rank == 0:
             if world == 1:
+                res["error_vs_oracle"] = error_vs_oracle(w, check)
                 f, s, desc = oracle_sample(w, 5, 128, args.cpu_baseline_seconds)
                 res["cpu_baseline"] = {"value": round(f / s / 1e12, 6), "unit": "TFLOP/s",
                                        "cores": blas_threads(), "kind": "oracle", "sample": desc}

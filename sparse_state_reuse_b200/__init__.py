@@ -54,7 +54,10 @@ class PartitionedAttention:
     state_bf16=True, a compressed cache; lse float32 [slots, B*H, Lmax]) is
     the attention-state cache: a step writes its fresh states into their
     slots and the merge reads every active unit from it, so after a step the
-    cache holds this step's fresh states and the reused ones.  group_off
+    cache holds this step's fresh states and the reused ones.  The merge also
+    leaves the next plan's mass score in the workspace, so the next plan does
+    not read the cache again; code that writes the cache tensors directly
+    must set mass_from_merge = False.  group_off
     (partition offsets of the KV groups) makes the units (query partition,
     KV group); None keeps one group per partition.
     """

@@ -24,7 +24,11 @@ struct DevGeom {
   int n_active;       // active units = slots
   int n_band;         // band units (plan only)
   int multi_run;      // some unit's active partitions are not adjacent
+  int F;              // frames of the frame-tile mask (0: none)
+  int token_mask;     // some active pair holds token pairs the frame mask forbids
   int part_off[kMaxP + 1];
+  int frame_off[kMaxP + 1];            // frame boundaries (F > 0)
+  unsigned long long frame_allow[kMaxP]; // bit f2 of entry f: query frame f attends key frame f2
   int group_off[kMaxP + 1];            // first partition of each KV group
   int row_start[kMaxP + 1];            // slot of the first active unit of row i
   unsigned long long row_mask[kMaxP];  // bit c set: unit (i, c) active

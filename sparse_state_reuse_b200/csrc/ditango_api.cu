@@ -7,6 +7,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 namespace ditango {
@@ -43,6 +45,13 @@ using namespace ditango;
 
 namespace {
 
+// An NVTX range over one entry point (shown by profilers; without one
+// attached a push/pop costs a few nanoseconds).
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
 // Process-wide limit of every device wait; set from any host thread.
 std::atomic<long long> g_wait_limit_ns{1000000000LL};
 
@@ -58,18 +67,19 @@ ditango_status make_geom(const ditango_geom *in, DevGeom *out) {
   for (int p = 0; p < in->P; ++p)
     if (in->part_off[p + 1] <= in->part_off[p]) return DITANGO_ERR_INVALID;
   if (in->F < 0 || in->F > kMaxP) return in->F < 0 ? DITANGO_ERR_INVALID : DITANGO_ERR_UNSUPPORTED;
-  int part_frame[kMaxP];
+  // frames of the first and the last token of every partition
+  int f_lo[kMaxP], f_hi[kMaxP];
   if (in->F > 0) {
     if (!in->frame_off || !in->frame_mask) return DITANGO_ERR_INVALID;
     if (in->frame_off[0] != 0 || in->frame_off[in->F] != in->N) return DITANGO_ERR_INVALID;
     for (int f = 0; f < in->F; ++f)
       if (in->frame_off[f + 1] <= in->frame_off[f]) return DITANGO_ERR_INVALID;
-    // every partition inside one frame: the frame mask is then exact per pair
-    for (int p = 0; p < in->P; ++p) {
-      int f = 0;
+    for (int p = 0, f = 0; p < in->P; ++p) {
       while (in->frame_off[f + 1] <= in->part_off[p]) ++f;
-      if (in->part_off[p + 1] > in->frame_off[f + 1]) return DITANGO_ERR_UNSUPPORTED;
-      part_frame[p] = f;
+      f_lo[p] = f;
+      int e = f;
+      while (in->frame_off[e + 1] < in->part_off[p + 1]) ++e;
+      f_hi[p] = e;
     }
   }
   DevGeom g;
@@ -102,12 +112,39 @@ ditango_status make_geom(const ditango_geom *in, DevGeom *out) {
   }
   for (int c = 0; c < g.G; ++c)
     for (int j = g.group_off[c]; j < g.group_off[c + 1]; ++j) g.part_group[j] = (signed char)c;
+  // Pair (i, j) is active when some token of partition i may attend some
+  // token of partition j.  When a partition straddles frames, an active
+  // pair can also hold token pairs the mask forbids: the kernels then mask
+  // those logits one by one (token_mask).
+  g.F = in->F;
+  g.token_mask = 0;
+  if (in->F > 0) {
+    for (int f = 0; f <= in->F; ++f) g.frame_off[f] = in->frame_off[f];
+    for (int f = 0; f < in->F; ++f) {
+      unsigned long long a = 0;
+      for (int f2 = 0; f2 < in->F; ++f2)
+        if (in->frame_mask[f * in->F + f2]) a |= 1ull << f2;
+      g.frame_allow[f] = a;
+    }
+  }
   for (int i = 0; i < in->P; ++i) {
     unsigned long long m = 0;
     for (int j = 0; j < in->P; ++j) {
-      bool act = true;
-      if (in->F > 0) act = in->frame_mask[part_frame[i] * in->F + part_frame[j]] != 0;
-      if (act) m |= 1ull << j;
+      if (in->F == 0) {
+        m |= 1ull << j;
+        continue;
+      }
+      const unsigned long long kf = bit_range(f_lo[j], f_hi[j] + 1);   // key frames of j
+      bool any = false, all = true;
+      for (int f = f_lo[i]; f <= f_hi[i]; ++f) {
+        const unsigned long long hit = g.frame_allow[f] & kf;
+        any = any || hit != 0ull;
+        all = all && hit == kf;
+      }
+      if (any) {
+        m |= 1ull << j;
+        if (!all) g.token_mask = 1;
+      }
     }
     g.pair_mask[i] = m;
   }
@@ -261,6 +298,7 @@ ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
                             int32_t anchor, int8_t *plan, int32_t *fresh_list, int32_t *counts,
                             float *score_out, void *workspace, size_t workspace_bytes,
                             ditango_stream stream) {
+  NvtxRange nvtx_range("ditango_plan");
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
   if (st != DITANGO_OK) return st;
@@ -281,6 +319,7 @@ ditango_status ditango_plan_from_mass(const ditango_geom *g, const float *mass_p
                                      int32_t band_k, double budget, int8_t *plan,
                                      int32_t *fresh_list, int32_t *counts, float *score_out,
                                      ditango_stream stream) {
+  NvtxRange nvtx_range("ditango_plan_from_mass");
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
   if (st != DITANGO_OK) return st;
@@ -302,6 +341,7 @@ ditango_status ditango_plan_error(const ditango_geom *g, const float *cache_lse,
                                   int32_t *fresh_list, int32_t *counts, float *score_out,
                                   void *workspace, size_t workspace_bytes,
                                   ditango_stream stream) {
+  NvtxRange nvtx_range("ditango_plan_error");
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
   if (st != DITANGO_OK) return st;
@@ -327,6 +367,7 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q, co
                                     float *out_lse, int32_t out_by_slot, int32_t state_bf16,
                                     uint8_t *out_valid, float *drift_rows, int32_t *dev_status,
                                     ditango_stream stream) {
+  NvtxRange nvtx_range("ditango_attn_partial");
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
   if (st != DITANGO_OK) return st;
@@ -366,6 +407,7 @@ ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan, const vo
                              uint8_t *cache_valid, int32_t writeback, int32_t state_bf16,
                              void *out, int32_t out_is_fp32, const int64_t *out_strides,
                              float *out_lse, float *mass_partials, ditango_stream stream) {
+  NvtxRange nvtx_range("ditango_merge");
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
   if (st != DITANGO_OK) return st;
@@ -396,6 +438,7 @@ ditango_status ditango_cache_update(const ditango_geom *g, const int8_t *plan,
                                     const void *part_O, const float *part_lse, void *cache_O,
                                     float *cache_lse, uint8_t *cache_valid, int32_t state_bf16,
                                     ditango_stream stream) {
+  NvtxRange nvtx_range("ditango_cache_update");
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
   if (st != DITANGO_OK) return st;
@@ -411,6 +454,7 @@ ditango_status ditango_cache_compose(const ditango_geom *fine, const ditango_geo
                                      const uint8_t *fine_valid, void *coarse_O,
                                      float *coarse_lse, uint8_t *coarse_valid,
                                      int32_t state_bf16, ditango_stream stream) {
+  NvtxRange nvtx_range("ditango_cache_compose");
   DevGeom gf, gc;
   ditango_status st = make_geom(fine, &gf);
   if (st != DITANGO_OK) return st;
@@ -518,6 +562,7 @@ extern "C" ditango_status ditango_plan_noalloc(const ditango_geom *g, const floa
                                                double budget, int32_t anchor, int8_t *plan,
                                                int32_t *fresh_list, int32_t *counts,
                                                float *score_out, ditango_stream stream) {
+  NvtxRange nvtx_range("ditango_plan_noalloc");
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
   if (st != DITANGO_OK) return st;

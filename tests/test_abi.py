@@ -60,12 +60,29 @@ def test_ragged_partitions_within_frames():
     assert dt.ditango_state_rows(g) == 445
 
 
+def test_partitions_straddling_frames():
+    """Partitions cut across frame boundaries: a pair is active when any of
+    its token pairs is allowed (the kernels then mask single logits)."""
+    fo = [0, 50, 100, 150, 200]
+    fm = [[1, 0, 0, 1], [1, 1, 0, 0], [0, 1, 1, 0], [0, 0, 1, 1]]
+    po = [0, 30, 75, 140, 170, 200]
+    g = dt.Geometry(1, 2, 200, 64, po, fo, fm)
+    A = masks.pair_mask(po, fo, fm)
+    assert dt.ditango_num_active(g) == int(A.sum())
+    assert (np.array(dt.ditango_slot_table(g)) == masks.slot_table(A)).all()
+    go = [0, 2, 5]
+    g = dt.Geometry(1, 2, 200, 64, po, fo, fm, group_off=go)
+    Au = groups.unit_mask(A, go)
+    assert (np.array(dt.ditango_slot_table(g)) == masks.slot_table(Au)).all()
+
+
 @pytest.mark.parametrize("kw,status", [
     (dict(part_off=[0, 10, 10, 64]), 1),          # empty partition
     (dict(part_off=[0, 32, 63]), 1),              # does not end at N
     (dict(d=80), 2),                              # head dim without a kernel
     (dict(part_off=list(range(0, 65 * 2, 2))[:66] + [130]), 2),  # P > 64
-    (dict(frame_off=[0, 40, 64], frame_mask=[[1, 1], [1, 1]]), 2),  # partition straddles frames
+    (dict(frame_off=[0, 40, 64], frame_mask=[[1, 1], [1, 1]]), 0),  # partition straddling frames
+    (dict(frame_off=[0, 40, 63], frame_mask=[[1, 1], [1, 1]]), 1),  # frames not ending at N
     (dict(B=0), 1),
 ])
 def test_geometry_validation(kw, status):

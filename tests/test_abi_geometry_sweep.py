@@ -1,7 +1,8 @@
 """Seeded sweep of the C ABI's host-side geometry logic (no GPU needed).
 
 Random valid geometries -- ragged partitions, frames holding one or more
-partitions, arbitrary frame masks, optional KV groups -- must give the
+partitions or partitions cut across frames, arbitrary frame masks, optional
+KV groups -- must give the
 oracle's active units, slot table and state rows; random geometries with one
 rule broken must be refused with the status that rule carries (invalid
 argument, or a valid but unsupported shape)."""
@@ -23,12 +24,18 @@ def random_geometry(rng):
     if F:
         frame_len = rng.integers(8, 40, size=F)
         frame_off = [0] + np.cumsum(frame_len).astype(int).tolist()
-        # each frame split into 1..3 partitions: every partition inside one frame
-        part_off = [0]
-        for f in range(F):
-            n = int(rng.integers(1, min(3, frame_len[f]) + 1))
-            sub = random_offsets(rng, int(frame_len[f]), n)
-            part_off += [frame_off[f] + s for s in sub[1:]]
+        if rng.random() < 0.5:
+            # each frame split into 1..3 partitions: every partition inside one frame
+            part_off = [0]
+            for f in range(F):
+                n = int(rng.integers(1, min(3, frame_len[f]) + 1))
+                sub = random_offsets(rng, int(frame_len[f]), n)
+                part_off += [frame_off[f] + s for s in sub[1:]]
+        else:
+            # partitions cut anywhere: some straddle frame boundaries
+            N = frame_off[-1]
+            P = int(rng.integers(1, min(N, 12) + 1))
+            part_off = random_offsets(rng, N, P) if P > 1 else [0, N]
         mask = (rng.random((F, F)) < 0.6).astype(int)
         frames = (frame_off, mask.tolist())
     else:
@@ -91,13 +98,10 @@ def broken(rng, kw, frames, go):
     if choice == 4 and P > 2:                     # groups that do not rise
         return kw, frames, [0, 2, 1, P], INVALID
     if choice == 5 and frames and len(frames[0]) > 2:
-        # a partition that straddles a frame boundary: merge the two partitions around it
-        fo = frames[0]
-        b = fo[1]
-        if b in po and po.index(b) < P:
-            k = po.index(b)
-            kw["part_off"] = po[:k] + po[k + 1:]
-            return kw, frames, None, UNSUPPORTED
+        # frame offsets that do not rise
+        fo = list(frames[0])
+        fo[1] = fo[2]
+        return kw, (fo, frames[1]), go, INVALID
     if choice == 6:
         kw["B"] = 0
         return kw, frames, go, INVALID

@@ -47,6 +47,10 @@ def all_pairs_partial(geom, Q, K, V, n, Lmax, d, BH, state_bf16=False):
             lse.cpu().numpy())
 
 
+# frame-tile mask of 5 frames: each frame attends itself, its neighbours and frame 0
+TILE5 = [[1 if (abs(f - g) <= 1 or g == 0) else 0 for g in range(5)] for f in range(5)]
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     dt.ditango_selftest_bounded_wait(2_000_000, st)
@@ -66,6 +70,11 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     (64, [0, 100, 130, 300, 555, 1000], None, True),   # bf16 states (compressed cache)
     (96, [0, 130, 300, 555, 1000], ([0, 300, 1000], [[1, 0], [1, 1]]), True),
     (128, [0, 257, 512, 640, 1024], None, True),
+    # partitions that straddle frames: single logits masked by the frame mask
+    (96, [0, 130, 400, 555, 1000], ([0, 300, 700, 1000], [[1, 1, 0], [1, 1, 1], [1, 1, 1]]), False),
+    (128, [0, 250, 520, 1000], ([0, 200, 400, 600, 800, 1000], TILE5), False),
+    (64, [0, 250, 520, 1000], ([0, 200, 400, 600, 800, 1000], TILE5), True),
+    (64, [0, 60, 61, 190, 1000], ([0, 45, 90, 135, 180, 1000], TILE5), False),
 ])
 def test_partial_states_every_row(d, part_off, frames, sb):
     if part_off is None:
@@ -142,6 +151,51 @@ def test_tiny_reuse_step_plan_and_output(sb):
         for i in range(w.P):
             rows = np.arange(w.part_off()[i], w.part_off()[i + 1])
             Oo, lo, _ = G.oracle_rows(w, plan_o, b, h, i, rows)
+            G.assert_close(o[b, h, rows], Oo, f"out bh {bh} part {i}")
+            G.assert_close(ol[b, h, rows], lo, f"out lse bh {bh} part {i}")
+
+
+@pytest.mark.parametrize("go", [None, [0, 2, 5]], ids=["pairs", "groups"])
+def test_reuse_step_with_partitions_straddling_frames(go):
+    """A reuse step whose partitions cut across the frames of a frame-tile
+    mask (5 partitions over 6 frames): some rows attend none of a pair's keys
+    (lse -inf, weight 0 in the merge).  The plan is compared with the
+    oracle's selection on the GPU's scores and on its own fp64 scores of the
+    GPU's cache; every output row with the oracle's composition."""
+    from oracle import groups as OG
+    w = configs.scaled(configs.TINY, N=1200, P=5, H=2, d=96, F=6, frame_component=0.5,
+                       band_k=0, budget=0.5, seed=91, drift_seed=191, name="straddle")
+    po = [0, 150, 410, 700, 990, 1200]
+    fo, fm = w.frame_off(), w.frame_mask()
+    Q, K, V = G.upload(w)
+    Kp, Vp = G.upload_prev(w)
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, po, fo, fm, group_off=go)
+    build_cache(pa, Q, Kp, Vp)
+    torch.cuda.synchronize()
+    lse_cache = pa.state_lse.cpu().numpy()
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    out_lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
+    pa.step(Q, K, V, out, out_lse, band_k=w.band_k, budget=w.budget)
+    torch.cuda.synchronize()
+    assert pa.status.item() == 0
+    A = OM.pair_mask(po, fo, fm)
+    gof = go if go is not None else list(range(w.P + 1))
+    Au, band = OG.unit_mask(A, gof), OG.unit_band(A, gof, w.band_k)
+    plan = pa.plan.cpu().numpy().reshape(Au.shape)
+    score = pa.score.cpu().numpy().reshape(Au.shape)
+    sel, _ = select(score.astype(np.float64), Au, w.band_k, w.budget, band=band)
+    assert (sel == plan).all()
+    w_o = mass_scores(lse_cache, Au, po)
+    np.testing.assert_allclose(score[Au], w_o[Au], rtol=1e-5)
+    plan_o, _ = select(w_o, Au, w.band_k, w.budget, band=band)
+    assert (plan_o == plan).all()
+    o, ol = out.cpu().numpy(), out_lse.cpu().numpy()
+    for bh in range(w.BH):
+        b, h = divmod(bh, w.H)
+        q, k, v, kp, vp = G.slabs(w, b, h)
+        for i in range(w.P):
+            rows = np.arange(po[i], po[i + 1])
+            Oo, lo = OG.step_rows_units(q, k, v, kp, vp, plan, po, gof, i, rows, fo, fm)
             G.assert_close(o[b, h, rows], Oo, f"out bh {bh} part {i}")
             G.assert_close(ol[b, h, rows], lo, f"out lse bh {bh} part {i}")
 
@@ -251,6 +305,7 @@ def test_step_captured_in_a_cuda_graph_replays_bit_identically():
 
     def restore():
         pa.state_O.copy_(cache0[0]); pa.state_lse.copy_(cache0[1]); pa.valid.copy_(cache0[2])
+        pa.mass_from_merge = False      # the cache changed behind the object: plan from it
 
     restore()
     s = torch.cuda.Stream()
