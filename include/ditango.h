@@ -81,9 +81,12 @@ typedef void *ditango_stream; /* cudaStream_t */
  *   F        frames of the frame-tile mask, 0 = no mask (all pairs active);
  *            else 1 <= F <= 64, frame_off host int32 [F+1] (same rules as
  *            part_off) and frame_mask host uint8 [F*F], row = query frame,
- *            nonzero = the query frame may attend the key frame.  Every
- *            partition must lie inside one frame (else UNSUPPORTED): the mask
- *            is then exact at pair granularity.
+ *            nonzero = the query frame may attend the key frame.  The mask
+ *            applies token by token; pair (i, j) is active when some token of
+ *            partition i may attend some token of partition j.  Partitions may
+ *            straddle frames: single logits are then masked inside the pair,
+ *            and a row that may attend none of a unit's keys gets lse = -inf,
+ *            O = 0 for that unit.
  *   q/k/v_strides  element strides of the (b, h, n) dimensions of the bf16
  *            Q, K, V tensors; the d dimension is contiguous.  Strides times 2
  *            bytes must be multiples of 16 and the base pointers 16-byte
@@ -206,6 +209,13 @@ ditango_status ditango_plan_from_mass(const ditango_geom *g, const float *mass_p
  *                (DiTango, "Predizione Online").
  *   dev_status   dev int32 or NULL; set to DITANGO_ERR_TIMEOUT if a pipeline
  *                wait exceeded the limit (the kernel then stops cleanly).
+ *   work_counter dev int32 [2], 8-byte aligned, or NULL.  With it, each CTA
+ *                of the persistent kernel takes the next work item when it is
+ *                ready for one (balanced whatever the items' sizes); without
+ *                it, items are dealt in a fixed stride.  Zero it once when it
+ *                is allocated: every launch leaves it at zero again.  Launches
+ *                that may run at the same time (other streams, concurrent
+ *                graph branches) must not share one.
  */
 ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q,
                                     const uint16_t *K, const uint16_t *V,
@@ -213,7 +223,8 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q,
                                     float scale, void *out_O, float *out_lse,
                                     int32_t out_by_slot, int32_t state_bf16,
                                     uint8_t *out_valid, float *drift_rows,
-                                    int32_t *dev_status, ditango_stream stream);
+                                    int32_t *dev_status, int32_t *work_counter,
+                                    ditango_stream stream);
 
 /* Merge: the final output of every token is the log-sum-exp composition of
  * the states of its partition's active units (DiTango, "Composizione dello

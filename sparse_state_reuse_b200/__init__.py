@@ -93,6 +93,8 @@ class PartitionedAttention:
         self.ws_bytes = ditango_plan_workspace_size(self.geom)
         self.workspace = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        # the attention kernel's work counter (each launch leaves it at zero)
+        self.work_counter = torch.zeros(2, dtype=torch.int32, device=dev)
         # the workspace holds the mass partials of the last merge, and the
         # cache has not changed since: the next plan need not read the cache
         self.mass_from_merge = False
@@ -145,7 +147,8 @@ class PartitionedAttention:
         self.mass_from_merge = False
         ditango_attn_partial(self.geom, Q, K, V, self.fresh_list, self.counts, scale,
                              self.state_O, self.state_lse, 1, self.valid, self.status, stream,
-                             state_bf16=self.state_bf16, drift_rows=drift_rows)
+                             state_bf16=self.state_bf16, drift_rows=drift_rows,
+                             work_counter=self.work_counter)
 
     def merge(self, out, out_lse=None, stream=None):
         import torch

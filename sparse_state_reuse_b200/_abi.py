@@ -68,7 +68,7 @@ _SIGS = {
     "ditango_plan": (C.c_int, [_G, _P, _P, C.c_int32, C.c_double, C.c_int32, _P, _P, _P, _P, _P,
                                C.c_size_t, _P]),
     "ditango_attn_partial": (C.c_int, [_G, _P, _P, _P, _P, _P, C.c_float, _P, _P, C.c_int32,
-                                       C.c_int32, _P, _P, _P, _P]),
+                                       C.c_int32, _P, _P, _P, _P, _P]),
     "ditango_plan_error": (C.c_int, [_G, _P, _P, C.c_int32, C.c_double, C.c_int32, C.c_int32,
                                      C.POINTER(ditango_error_state), _P, _P, _P, _P, _P,
                                      C.c_size_t, _P]),
@@ -208,11 +208,11 @@ def ditango_plan(geom, cache_lse, cache_valid, band_k, budget, anchor, plan, fre
 
 def ditango_attn_partial(geom, Q, K, V, fresh_list, counts, scale, out_O, out_lse,
                          out_by_slot=0, out_valid=None, dev_status=None, stream=None,
-                         state_bf16=0, drift_rows=None):
+                         state_bf16=0, drift_rows=None, work_counter=None):
     _check("ditango_attn_partial", _lib.ditango_attn_partial(
         geom.ref, _ptr(Q), _ptr(K), _ptr(V), _ptr(fresh_list), _ptr(counts), float(scale),
         _ptr(out_O), _ptr(out_lse), int(out_by_slot), int(bool(state_bf16)), _ptr(out_valid),
-        _ptr(drift_rows), _ptr(dev_status), _stream(stream)))
+        _ptr(drift_rows), _ptr(dev_status), _ptr(work_counter), _stream(stream)))
 
 
 def error_state(w, age, delta, local_ok, drift_rows):

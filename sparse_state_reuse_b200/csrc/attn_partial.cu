@@ -27,13 +27,15 @@
 // the P V product straight from TMEM.  The two Q tiles ping-pong: while one
 // warpgroup exponentiates its S tile, the tensor pipe runs the other tile's
 // P V and next Q K^T.  One thread owns one query row, so row max and row sum
-// need no cross-thread reduction.  Each tile is exponentiated against the
-// base carried from the previous tile (or the previous unit of the same
-// rows) while its maximum is still being found, so the exponentials start as
-// soon as the first half of S is in registers; the base, and with it O, is
-// rescaled only when a row's maximum passes it by more than 2^8 (exact: O
-// and l share the base).  Work items are taken in (b*h, partition, rows)
-// order, so the CTAs running at the same time read the same K/V from L2.
+// need no cross-thread reduction.  O is rescaled only when a row's running
+// maximum grows by more than 2^8 (exact: O and l share the stale maximum).
+// Work items go from the producer warp to the other roles through a 2-slot
+// ring in shared memory; with a work counter each CTA takes the next item
+// when it is ready for it (balanced whatever the items' sizes), otherwise
+// items are taken in a fixed stride.  Items are numbered in (b*h, partition,
+// rows) order, every partition's last block of rows after all the others:
+// the CTAs running at the same time share one (b, h)'s K/V in L2, and the
+// small items fill the end of the schedule.
 #include <mutex>
 #include <set>
 #include <utility>
@@ -83,6 +85,7 @@ struct Params {
   float *drift_rows;       // [P][B*H][Lmax] local-state drift, or null
   int *dev_status;
   long long wait_limit_ns;
+  int *sched;              // [2] work counter (next item, CTAs done) or null: fixed stride
 };
 
 // A work item: up to 256 query rows of partition i for one (b, h).  The item
@@ -149,11 +152,16 @@ struct KeyCursor {
 __device__ __forceinline__ Item decode_item(const Params &p, const int *row_fresh, int it, int nqt2) {
   Item w;
   const DevGeom &g = p.g;
-  // b*h-major order: the CTAs working at the same time share one (b, h)'s
-  // K/V, which then stays in L2 for every query partition that reads it
-  const int qt2 = it % nqt2;
-  const int rest = it / nqt2;
-  w.i = rest % g.P;
+  const int n_main = g.P * g.BH * (nqt2 - 1);
+  int qt2, rest;
+  if (it < n_main) {
+    qt2 = it % (nqt2 - 1);
+    rest = it / (nqt2 - 1);
+  } else {
+    qt2 = nqt2 - 1;   // the last block of rows of every partition, after all the others
+    rest = it - n_main;
+  }
+  w.i = rest % g.P;   // b*h-major: the CTAs running together share one (b, h)'s K/V
   w.bh = rest / g.P;
   w.b = w.bh / g.H;
   w.h = w.bh - w.b * g.H;
@@ -279,8 +287,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
-constexpr float kRebaseDownLog2 = 64.0f;
-
 // Frame of a token (tokens past the end count in the last frame).
 __device__ __forceinline__ int frame_of(const DevGeom &g, int tok) {
   int lo = 0, hi = g.F - 1;
@@ -291,7 +297,7 @@ __device__ __forceinline__ int frame_of(const DevGeom &g, int tok) {
   return lo;
 }
 
-// Token-level frame mask (Efficient-vDiT's frame tiles with partitions that
+// Token-level frame mask (Efficient-vDiT's frame tiles, with partitions that
 // straddle frames): in the key tile starting at token k0 (valid keys), the
 // logits of keys whose frame this row may not attend become -inf.
 __device__ __forceinline__ void mask_frames(const DevGeom &g, int k0, int valid,
@@ -304,32 +310,6 @@ __device__ __forceinline__ void mask_frames(const DevGeom &g, int k0, int valid,
 #pragma unroll
     for (int c = 0; c < BN; ++c)
       if (c >= c0 && c < c1) sv[c] = __float_as_uint(-INFINITY);
-  }
-}
-
-// P = 2^(s * scale * log2e - base) for the columns [c0, c1) of the row
-// (multiples of 16): rounded to bf16 in pairs into the first 64 columns of
-// this tile's S (16 probabilities -> 8 TMEM columns), with the packed partial
-// row sums accumulated in lsum0/lsum1.
-template <int D>
-__device__ __forceinline__ void exp_store(const uint32_t (&sv)[BN], int c0, int c1, uint64_t sl2x2,
-                                          uint64_t negx2, uint64_t &lsum0, uint64_t &lsum1,
-                                          uint32_t tS) {
-#pragma unroll
-  for (int g8 = 0; g8 < BN / 16; ++g8) {
-    if (g8 * 16 < c0 || g8 * 16 >= c1) continue;
-    uint32_t pk[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int c = g8 * 16 + 2 * e;
-      float xa, xb;
-      unf2(fma2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, negx2), xa, xb);
-      const float a = (2 * e < emu_per16<D>()) ? exp2_poly(xa) : ex2(xa);
-      const float b = (2 * e + 1 < emu_per16<D>()) ? exp2_poly(xb) : ex2(xb);
-      if (e & 1) lsum1 = add2(lsum1, f2(a, b)); else lsum0 = add2(lsum0, f2(a, b));
-      pk[e] = pack_bf16(a, b);
-    }
-    tmem_st8(tS + g8 * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
   }
 }
 
@@ -359,6 +339,10 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   auto o_full = [&](int k) { return bar + 112 + 8 * k; };
   auto o_empty = [&](int k) { return bar + 128 + 8 * k; };
   const uint32_t drain = bar + 144;
+  // work items pass from the producer to the other roles through a 2-slot ring
+  auto item_full = [&](int s) { return bar + 152 + 8 * s; };
+  auto item_empty = [&](int s) { return bar + 168 + 8 * s; };
+  volatile int *item_slot = reinterpret_cast<volatile int *>(smem + C::OFF_BAR + 208);
 
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + 192);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_BAR + 200);
@@ -401,6 +385,10 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       mbar_init(o_empty(k), 4);
     }
     mbar_init(drain, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(item_full(s), 1);
+      mbar_init(item_empty(s), 9);   // the MMA warp and the eight softmax warps
+    }
 
     *abort_flag = 0;
     fence_barrier_init();
@@ -432,9 +420,38 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       int q_armed = -1;
       uint32_t k_armed = 0, v_armed = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const Item w = decode_item(p, row_fresh, it, nqt2);
-        if (!w.live) continue;
+      uint32_t ic = 0;                 // items published to the other roles
+      int next_static = blockIdx.x;
+      while (ok) {
+        // the next live item: from the work counter (each CTA takes the next
+        // one when it is ready for it), or in a fixed stride without one
+        int it;
+        Item w;
+        for (;;) {
+          if (p.sched != nullptr) {
+            int v = 0;
+            if (lane == 0) v = atomicAdd(p.sched, 1);
+            it = __shfl_sync(0xffffffffu, v, 0);
+          } else {
+            it = next_static;
+            next_static += gridDim.x;
+          }
+          if (it >= n_items) {
+            it = -1;
+            break;
+          }
+          w = decode_item(p, row_fresh, it, nqt2);
+          if (w.live) break;
+        }
+        // publish it (or the end, -1) to the MMA and softmax warps
+        const int is = ic & 1;
+        if (!(ok = wait_warp(item_empty(is), ((ic >> 1) & 1) ^ 1, ctl))) break;
+        if (leader) {
+          item_slot[is] = it;
+          mbar_arrive(item_full(is));
+        }
+        ++ic;
+        if (it < 0) break;
         if (!(ok = wait_warp(q_empty, (uc & 1) ^ 1, ctl))) break;
         const uint32_t qbytes = C::TILE * (w.rows1 > 0 ? 2 : 1);
         if (leader) mbar_arrive_expect_tx(q_full, qbytes);
@@ -535,9 +552,16 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int kk = 0; kk < BN / 16; ++kk)
           if (leader) mma_ts(d_tmem, a_tmem + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv, (acc || kk > 0));
       };
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      uint32_t ic = 0;
+      while (ok) {
+        const int is = ic & 1;
+        if (!(ok = wait_warp(item_full(is), (ic >> 1) & 1, ctl))) break;
+        const int it = item_slot[is];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(item_empty(is));
+        ++ic;
+        if (it < 0) break;
         const Item w = decode_item(p, row_fresh, it, nqt2);
-        if (!w.live) continue;
         const bool has1 = w.rows1 > 0;
         if (!(ok = wait_warp(q_full, uc & 1, ctl))) break;
         for (int f = w.f0; f < w.f1 && ok; ++f) {
@@ -616,6 +640,16 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       named_bar_sync(1, kThreads);
       tc_fence_after();
       tmem_dealloc(tmem, 512);
+      if (p.sched != nullptr && lane == 0) {
+        // the last CTA to finish (every producer has taken its last item by
+        // then) leaves the counter at zero for the next launch
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
+          p.sched[0] = 0;
+          p.sched[1] = 0;
+          __threadfence();
+        }
+      }
     } else {
       tc_fence_before();
       named_bar_arrive(1, kThreads);
@@ -632,124 +666,73 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const float sl2 = p.scale_log2;
     uint32_t sc = 0, ofc = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    uint32_t ic = 0;
+    while (ok) {
+      const int is = ic & 1;
+      if (!(ok = wait_warp(item_full(is), (ic >> 1) & 1, ctl))) break;
+      const int it = item_slot[is];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(item_empty(is));
+      ++ic;
+      if (it < 0) break;
       const Item w = decode_item(p, row_fresh, it, nqt2);
-      if (!w.live) continue;
       const int rows_k = (k == 0) ? w.rows0 : w.rows1;
       if (rows_k <= 0) continue;
-     float m_seed = -INFINITY;   // this row's base at the end of the previous unit
-     // key frames this row may attend (a frame mask with partitions that
-     // straddle frames masks single logits)
-     unsigned long long allow = ~0ull;
-     if constexpr (MR) {
-       if (p.g.token_mask) allow = p.g.frame_allow[frame_of(p.g, w.q0 + k * BM + r)];
-     }
+      // key frames this row may attend (partitions that straddle frames)
+      unsigned long long allow = ~0ull;
+      if constexpr (MR) {
+        if (p.g.token_mask) allow = p.g.frame_allow[frame_of(p.g, w.q0 + k * BM + r)];
+      }
      for (int f = w.f0; f < w.f1 && ok; ++f) {
       const UnitRange pr = unit_at<MR>(p, w.i, f);
       KeyCursor cur;
       if constexpr (MR) cur.start(p.g, w.i, pr.c);
-      // Base of the exponentials (log2 units).  Exponentials are taken
-      // against the base carried from the previous tile (or the previous unit
-      // of the same rows) while the tile's maximum is still being found; the
-      // base moves only when the maximum exceeds it by more than 2^8 (or, on
-      // a unit's first tile, lies more than 2^64 below it) -- then the tile is
-      // exponentiated again, rarely.  O and l always share the base, so the
-      // state is exact whichever base is used.
-      float m_used = m_seed;
+      float m_used = -INFINITY;   // running maximum used for exponentiation (log2 units)
       float l = 0.f;
       for (int t = 0; t < pr.T; ++t) {
         if constexpr (MR) {
           if (t > 0) cur.next(p.g, w.i, pr.c);
         }
-        if (!(ok = wait_warp(s_full(k), sc & 1, ctl))) break;   // warp-uniform: the votes below need every lane
+        if (!(ok = wait_bounded(s_full(k), sc & 1, ctl))) break;
         ++sc;
         tc_fence_after();
-        const int valid = MR ? cur.valid() : pr.Lk - t * BN;
+        // the whole S row of this thread: eight loads in flight, one wait
         uint32_t sv[BN];
-        uint64_t lsum0 = 0, lsum1 = 0;   // packed partial row sums (+0.0f bits)
-        const uint64_t sl2x2 = f2(sl2, sl2);
-        float mx;
-        // every lane of the warp has a finite base: exponentiate while the
-        // second half of S is still loading
-        const bool spec = !(MR && p.g.token_mask) && __all_sync(0xffffffffu, m_used > -INFINITY);
-        if (spec) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld16p(tS + c * 16, &sv[c * 16]);
-          tc_wait_ld();
+        for (int c = 0; c < BN / 16; ++c) tmem_ld16p(tS + c * 16, &sv[c * 16]);
+        tc_wait_ld();
+        const int valid = MR ? cur.valid() : pr.Lk - t * BN;
+        if (valid < BN) {
 #pragma unroll
-          for (int c = 4; c < 8; ++c) tmem_ld16p(tS + c * 16, &sv[c * 16]);
-          if (valid < BN / 2) {
+          for (int c = 0; c < BN; ++c)
+            if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
+        }
+        if constexpr (MR) {
+          if (p.g.token_mask) mask_frames(p.g, cur.row(), valid, allow, sv);
+        }
+        // row maximum: 8 independent chains of 3-input max, then a tree
+        float m8[8];
 #pragma unroll
-            for (int c = 0; c < BN / 2; ++c)
-              if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
-          }
-          const float neg = -m_used;
-          const uint64_t negx2 = f2(neg, neg);
-          float m4[4];
+        for (int q = 0; q < 8; ++q)
+          m8[q] = max3(__uint_as_float(sv[q]), __uint_as_float(sv[q + 8]), __uint_as_float(sv[q + 16]));
 #pragma unroll
-          for (int q = 0; q < 4; ++q) m4[q] = fmaxf(__uint_as_float(sv[q]), __uint_as_float(sv[q + 4]));
-#pragma unroll
-          for (int c = 8; c < BN / 2; c += 8)
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              m4[q] = max3(m4[q], __uint_as_float(sv[c + q]), __uint_as_float(sv[c + q + 4]));
-          exp_store<D>(sv, 0, BN / 2, sl2x2, negx2, lsum0, lsum1, tS);
-          tc_wait_ld();
-          if (valid < BN) {
-#pragma unroll
-            for (int c = BN / 2; c < BN; ++c)
-              if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
-          }
-#pragma unroll
-          for (int c = BN / 2; c < BN; c += 8)
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              m4[q] = max3(m4[q], __uint_as_float(sv[c + q]), __uint_as_float(sv[c + q + 4]));
-          exp_store<D>(sv, BN / 2, BN, sl2x2, negx2, lsum0, lsum1, tS);
-          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        } else {
-          // the whole S row first, then its maximum: the base of a row that
-          // has none yet
-#pragma unroll
-          for (int c = 0; c < BN / 16; ++c) tmem_ld16p(tS + c * 16, &sv[c * 16]);
-          tc_wait_ld();
-          if (valid < BN) {
-#pragma unroll
-            for (int c = 0; c < BN; ++c)
-              if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
-          }
-          if constexpr (MR) {
-            if (p.g.token_mask) mask_frames(p.g, cur.row(), valid, allow, sv);
-          }
-          float m8[8];
+        for (int c = 24; c < BN; c += 16)
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            m8[q] = max3(__uint_as_float(sv[q]), __uint_as_float(sv[q + 8]), __uint_as_float(sv[q + 16]));
-#pragma unroll
-          for (int c = 24; c < BN; c += 16)
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              m8[q] = max3(m8[q], __uint_as_float(sv[c + q]), __uint_as_float(sv[c + q + 8]));
-          mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-        }
+            m8[q] = max3(m8[q], __uint_as_float(sv[c + q]), __uint_as_float(sv[c + q + 8]));
+        const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
         const float mx2 = mx * sl2;
-        // does this row need another base?  up: the maximum passed the base
-        // by more than 2^8 (or the row had no base yet); down: the row holds
-        // no mass yet (l = 0) and its logits lie more than 2^64 below the
-        // base it carried from an earlier unit
-        const bool need_up = mx2 > m_used + kRescaleLog2;
-        const bool need_down = l == 0.f && mx2 > -INFINITY && mx2 < m_used - kRebaseDownLog2;
-        const bool need = need_up || need_down;
-        if (!spec || __any_sync(0xffffffffu, need)) {
-          if (spec) tc_wait_st();        // the speculative P stores land first
-          const float m_new = need ? mx2 : m_used;
-          // O holds mass only where l > 0; a row with l = 0 has O = 0
-          const bool resc = need_up && l > 0.f;
-          if (__any_sync(0xffffffffu, resc)) {
+        if (t == 0) {
+          m_used = mx2;
+        } else {
+          const bool need = mx2 > m_used + kRescaleLog2;
+          if (__any_sync(0xffffffffu, need)) {
             // O of this row already holds every P V of earlier tiles: the
             // commit that released S(t) covers all earlier MMAs.
-            const float alpha = resc ? ex2(m_used - m_new) : 1.f;
+            const float m_new = need ? mx2 : m_used;
+            const float alpha = ex2(m_used - m_new);
             l *= alpha;
+            m_used = m_new;
             uint32_t v[32];
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
@@ -760,13 +743,27 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
               tmem_st32(tO + c * 32, v);
             }
           }
-          m_used = m_new;
-          // a row with no admissible key so far exponentiates against 0
-          const float neg = (m_used > -INFINITY) ? -m_used : 0.f;
-          const uint64_t negx2 = f2(neg, neg);
-          lsum0 = 0;
-          lsum1 = 0;
-          exp_store<D>(sv, 0, BN, sl2x2, negx2, lsum0, lsum1, tS);
+        }
+        // P = 2^(s*scale*log2e - m), rounded to bf16 into the first 64 S columns
+        // (general variant) a row with no admissible key so far exponentiates against 0
+        const float neg = (MR && !(m_used > -INFINITY)) ? 0.f : -m_used;
+        const uint64_t sl2x2 = f2(sl2, sl2), negx2 = f2(neg, neg);
+        uint64_t lsum0 = 0, lsum1 = 0;   // packed partial row sums (+0.0f bits)
+#pragma unroll
+        for (int g8 = 0; g8 < BN / 16; ++g8) {
+          // 16 probabilities -> 8 packed bf16 pairs -> TMEM columns [8*g8, 8*g8+8)
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int c = g8 * 16 + 2 * e;
+            float xa, xb;
+            unf2(fma2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, negx2), xa, xb);
+            const float a = (2 * e < emu_per16<D>()) ? exp2_poly(xa) : ex2(xa);
+            const float b = (2 * e + 1 < emu_per16<D>()) ? exp2_poly(xb) : ex2(xb);
+            if (e & 1) lsum1 = add2(lsum1, f2(a, b)); else lsum0 = add2(lsum0, f2(a, b));
+            pk[e] = pack_bf16(a, b);
+          }
+          tmem_st8(tS + g8 * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
         }
         {
           float s0, s1, s2, s3;
@@ -782,7 +779,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       if (!ok) break;
       // ---- epilogue: O of this row into registers, release the TMEM
       // accumulator to the next pair at once, then normalise and store.
-      if (!(ok = wait_warp(o_full(k), ofc & 1, ctl))) break;
+      if (!(ok = wait_bounded(o_full(k), ofc & 1, ctl))) break;
       ++ofc;
       tc_fence_after();
       // O is read in halves of up to 64 columns (fewer live registers); the
@@ -797,7 +794,6 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       const int rloc = w.rloc0 + k * BM + r;
       const size_t row_off = ((size_t)idx * p.g.BH + w.bh) * (size_t)p.g.Lmax + rloc;
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;   // a row with no admissible key: O = 0
-      m_seed = m_used;
       float4 *epi = reinterpret_cast<float4 *>(smem + C::OFF_EPI + (warp & 7) * 4096);
       // a masked unit in the fresh list has no slot: nothing is stored by slot
       const bool store = !p.out_by_slot || unit_pairs(p.g, w.i, pr.c) != 0ull;
@@ -912,7 +908,7 @@ cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const C
                                 float scale, void *out_O, float *out_lse, int out_by_slot,
                                 int state_bf16, unsigned char *out_valid, float *drift_rows,
                                 int *dev_status, long long wait_limit_ns, int num_sms,
-                                cudaStream_t stream) {
+                                int *work_counter, cudaStream_t stream) {
   attn::Params p;
   p.g = g;
   p.fresh_list = fresh_list;
@@ -925,6 +921,7 @@ cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const C
   p.drift_rows = out_by_slot ? drift_rows : nullptr;
   p.dev_status = dev_status;
   p.wait_limit_ns = wait_limit_ns;
+  p.sched = work_counter;
   const long long nqt2 = (g.Lmax + 255) / 256;
   const long long max_units = (long long)g.n_active * g.BH * nqt2;
   if (max_units == 0) return cudaSuccess;

@@ -17,7 +17,7 @@ cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const C
                                 float scale, void *out_O, float *out_lse, int out_by_slot,
                                 int state_bf16, unsigned char *out_valid, float *drift_rows,
                                 int *dev_status, long long wait_limit_ns, int num_sms,
-                                cudaStream_t stream);
+                                int *work_counter, cudaStream_t stream);
 size_t plan_workspace_bytes(const DevGeom &g);
 cudaError_t launch_plan(const DevGeom &g, const float *cache_lse, const unsigned char *cache_valid,
                         int band_k, int target, int anchor, signed char *plan_out, int *fresh_list,
@@ -366,7 +366,7 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q, co
                                     const int32_t *counts, float scale, void *out_O,
                                     float *out_lse, int32_t out_by_slot, int32_t state_bf16,
                                     uint8_t *out_valid, float *drift_rows, int32_t *dev_status,
-                                    ditango_stream stream) {
+                                    int32_t *work_counter, ditango_stream stream) {
   NvtxRange nvtx_range("ditango_attn_partial");
   DevGeom dg;
   ditango_status st = make_geom(g, &dg);
@@ -375,6 +375,7 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q, co
   if (drift_rows && !out_by_slot) return DITANGO_ERR_INVALID;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out_O))
     return DITANGO_ERR_INVALID;
+  if (work_counter && (reinterpret_cast<uintptr_t>(work_counter) & 7u)) return DITANGO_ERR_INVALID;
   // the stride of a dimension of size 1 is never used (frameworks report 0
   // or anything for it): give it the packed value
   int64_t qs[3], ks[3], vs[3];
@@ -399,7 +400,8 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q, co
   return cuda_status(launch_attn_partial(dg, tq, tk, tv, fresh_list, counts, scale, out_O, out_lse,
                                          out_by_slot ? 1 : 0, state_bf16 ? 1 : 0, out_valid,
                                          drift_rows, dev_status, g_wait_limit_ns.load(),
-                                         num_sms_current(), static_cast<cudaStream_t>(stream)));
+                                         num_sms_current(), work_counter,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan, const void *part_O,

@@ -102,15 +102,23 @@ mass_kernel(DevGeom g, const float *__restrict__ cache_lse,
   }
 }
 
-// Sum of a unit's (or the drift column's) block sums over every (b*h, row
-// block) of query partition i, in that order, in double precision.
-__device__ __forceinline__ double sum_blocks(const DevGeom &g, const float *partial, int i, int col) {
+// Mean over the rows of query partition i of a unit's (or the drift
+// column's) per-row values, from its block sums: one warp, lane l adds the
+// blocks j = l, l + 32, ... of the (b*h, block) sequence in double
+// precision, then a butterfly; every lane returns the same value.
+__device__ __forceinline__ float mean_blocks(const DevGeom &g, const float *partial, int i, int col,
+                                             int lane) {
   const int Li = g.part_off[i + 1] - g.part_off[i];
   const int nrb_i = weights::n_row_blocks(Li);
+  const int n = g.BH * nrb_i;
   double acc = 0.0;
-  for (int bh = 0; bh < g.BH; ++bh)
-    for (int rb = 0; rb < nrb_i; ++rb) acc += (double)partial[weights::partial_index(g, i, bh, rb, col)];
-  return acc;
+  for (int j = lane; j < n; j += 32) {
+    const int bh = j / nrb_i;
+    acc += (double)partial[weights::partial_index(g, i, bh, j - bh * nrb_i, col)];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return (float)(acc / ((double)g.BH * Li));
 }
 
 __global__ void __launch_bounds__(kSelThreads)
@@ -129,21 +137,44 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial,
   int n = 1;
   while (n < PP) n <<= 1;
   if (threadIdx.x == 0) n_forced = 0;
-  if (err && !anchor && threadIdx.x < g.P) {
+  // the importance w of every active unit (when it is computed from the
+  // block sums) and the local drift of every partition (error mode): one
+  // warp per value; w is kept in the first half of the key array until the
+  // keys are built
+  float *s_w = reinterpret_cast<float *>(keys);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool sum_w = !anchor && (!err || ea.refresh_w);
+  for (int p = warp; p < PP; p += kSelThreads / 32) {
+    const int i = p / G, c = p - (p / G) * G;
+    float wv = 0.f;
+    if (sum_w && ((g.row_mask[i] >> c) & 1ull)) wv = mean_blocks(g, partial, i, c, lane);
+    if (lane == 0) s_w[p] = wv;
+  }
+  if (err && !anchor) {
     // local drift of partition i in the last step (0 if it had no earlier state)
-    const int i = threadIdx.x;
-    float d = 0.f;
-    if (ea.local_ok[i]) {
-      const int Li = g.part_off[i + 1] - g.part_off[i];
-      d = (float)(sum_blocks(g, partial, i, G) / ((double)g.BH * Li));
+    for (int i = warp; i < g.P; i += kSelThreads / 32) {
+      const float d = ea.local_ok[i] ? mean_blocks(g, partial, i, G, lane) : 0.f;
+      if (lane == 0) {
+        s_delta[i] = d;
+        ea.delta[i] = d;
+      }
     }
-    s_delta[i] = d;
-    ea.delta[i] = d;
   }
   __syncthreads();
+  constexpr int kPerThread = kMaxP * kMaxP / kSelThreads;
+  float w_mine[kPerThread];
+#pragma unroll
+  for (int q = 0; q < kPerThread; ++q) {
+    const int p = threadIdx.x + q * kSelThreads;
+    w_mine[q] = (p < PP) ? s_w[p] : 0.f;
+  }
+  __syncthreads();   // the keys overwrite s_w from here on
 
   int my_forced = 0;
-  for (int p = threadIdx.x; p < n; p += kSelThreads) {
+#pragma unroll
+  for (int q = 0; q < kPerThread; ++q) {
+    const int p = threadIdx.x + q * kSelThreads;
+    if (p >= n) break;
     unsigned long long key = ~0ull;
     if (p < PP) {
       const int i = p / G, c = p - (p / G) * G;
@@ -154,9 +185,8 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial,
         const int slot = slot_of(g, i, c);
         const bool valid = cache_valid == nullptr || cache_valid[slot] != 0;
         if (!anchor) {
-          if (!err || ea.refresh_w) {
-            const int Li = g.part_off[i + 1] - g.part_off[i];
-            w = (float)(sum_blocks(g, partial, i, c) / ((double)g.BH * Li));
+          if (sum_w) {
+            w = w_mine[q];
             if (err) ea.w[p] = w;
           } else {
             w = ea.w[p];
@@ -211,7 +241,6 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial,
   const int p0 = threadIdx.x * per;
   int cnt = 0;
   for (int p = p0; p < p0 + per && p < PP; ++p) cnt += fresh[p];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = cnt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {

@@ -71,7 +71,7 @@ int main(int argc, char **argv) {
   float *sO, *slse, *out, *olse;
   uint8_t *valid;
   int8_t *plan;
-  int32_t *fresh, *counts, *status;
+  int32_t *fresh, *counts, *status, *work;
   CK(cudaMalloc((void **)&q, nqkv * 2));
   CK(cudaMalloc((void **)&k, nqkv * 2));
   CK(cudaMalloc((void **)&v, nqkv * 2));
@@ -82,9 +82,11 @@ int main(int argc, char **argv) {
   CK(cudaMalloc((void **)&fresh, slots * 4));
   CK(cudaMalloc((void **)&counts, 8));
   CK(cudaMalloc((void **)&status, 4));
+  CK(cudaMalloc((void **)&work, 8));
   CK(cudaMalloc((void **)&out, nqkv * 4));
   CK(cudaMalloc((void **)&olse, (size_t)B * H * N * 4));
   CK(cudaMemset(status, 0, 4));
+  CK(cudaMemset(work, 0, 8));   /* the attention kernel's work counter, zeroed once */
   CK(cudaMemset(valid, 0, slots));
   CK(cudaMemcpy(q, hq, nqkv * 2, cudaMemcpyHostToDevice));
   CK(cudaMemcpy(k, hk, nqkv * 2, cudaMemcpyHostToDevice));
@@ -93,7 +95,8 @@ int main(int argc, char **argv) {
   CK(cudaStreamCreate(&st));
   /* an anchor step: every pair fresh, states written into the cache slots */
   DK(ditango_plan(&g, NULL, valid, 0, 1.0, 1, plan, fresh, counts, NULL, NULL, 0, st));
-  DK(ditango_attn_partial(&g, q, k, v, fresh, counts, 0.0f, sO, slse, 1, 0, valid, NULL, status, st));
+  DK(ditango_attn_partial(&g, q, k, v, fresh, counts, 0.0f, sO, slse, 1, 0, valid, NULL, status, work,
+                          st));
   DK(ditango_merge(&g, plan, NULL, NULL, sO, slse, valid, 0, 0, out, 1, NULL, olse, NULL, st));
   CK(cudaStreamSynchronize(st));
   int32_t hstatus = -1;

@@ -3,6 +3,10 @@
 interleavings.
 
 The kernel's roles talk only through mbarriers in shared memory:
+  * the producer warp takes each work item (from the work counter or a fixed
+    stride), writes its index into a 2-slot ring in shared memory and
+    publishes it (item_full); the MMA warp and the eight softmax warps read
+    it and free the slot (item_empty); an index of -1 ends the CTA's work;
   * the producer warp arms a full barrier (arrive + expect_tx) and issues TMA
     loads of the Q tiles and of the two K and V stages;
   * the MMA warp issues tcgen05.mma (S = Q K^T into TMEM, O += P V with P
@@ -22,6 +26,8 @@ Checked on every interleaving:
     so while a role waits for phase n its barrier never completes phase
     n + 1; and each parity the kernel computes is that of the phase it means;
   * no arrival beyond a barrier's count within one phase;
+  * no data race on the item ring: the producer never writes a slot while
+    a consumer reads it;
   * no data race on TMEM (S/P and O of each Q tile) or on the shared-memory
     tiles (Q0, Q1, K and V stages): a softmax access never overlaps an
     asynchronous operation in flight that writes the region (or reads it,
@@ -72,8 +78,14 @@ class Bar:
             self.pending = self.count
 
 
+CONSUMERS = 1 + 2 * WARPS_PER_TILE      # the MMA warp and the eight softmax warps
+
+
 def barriers():
     b = {"q_full": 1, "q_empty": 1, "drain": 1}
+    for s in range(2):
+        b[f"item_full{s}"] = 1
+        b[f"item_empty{s}"] = CONSUMERS
     for s in range(STAGES):
         for n in ("k_full", "k_empty", "v_full", "v_empty"):
             b[f"{n}{s}"] = 1
@@ -99,12 +111,46 @@ def W(bar, parity, n, abortable=True):
     return ("wait", bar, parity, n, abortable)
 
 
+def publish(ic, mut):
+    """The producer writes item ic's index (or the end marker) into slot
+    ic % 2 once every consumer has read the slot's previous entry."""
+    s = ic & 1
+    if mut != "producer_skips_item_empty":
+        ok = yield W(f"item_empty{s}", ((ic >> 1) & 1) ^ 1, (ic >> 1) - 1)
+        if not ok:
+            return False
+    yield ("hold", f"ITEM{s}", "w")
+    yield ("release", f"ITEM{s}")
+    yield ("arrive", f"item_full{s}")
+    return True
+
+
+def take(ic, mut):
+    """A consumer reads entry ic of the ring and frees the slot."""
+    s = ic & 1
+    ok = yield W(f"item_full{s}", (ic >> 1) & 1, ic >> 1)
+    if not ok:
+        return False
+    if mut == "consumer_frees_slot_before_reading":
+        yield ("arrive", f"item_empty{s}")
+    yield ("hold", f"ITEM{s}", "r")
+    yield ("release", f"ITEM{s}")
+    if mut != "consumer_frees_slot_before_reading":
+        yield ("arrive", f"item_empty{s}")
+    return True
+
+
 def producer(items, mut):
     kc = vc = uc = 0
     q_armed = None              # phase index of the last arming, per barrier
     k_armed, v_armed = {}, {}
     ok = True
+    ic = 0
     for has1, Ts in items:
+        ok = yield from publish(ic, mut)
+        ic += 1
+        if not ok:
+            break
         ok = yield W("q_empty", (uc & 1) ^ 1, uc - 1)
         if not ok:
             break
@@ -137,6 +183,8 @@ def producer(items, mut):
         if not ok:
             break
         uc += 1
+    if ok:
+        ok = yield from publish(ic, mut)          # the end marker
     # every load issued lands before the warp exits, on both paths: when
     # another role gave up, this warp may still end its loop with ok (each
     # of its last waits completed at once) while nothing consumes its loads
@@ -165,7 +213,12 @@ def mma(items, mut):
     def pv(k, vs, acc):
         return ("mma", {f"S{k}", f"V{vs}"} | ({f"O{k}"} if acc else set()), {f"O{k}"})
 
+    ic = 0
     for has1, Ts in items:
+        ok = yield from take(ic, mut)
+        ic += 1
+        if not ok:
+            break
         ok = yield W("q_full", uc & 1, uc)
         if not ok:
             break
@@ -232,6 +285,8 @@ def mma(items, mut):
         if not ok:
             break
         uc += 1
+    if ok:
+        yield from take(ic, mut)                  # the end marker
     # drain: every MMA issued must finish before TMEM is released
     if mut != "mma_stops_without_drain":
         yield ("commit", "drain")
@@ -242,7 +297,12 @@ def softmax_warp(k, items, rng, rescale_p, mut):
     sc = ofc = 0
     S, O = f"S{k}", f"O{k}"
     ok = True
+    ic = 0
     for has1, Ts in items:
+        ok = yield from take(ic, mut)
+        ic += 1
+        if not ok:
+            break
         if k == 1 and not has1:
             continue
         for T in Ts:
@@ -273,6 +333,8 @@ def softmax_warp(k, items, rng, rescale_p, mut):
             yield ("arrive", f"o_empty{k}")
         if not ok:
             break
+    if ok:
+        yield from take(ic, mut)                  # the end marker
 
 
 # ---------------------------------------------------------------- scheduler
@@ -395,6 +457,11 @@ def run(items, seed, rescale_p=0.5, mut=None, timeout_p=0.0, max_steps=2_000_000
             mma_q.append(op)
         elif what == "hold":
             region, mode = op[1], op[2]
+            if region.startswith("ITEM"):
+                # the ring slots are plain shared memory written and read by roles
+                for other, h in holds.items():
+                    if other != role and region in h and "w" in (mode, h[region]):
+                        raise Violation(f"{role} and {other} race on {region}")
             r_set = {region}
             w_set = {region} if mode == "w" else set()
             for m in mma_in_flight():
@@ -435,6 +502,9 @@ def test_protocol_on_random_items_and_interleavings(seed):
     n_units1 = sum(len(Ts) for has1, Ts in items if has1)
     n_tiles1 = sum(sum(Ts) for has1, Ts in items if has1)
     assert B["q_full"].phase == B["q_empty"].phase == len(items)
+    # every item and the end marker went through the ring
+    assert B["item_full0"].phase + B["item_full1"].phase == len(items) + 1
+    assert B["item_empty0"].phase + B["item_empty1"].phase == len(items) + 1
     assert sum(B[f"k_full{s}"].phase for s in range(STAGES)) == n_tiles
     assert sum(B[f"v_empty{s}"].phase for s in range(STAGES)) == n_tiles
     assert B["s_full0"].phase == B["p_full0"].phase == n_tiles
@@ -457,15 +527,20 @@ def test_protocol_edge_items(items):
 
 
 @pytest.mark.parametrize("mut", ["mma_skips_p_full", "softmax_skips_o_full", "k_released_before_qk",
-                                 "p_full_before_p_written", "producer_skips_k_empty"])
+                                 "p_full_before_p_written", "producer_skips_k_empty",
+                                 "producer_skips_item_empty", "consumer_frees_slot_before_reading"])
 def test_planted_mistakes_are_caught(mut):
-    items = [(True, [3, 2]), (True, [1, 4]), (False, [2])]
+    # items without a second Q tile let the MMA warp and the producer run
+    # ahead of the second softmax warpgroup, which only reads their entries
+    item_lists = [[(True, [3, 2]), (True, [1, 4]), (False, [2])],
+                  [(True, [3]), (False, [1]), (False, [1]), (False, [1]), (True, [1])]]
     caught = 0
-    for seed in range(40):
-        try:
-            run(items, seed, mut=mut)
-        except Violation:
-            caught += 1
+    for items in item_lists:
+        for seed in range(40):
+            try:
+                run(items, seed, mut=mut)
+            except Violation:
+                caught += 1
     assert caught > 0, mut
 
 
@@ -512,17 +587,22 @@ def test_stop_path_without_its_drain_is_caught(mut):
 
 
 def cta_items(part_off, fresh_rows, BH, cta, grid, BM=128, BN=128):
-    """The item list one CTA of the persistent grid walks: items are
-    (partition, batch-head, pair of 128-row Q tiles) in the kernel's order,
-    taken round-robin with stride `grid`; fresh_rows[i] lists the key counts
-    of the fresh units of partition i."""
+    """The item list one CTA of the persistent grid walks without a work
+    counter: items are (partition, batch-head, pair of 128-row Q tiles) in
+    the kernel's order -- b*h-major, every partition's last pair of Q tiles
+    after all the others -- taken with stride `grid`; fresh_rows[i] lists
+    the key counts of the fresh units of partition i."""
     P = len(part_off) - 1
     Lmax = max(part_off[i + 1] - part_off[i] for i in range(P))
     nqt2 = -(-Lmax // (2 * BM))
+    n_main = P * BH * (nqt2 - 1)
     items = []
     for it in range(cta, P * BH * nqt2, grid):
-        qt2, rest = it % nqt2, it // nqt2
-        i = rest // BH
+        if it < n_main:
+            qt2, rest = it % (nqt2 - 1), it // (nqt2 - 1)
+        else:
+            qt2, rest = nqt2 - 1, it - n_main
+        i = rest % P
         rem = part_off[i + 1] - part_off[i] - qt2 * 2 * BM
         if rem <= 0 or not fresh_rows[i]:
             continue                     # not live: no role touches it
