@@ -67,7 +67,9 @@ typedef enum {
   DITANGO_ERR_INVALID = 1,      /* bad argument (null, negative, inconsistent) */
   DITANGO_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels handle */
   DITANGO_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
-  DITANGO_ERR_TIMEOUT = 4       /* device: a pipeline wait exceeded its limit */
+  DITANGO_ERR_TIMEOUT = 4,      /* device: a pipeline wait exceeded its limit */
+  DITANGO_ERR_BOUNDS = 5        /* device, checked builds: a device-resident input (a count,
+                                   a fresh list, a plan code) out of range */
 } ditango_status;
 
 enum { DITANGO_PLAN_SKIP = 0, DITANGO_PLAN_FRESH = 1, DITANGO_PLAN_REUSE = 2 };
@@ -134,6 +136,9 @@ ditango_status ditango_slot_table(const ditango_geom *g, int32_t *slot_out);
  * [P][B*H][ceil(Lmax / 128)][G + 1], see ditango_merge). */
 size_t ditango_plan_workspace_size(const ditango_geom *g);
 
+/* The same value under its shorter name. */
+size_t ditango_workspace_size(const ditango_geom *g);
+
 /* Plan: per unit, fresh or reuse (DiTango, 1. Anchor-Guided Selection
  * Planner and its group strategy; spatial locality from Metodologia).
  *   cache_lse    dev float32 state-buffer lse indexed by slot (the previous
@@ -173,9 +178,12 @@ ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
  * whose composed states are the cache's valid states, the plan and scores
  * are bit-identical to ditango_plan's on that cache.
  *   mass_partials  dev, written by ditango_merge, mass_bytes >=
- *                  ditango_plan_workspace_size (else INVALID).
+ *                  ditango_plan_workspace_size (else INVALID); the part of
+ *                  the buffer past the block sums serves as scratch (the
+ *                  per-unit means), so the block sums themselves are left
+ *                  unchanged.
  *   cache_valid    as for ditango_plan (invalid slots are forced fresh). */
-ditango_status ditango_plan_from_mass(const ditango_geom *g, const float *mass_partials,
+ditango_status ditango_plan_from_mass(const ditango_geom *g, float *mass_partials,
                                      size_t mass_bytes, const uint8_t *cache_valid,
                                      int32_t band_k, double budget, int8_t *plan,
                                      int32_t *fresh_list, int32_t *counts, float *score_out,
@@ -366,6 +374,21 @@ ditango_status ditango_plan_noalloc(const ditango_geom *g, const float *cache_ls
 /* Time limit, in nanoseconds, of every wait inside the kernels (default
  * 1e9).  Process-wide; read at each launch. */
 void ditango_set_wait_limit_ns(int64_t ns);
+
+/* Checked builds.  The library built with -DDITANGO_CHECK
+ * (libditango_check.so) validates the device-resident inputs the host cannot
+ * see without a synchronisation -- ditango_attn_partial's counts[0] (at most
+ * the active units) and fresh list (unit indices in range, active, strictly
+ * row-major), and the plan codes ditango_merge reads -- before using them.  A
+ * bad attention input makes the kernel compute nothing and record
+ * DITANGO_ERR_BOUNDS (also in dev_status when given); a bad plan code is
+ * recorded and the unit left out.  The release build skips these checks.
+ * ditango_checked_build: 1 in a checked build, 0 otherwise.
+ * ditango_check_status: the recorded status (DITANGO_OK if none) into
+ * *status_out (host), cleared when reset != 0; synchronises with the device.
+ * Always 0 in the release build. */
+int32_t ditango_checked_build(void);
+ditango_status ditango_check_status(int32_t *status_out, int32_t reset);
 
 /* Failure-detection self-test: launches one block that waits on a barrier
  * nothing will complete, with a limit of limit_ns; the kernel returns and

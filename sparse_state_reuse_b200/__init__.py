@@ -23,7 +23,8 @@ from ._abi import (  # noqa: F401
     ditango_slot_table, ditango_plan_workspace_size, ditango_plan, ditango_attn_partial,
     ditango_merge, ditango_cache_update, ditango_set_wait_limit_ns,
     ditango_selftest_bounded_wait, ditango_plan_noalloc, ditango_cache_compose, status_string,
-    ditango_plan_error, error_state, ditango_plan_from_mass,
+    ditango_plan_error, error_state, ditango_plan_from_mass, ditango_checked_build,
+    ditango_check_status,
 )
 
 

@@ -12,9 +12,11 @@ import ctypes as C
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libditango.so")
+# DITANGO_LIBRARY selects another build of the same ABI, e.g. the checked
+# build libditango_check.so
+LIB_PATH = os.environ.get("DITANGO_LIBRARY") or os.path.join(_HERE, "libditango.so")
 
-OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = 0, 1, 2, 3, 4, 5
 PLAN_SKIP, PLAN_FRESH, PLAN_REUSE = 0, 1, 2
 
 
@@ -65,6 +67,7 @@ _SIGS = {
     "ditango_state_rows": (C.c_int64, [_G]),
     "ditango_slot_table": (C.c_int, [_G, _P]),
     "ditango_plan_workspace_size": (C.c_size_t, [_G]),
+    "ditango_workspace_size": (C.c_size_t, [_G]),
     "ditango_plan": (C.c_int, [_G, _P, _P, C.c_int32, C.c_double, C.c_int32, _P, _P, _P, _P, _P,
                                C.c_size_t, _P]),
     "ditango_attn_partial": (C.c_int, [_G, _P, _P, _P, _P, _P, C.c_float, _P, _P, C.c_int32,
@@ -81,6 +84,8 @@ _SIGS = {
                                        _P, _P]),
     "ditango_cache_compose": (C.c_int, [_G, _G, _P, _P, _P, _P, _P, _P, C.c_int32, _P]),
     "ditango_set_wait_limit_ns": (None, [C.c_int64]),
+    "ditango_checked_build": (C.c_int32, []),
+    "ditango_check_status": (C.c_int, [_P, C.c_int32]),
     "ditango_selftest_bounded_wait": (C.c_int, [C.c_int64, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -264,6 +269,17 @@ def ditango_cache_compose(fine, coarse, fine_O, fine_lse, fine_valid, coarse_O, 
     _check("ditango_cache_compose", _lib.ditango_cache_compose(
         fine.ref, coarse.ref, _ptr(fine_O), _ptr(fine_lse), _ptr(fine_valid), _ptr(coarse_O),
         _ptr(coarse_lse), _ptr(coarse_valid), int(bool(state_bf16)), _stream(stream)))
+
+
+def ditango_checked_build() -> bool:
+    return bool(_lib.ditango_checked_build())
+
+
+def ditango_check_status(reset=False) -> int:
+    """Status recorded by a checked build's device-side input checks (0: none)."""
+    out = C.c_int32(0)
+    _check("ditango_check_status", _lib.ditango_check_status(C.byref(out), int(bool(reset))))
+    return out.value
 
 
 def ditango_set_wait_limit_ns(ns: int) -> None:

@@ -1,9 +1,11 @@
 """Build libditango.so in-tree with nvcc for sm_100a.
 
-    python sparse_state_reuse_b200/build.py
+    python sparse_state_reuse_b200/build.py [--check]
 
 Objects go to _build/ at the repository root; the shared library is written
-next to this file so that it travels with the source tree.
+next to this file so that it travels with the source tree.  --check builds
+the checked library libditango_check.so instead (-DDITANGO_CHECK: the
+kernels validate their device-resident inputs; objects in _build/check).
 """
 from __future__ import annotations
 
@@ -18,7 +20,7 @@ CSRC = os.path.join(HERE, "csrc")
 OBJDIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libditango.so")
 SOURCES = ["ditango_api.cu", "attn_partial.cu", "plan.cu", "merge.cu", "selftest.cu"]
-HEADERS = ["common.cuh"]
+HEADERS = ["common.cuh", "weights.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
@@ -36,15 +38,18 @@ def _newer(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    os.makedirs(OBJDIR, exist_ok=True)
+def build(verbose: bool = False, force: bool = False, check: bool = False) -> str:
+    objdir = os.path.join(OBJDIR, "check") if check else OBJDIR
+    lib = os.path.join(HERE, "libditango_check.so") if check else LIB
+    flags = FLAGS + (["-DDITANGO_CHECK"] if check else [])
+    os.makedirs(objdir, exist_ok=True)
     hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(ROOT, "include", "ditango.h")]
     jobs = []
     for src in SOURCES:
         s = os.path.join(CSRC, src)
-        o = os.path.join(OBJDIR, src.replace(".cu", ".o"))
+        o = os.path.join(objdir, src.replace(".cu", ".o"))
         if force or _newer(o, [s] + hdrs):
-            jobs.append([NVCC, *FLAGS, "-c", s, "-o", o])
+            jobs.append([NVCC, *flags, "-c", s, "-o", o])
 
     def run(cmd):
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -55,11 +60,11 @@ def build(verbose: bool = False, force: bool = False) -> str:
 
     with ThreadPoolExecutor(max(1, min(len(jobs), os.cpu_count() or 1))) as ex:
         list(ex.map(run, jobs))
-    objs = [os.path.join(OBJDIR, s.replace(".cu", ".o")) for s in SOURCES]
-    if force or jobs or _newer(LIB, objs):
-        run([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", LIB, *objs])
-    return LIB
+    objs = [os.path.join(objdir, s.replace(".cu", ".o")) for s in SOURCES]
+    if force or jobs or _newer(lib, objs):
+        run([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", lib, *objs])
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv, force="-f" in sys.argv))
+    print(build(verbose="-v" in sys.argv, force="-f" in sys.argv, check="--check" in sys.argv))

@@ -287,6 +287,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
+// Checked builds record a bad device-resident input here (and in the
+// caller's dev_status); read and cleared by ditango_check_status.
+__device__ int g_attn_check_status;
+
+__device__ __forceinline__ void record_check_failure(int *dev_status) {
+  atomicExch(&g_attn_check_status, (int)DITANGO_ERR_BOUNDS);
+  if (dev_status) atomicExch(dev_status, (int)DITANGO_ERR_BOUNDS);
+}
+
 // Frame of a token (tokens past the end count in the last frame).
 __device__ __forceinline__ int frame_of(const DevGeom &g, int tok) {
   int lo = 0, hi = g.F - 1;
@@ -356,9 +365,37 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   // fresh-list range of every query partition (the list is row-major)
   __shared__ int row_fresh[kMaxP + 1];
   if (threadIdx.x <= p.g.P) row_fresh[threadIdx.x] = 0;
+#ifdef DITANGO_CHECK
+  // Checked build: the device-resident inputs are validated before any use.
+  // A count beyond the active units, a unit index out of range or inactive,
+  // or a list that is not strictly row-major: nothing is computed and
+  // DITANGO_ERR_BOUNDS is recorded.
+  __shared__ int s_bad;
+  if (threadIdx.x == 0) s_bad = 0;
   __syncthreads();
   {
     const int n_fresh = __ldg(p.counts);
+    if (n_fresh < 0 || n_fresh > p.g.n_active) {
+      s_bad = 1;   // every thread writes the same value
+    } else {
+      for (int f = threadIdx.x; f < n_fresh; f += blockDim.x) {
+        const int u = __ldg(p.fresh_list + f);
+        bool ok = u >= 0 && u < p.g.P * p.g.G;
+        if (ok) ok = ((p.g.row_mask[u / p.g.G] >> (u % p.g.G)) & 1ull) != 0ull;
+        if (ok && f > 0) ok = __ldg(p.fresh_list + f - 1) < u;
+        if (!ok) s_bad = 1;
+      }
+    }
+  }
+  __syncthreads();
+  const bool bad_input = s_bad != 0;
+  if (bad_input && threadIdx.x == 0) record_check_failure(p.dev_status);
+#else
+  constexpr bool bad_input = false;
+#endif
+  __syncthreads();
+  {
+    const int n_fresh = bad_input ? 0 : __ldg(p.counts);
     const int n_units = p.g.P * p.g.G;
     for (int f = threadIdx.x; f < n_fresh; f += blockDim.x) {
       const int u = __ldg(p.fresh_list + f);
@@ -730,7 +767,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             // O of this row already holds every P V of earlier tiles: the
             // commit that released S(t) covers all earlier MMAs.
             const float m_new = need ? mx2 : m_used;
-            const float alpha = ex2(m_used - m_new);
+            const float alpha = need ? ex2(m_used - m_new) : 1.f;   // 1, not NaN, for a row still at -inf
             l *= alpha;
             m_used = m_new;
             uint32_t v[32];
@@ -947,6 +984,14 @@ cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const C
     default:
       return cudaErrorInvalidValue;
   }
+}
+
+// Read (and optionally clear) this file's check word.
+cudaError_t attn_check_status(int *out, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, attn::g_attn_check_status, sizeof(int));
+  if (e != cudaSuccess || !reset) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(attn::g_attn_check_status, &zero, sizeof(int));
 }
 
 }  // namespace ditango

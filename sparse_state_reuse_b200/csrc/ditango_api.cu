@@ -39,6 +39,8 @@ cudaError_t launch_cache_compose(const DevGeom &fine, const DevGeom &coarse, con
                                  int state_bf16, cudaStream_t stream);
 cudaError_t launch_bounded_wait_selftest(long long limit_ns, int *dev_status,
                                          cudaStream_t stream);
+cudaError_t attn_check_status(int *out, bool reset);
+cudaError_t merge_check_status(int *out, bool reset);
 }  // namespace ditango
 
 using namespace ditango;
@@ -255,6 +257,7 @@ const char *ditango_status_string(int32_t s) {
     case DITANGO_ERR_UNSUPPORTED: return "unsupported shape";
     case DITANGO_ERR_CUDA: return "CUDA error";
     case DITANGO_ERR_TIMEOUT: return "device wait timed out";
+    case DITANGO_ERR_BOUNDS: return "device input out of range";
     default: return "unknown status";
   }
 }
@@ -293,6 +296,8 @@ size_t ditango_plan_workspace_size(const ditango_geom *g) {
   return plan_workspace_bytes(dg);
 }
 
+size_t ditango_workspace_size(const ditango_geom *g) { return ditango_plan_workspace_size(g); }
+
 ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
                             const uint8_t *cache_valid, int32_t band_k, double budget,
                             int32_t anchor, int8_t *plan, int32_t *fresh_list, int32_t *counts,
@@ -314,7 +319,7 @@ ditango_status ditango_plan(const ditango_geom *g, const float *cache_lse,
                                  nullptr, nullptr, nullptr, nullptr, 0, 0));
 }
 
-ditango_status ditango_plan_from_mass(const ditango_geom *g, const float *mass_partials,
+ditango_status ditango_plan_from_mass(const ditango_geom *g, float *mass_partials,
                                      size_t mass_bytes, const uint8_t *cache_valid,
                                      int32_t band_k, double budget, int8_t *plan,
                                      int32_t *fresh_list, int32_t *counts, float *score_out,
@@ -329,7 +334,7 @@ ditango_status ditango_plan_from_mass(const ditango_geom *g, const float *mass_p
   const int target = plan_target(&dg, band_k, budget);
   return cuda_status(launch_plan(dg, nullptr, cache_valid, band_k, target, 0,
                                  reinterpret_cast<signed char *>(plan), fresh_list, counts,
-                                 score_out, const_cast<float *>(mass_partials),
+                                 score_out, mass_partials,
                                  static_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr,
                                  nullptr, nullptr, 0, 1));
 }
@@ -493,6 +498,24 @@ ditango_status ditango_cache_compose(const ditango_geom *fine, const ditango_geo
 }
 
 void ditango_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns.store(ns > 0 ? ns : 1); }
+
+int32_t ditango_checked_build(void) {
+#ifdef DITANGO_CHECK
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+ditango_status ditango_check_status(int32_t *status_out, int32_t reset) {
+  if (!status_out) return DITANGO_ERR_INVALID;
+  int a = 0, m = 0;
+  cudaError_t e = attn_check_status(&a, reset != 0);
+  if (e == cudaSuccess) e = merge_check_status(&m, reset != 0);
+  if (e != cudaSuccess) return cuda_status(e);
+  *status_out = a != 0 ? a : m;
+  return DITANGO_OK;
+}
 
 ditango_status ditango_selftest_bounded_wait(int64_t limit_ns, int32_t *dev_status,
                                              ditango_stream stream) {

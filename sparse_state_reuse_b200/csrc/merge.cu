@@ -31,6 +31,10 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kRowsPerBlock = 128;
 constexpr int kBatch = 4;    // O vectors per row in flight per lane
 
+// Checked builds record a bad plan code here; read and cleared by
+// ditango_check_status.
+__device__ int g_merge_check_status;
+
 struct Src {
   const char *O;     // [Lmax][d] block of this (index, b*h): float32, or bf16 (SB)
   const float *lse;  // [Lmax]
@@ -185,6 +189,16 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
     int a = 0;
     for (int c = 0; c < G; ++c) {
       s_state_of[c] = -1;
+#ifdef DITANGO_CHECK
+      {
+        // a plan code outside {skip, fresh, reuse}, or anything but skip on a
+        // masked unit: recorded (the unit is then left out, as always)
+        const int code = plan[i * G + c];
+        const bool act = (g.row_mask[i] >> c) & 1ull;
+        if (code < 0 || code > 2 || (!act && code != 0))
+          atomicExch(&g_merge_check_status, (int)DITANGO_ERR_BOUNDS);
+      }
+#endif
       if (!((g.row_mask[i] >> c) & 1ull)) continue;
       const int code = plan[i * G + c];
       const int slot = slot_of(g, i, c);
@@ -513,6 +527,14 @@ cudaError_t launch_cache_compose(const DevGeom &fine, const DevGeom &coarse, con
     default:
       return cudaErrorInvalidValue;
   }
+}
+
+// Read (and optionally clear) this file's check word.
+cudaError_t merge_check_status(int *out, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, merge::g_merge_check_status, sizeof(int));
+  if (e != cudaSuccess || !reset) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(merge::g_merge_check_status, &zero, sizeof(int));
 }
 
 }  // namespace ditango

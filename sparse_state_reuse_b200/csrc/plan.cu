@@ -103,22 +103,52 @@ mass_kernel(DevGeom g, const float *__restrict__ cache_lse,
 }
 
 // Mean over the rows of query partition i of a unit's (or the drift
-// column's) per-row values, from its block sums: one warp, lane l adds the
-// blocks j = l, l + 32, ... of the (b*h, block) sequence in double
-// precision, then a butterfly; every lane returns the same value.
+// column's) per-row values, from its block sums: one warp; lane l adds the
+// blocks j = l + 32 m of the (b*h, block) sequence into accumulator m % 4
+// (four loads in flight), the four accumulators are added in order, then a
+// butterfly; every lane returns the same value.  Double precision.
 __device__ __forceinline__ float mean_blocks(const DevGeom &g, const float *partial, int i, int col,
                                              int lane) {
   const int Li = g.part_off[i + 1] - g.part_off[i];
   const int nrb_i = weights::n_row_blocks(Li);
   const int n = g.BH * nrb_i;
-  double acc = 0.0;
-  for (int j = lane; j < n; j += 32) {
-    const int bh = j / nrb_i;
-    acc += (double)partial[weights::partial_index(g, i, bh, j - bh * nrb_i, col)];
-  }
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int j0 = lane; j0 < n; j0 += 4 * 32) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  return (float)(acc / ((double)g.BH * Li));
+    for (int m = 0; m < 4; ++m) {
+      const int j = j0 + m * 32;
+      if (j < n) {
+        const int bh = j / nrb_i;
+        acc[m] += (double)partial[weights::partial_index(g, i, bh, j - bh * nrb_i, col)];
+      }
+    }
+  }
+  double a = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+  return (float)(a / ((double)g.BH * Li));
+}
+
+// Second stage of the mass score: one warp per active unit -- and, in error
+// mode, per partition's drift column -- turns the block sums into the mean
+// (w, or delta), written to the end of the workspace: [P*G] then [P].
+constexpr int kReduceWarps = 8;
+__global__ void __launch_bounds__(kReduceWarps * 32)
+mass_reduce_kernel(DevGeom g, const float *__restrict__ partial, float *__restrict__ means,
+                   int do_mass, int do_drift, const unsigned char *__restrict__ local_ok) {
+  const int lane = threadIdx.x & 31;
+  const int v = blockIdx.x * kReduceWarps + (threadIdx.x >> 5);
+  const int PG = g.P * g.G;
+  if (v < PG) {
+    const int i = v / g.G, c = v - (v / g.G) * g.G;
+    float m = 0.f;
+    if (do_mass && ((g.row_mask[i] >> c) & 1ull)) m = mean_blocks(g, partial, i, c, lane);
+    if (lane == 0) means[v] = m;
+  } else if (v < PG + g.P && do_drift) {
+    const int i = v - PG;
+    const float d = (local_ok == nullptr || local_ok[i]) ? mean_blocks(g, partial, i, g.G, lane) : 0.f;
+    if (lane == 0) means[v] = d;
+  }
 }
 
 __global__ void __launch_bounds__(kSelThreads)
@@ -138,38 +168,17 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial,
   while (n < PP) n <<= 1;
   if (threadIdx.x == 0) n_forced = 0;
   // the importance w of every active unit (when it is computed from the
-  // block sums) and the local drift of every partition (error mode): one
-  // warp per value; w is kept in the first half of the key array until the
-  // keys are built
-  float *s_w = reinterpret_cast<float *>(keys);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // block sums) and the local drift of every partition (error mode), as the
+  // reduction kernel left them at the end of the workspace
   const bool sum_w = !anchor && (!err || ea.refresh_w);
-  for (int p = warp; p < PP; p += kSelThreads / 32) {
-    const int i = p / G, c = p - (p / G) * G;
-    float wv = 0.f;
-    if (sum_w && ((g.row_mask[i] >> c) & 1ull)) wv = mean_blocks(g, partial, i, c, lane);
-    if (lane == 0) s_w[p] = wv;
-  }
-  if (err && !anchor) {
-    // local drift of partition i in the last step (0 if it had no earlier state)
-    for (int i = warp; i < g.P; i += kSelThreads / 32) {
-      const float d = ea.local_ok[i] ? mean_blocks(g, partial, i, G, lane) : 0.f;
-      if (lane == 0) {
-        s_delta[i] = d;
-        ea.delta[i] = d;
-      }
-    }
+  const float *means = partial + weights::n_partials(g);
+  if (err && !anchor && threadIdx.x < g.P) {
+    const float d = means[PP + threadIdx.x];
+    s_delta[threadIdx.x] = d;
+    ea.delta[threadIdx.x] = d;
   }
   __syncthreads();
   constexpr int kPerThread = kMaxP * kMaxP / kSelThreads;
-  float w_mine[kPerThread];
-#pragma unroll
-  for (int q = 0; q < kPerThread; ++q) {
-    const int p = threadIdx.x + q * kSelThreads;
-    w_mine[q] = (p < PP) ? s_w[p] : 0.f;
-  }
-  __syncthreads();   // the keys overwrite s_w from here on
-
   int my_forced = 0;
 #pragma unroll
   for (int q = 0; q < kPerThread; ++q) {
@@ -186,7 +195,7 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial,
         const bool valid = cache_valid == nullptr || cache_valid[slot] != 0;
         if (!anchor) {
           if (sum_w) {
-            w = w_mine[q];
+            w = means[p];
             if (err) ea.w[p] = w;
           } else {
             w = ea.w[p];
@@ -241,6 +250,7 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial,
   const int p0 = threadIdx.x * per;
   int cnt = 0;
   for (int p = p0; p < p0 + per && p < PP; ++p) cnt += fresh[p];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = cnt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -283,7 +293,8 @@ plan_select_kernel(DevGeom g, const float *__restrict__ partial,
 }  // namespace plan
 
 size_t plan_workspace_bytes(const DevGeom &g) {
-  return (size_t)g.P * g.BH * weights::n_row_blocks(g.Lmax) * (g.G + 1) * sizeof(float);
+  // the block sums, then the means of the units and of the drift columns
+  return (weights::n_partials(g) + (size_t)g.P * g.G + g.P) * sizeof(float);
 }
 
 // mass_source: the block sums are already in `workspace` (written by the
@@ -307,6 +318,15 @@ cudaError_t launch_plan(const DevGeom &g, const float *cache_lse, const unsigned
     dim3 grid(weights::n_row_blocks(g.Lmax), g.P, g.BH);
     plan::mass_kernel<<<grid, weights::kWRows, smem, stream>>>(
         g, cache_lse, cache_valid, partial, do_mass, err ? drift_rows : nullptr, local_ok);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (!anchor && (do_mass || err)) {
+    // block sums -> per-unit means (and per-partition drift), in parallel
+    const int nv = g.P * g.G + (err ? g.P : 0);
+    const int blocks = (nv + plan::kReduceWarps - 1) / plan::kReduceWarps;
+    plan::mass_reduce_kernel<<<blocks, plan::kReduceWarps * 32, 0, stream>>>(
+        g, partial, partial + weights::n_partials(g), do_mass, err ? 1 : 0, local_ok);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

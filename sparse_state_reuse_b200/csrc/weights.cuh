@@ -84,6 +84,10 @@ __host__ __device__ inline int n_row_blocks(int Lmax) { return (Lmax + kWRows - 
 __host__ __device__ inline size_t partial_index(const DevGeom &g, int i, int bh, int rb, int col) {
   return (((size_t)i * g.BH + bh) * n_row_blocks(g.Lmax) + rb) * (size_t)(g.G + 1) + col;
 }
+// Floats of the block sums (the mass partials a merge writes).
+__host__ __device__ inline size_t n_partials(const DevGeom &g) {
+  return (size_t)g.P * g.BH * n_row_blocks(g.Lmax) * (size_t)(g.G + 1);
+}
 
 }  // namespace weights
 }  // namespace ditango

@@ -86,7 +86,7 @@ int main(void) {
     CHECK(ditango_plan_from_mass(&geo, NULL, 0, NULL, 1, 0.5, (int8_t *)fake, (int32_t *)fake,
                                  (int32_t *)fake, NULL, NULL) == DITANGO_ERR_INVALID,
           "plan from mass without partials");
-    CHECK(ditango_plan_from_mass(&geo, (const float *)fake, ditango_plan_workspace_size(&geo) - 4,
+    CHECK(ditango_plan_from_mass(&geo, (float *)fake, ditango_plan_workspace_size(&geo) - 4,
                                  NULL, 1, 0.5, (int8_t *)fake, (int32_t *)fake, (int32_t *)fake,
                                  NULL, NULL) == DITANGO_ERR_INVALID,
           "plan from mass partials that are too small");
