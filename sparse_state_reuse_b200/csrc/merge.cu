@@ -147,7 +147,7 @@ __device__ __forceinline__ void lse_weights(float l0, float l1, float &w0, float
 // Merge of one block of rows (see the file comment).  Dynamic shared memory:
 // the weights, [states][kWRows] floats.
 template <int D, bool SB>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 3)
 merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__restrict__ part_O,
              const float *__restrict__ part_lse, char *cache_O, float *cache_lse,
              unsigned char *cache_valid, int writeback, void *out, int out_is_fp32, long long osb,
@@ -155,7 +155,7 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
   constexpr int Q4 = D / 4;                 // 4-value groups per row
   constexpr int ES = SB ? 2 : 4;            // bytes per stored O element
   constexpr size_t ROWB = (size_t)D * ES;   // bytes per state row
-  constexpr int U = SB ? 8 : 4;             // groups per thread per pass
+  constexpr int U = SB ? 4 : 2;             // groups per thread per pass
   constexpr int SBATCH = 4;                 // states per batch of loads
   using weights::kWRows;
   const int i = blockIdx.y;

@@ -30,10 +30,30 @@ def test_every_declared_symbol_is_exported():
     assert set(names) == set(dt.EXPORTED)
 
 
+def test_checked_build_exports_the_same_abi():
+    """libditango_check.so (built with -DDITANGO_CHECK) exports every declared
+    symbol too, and says it is the checked build; the release library says
+    it is not.  No GPU needed: neither call touches the device."""
+    import ctypes
+    import subprocess
+    import sys
+    path = os.path.join(os.path.dirname(dt.LIB_PATH), "libditango_check.so")
+    if not os.path.exists(path):
+        subprocess.run([sys.executable, os.path.join(os.path.dirname(dt.LIB_PATH), "build.py"),
+                        "--check"], check=True, capture_output=True)
+    lib = ctypes.CDLL(path)
+    for n in declared():
+        assert hasattr(lib, n), n
+    lib.ditango_checked_build.restype = ctypes.c_int32
+    assert lib.ditango_checked_build() == 1
+    assert not dt.ditango_checked_build()
+
+
 def test_version_and_status_strings():
     assert dt.ditango_version() >= 10000
     assert dt.status_string(0) == "ok"
     assert "timed out" in dt.status_string(4)
+    assert "out of range" in dt.status_string(5)
 
 
 @pytest.mark.parametrize("w", configs.ALL, ids=lambda w: w.name)
