@@ -222,8 +222,9 @@ def run_ours(args, w, rank, world, local_rank):
     fresh = plan == 1
     flops = effective_flops(w, fresh_pairs_of_units(w, plan, pair_mask(w)))
     mbytes = merge_bytes(w, A, fresh, state_o_bytes=2 if args.state_bf16 else 4)
-    # plan (selection alone: the merge before it left the mass score), attention, merge
-    launches_per_step = 3
+    # plan (anchor: the selection alone; reuse: the mean of the mass block sums
+    # the previous merge left, then the selection), attention, merge
+    launches_per_step = (1 if w.anchor else 2) + 1 + 1
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     n_ev = args.steps
@@ -372,9 +373,9 @@ def run_ours(args, w, rank, world, local_rank):
                            "kernel_ms": round(merge_ms, 4),
                            "algorithmic_bytes_per_launch": mbytes,
                            "traffic": recorded_traffic("merge.cu", w.name)},
-        "plan": {"us": round(plan_us, 2), "launches": 1,
-                 "note": "selection alone: anchor steps need no mass score, and reuse steps take "
-                         "it from the previous step's merge (mass partials)"},
+        "plan": {"us": round(plan_us, 2), "launches": 1 if w.anchor else 2,
+                 "note": "anchor steps: the selection alone; reuse steps: the mass score from the "
+                         "previous step's merge (its block sums reduced per unit) and the selection"},
         "e2e": {"value": round(aggregate_tflops(world, flops, e2e_ms), 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

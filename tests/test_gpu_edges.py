@@ -131,3 +131,61 @@ def test_mismatched_tensors_are_refused_before_any_launch():
         pa.merge(out.half())
     torch.cuda.synchronize()
     assert pa.status.item() == 0
+
+
+@pytest.mark.parametrize("band_k,budget", [(0, 0.0), (0, 1.0), (3, 0.0), (0, 0.3125)],
+                         ids=["diagonal_only", "budget_all", "band_covers_all", "one_unit_by_mass"])
+def test_degenerate_budgets_and_bands(band_k, budget):
+    """Budget 0 (only the band is recomputed), budget 1 (everything is), a
+    band covering every pair, and a budget one unit above the band: the
+    plan equals the oracle's selection on its own fp64 scores of the GPU's
+    cache, and the output equals the oracle's composition of that plan."""
+    from oracle.plan import mass_scores, select, budget_target
+    w = configs.TINY
+    Q, K, V = G.upload(w)
+    Kp, Vp = G.upload_prev(w)
+    pa = dt.PartitionedAttention(w.B, w.H, w.N, w.d, w.part_off())
+    pa.plan_step(anchor=True)
+    pa.partial(Q, Kp, Vp)
+    torch.cuda.synchronize()
+    lse = pa.state_lse.cpu().numpy()
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    pa.step(Q, K, V, out, band_k=band_k, budget=budget)
+    torch.cuda.synchronize()
+    assert pa.status.item() == 0
+    A = OM.pair_mask(w.part_off())
+    plan = pa.plan.cpu().numpy().reshape(w.P, w.P)
+    score = pa.score.cpu().numpy().reshape(w.P, w.P)
+    plan_s, _ = select(score.astype(np.float64), A, band_k, budget)     # the selection rule, exactly
+    assert (plan == plan_s).all(), (plan, plan_s)
+    w_o = mass_scores(lse, A, w.part_off())
+    np.testing.assert_allclose(score, w_o, rtol=1e-5, atol=1e-9)
+    plan_o, _ = select(w_o, A, band_k, budget)                            # and on fp64 scores
+    for i, j in zip(*np.nonzero(plan_o != plan)):                          # only ties at the cut
+        cut = w_o[(plan_o == 1) & (np.abs(np.subtract.outer(np.arange(w.P), np.arange(w.P))) > band_k)].min()
+        assert abs(w_o[i, j] - cut) <= 1e-5 * cut
+    n_band = int((np.abs(np.subtract.outer(np.arange(w.P), np.arange(w.P))) <= band_k).sum())
+    assert int(pa.counts[0]) == budget_target(n_band, w.P * w.P, budget)
+    o = out.cpu().numpy()
+    for h in range(w.H):
+        for i in range(w.P):
+            rows = np.arange(w.part_off()[i], w.part_off()[i + 1])
+            Oo, _, _ = G.oracle_rows(w, plan, 0, h, i, rows)
+            G.assert_close(o[0, h, rows], Oo, f"out h {h} part {i}")
+
+
+def test_many_heads_short_sequence():
+    """B*H = 3000 slabs of 320 tokens in 3 ragged partitions: thousands of
+    small work items and a merge grid of 3000 (b, h) blocks deep."""
+    po = [0, 100, 130, 320]
+    w = configs.scaled(configs.TINY, N=320, d=64, B=3, H=1000, P=1, seed=909, name="many_heads")
+    geom_po = po
+    Au, fresh, O, lse, out, out_lse = all_fresh_states(w, geom_po)
+    assert len(fresh) == 9
+    for bh in (0, 1, 1499, 2998, 2999):
+        b, h = divmod(bh, w.H)
+        q, k, v, _, _ = G.slabs(w, b, h, with_prev=False)
+        from oracle.attention import dense_attention
+        Od, ld = dense_attention(q, k, v)
+        G.assert_close(out[b, h], Od, f"merged output bh {bh}")
+        G.assert_close(out_lse[b, h], ld, f"merged lse bh {bh}")
