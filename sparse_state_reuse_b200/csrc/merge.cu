@@ -28,31 +28,10 @@ namespace merge {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kRowsPerBlock = 128;
-constexpr int kBatch = 4;    // O vectors per row in flight per lane
 
 // Checked builds record a bad plan code here; read and cleared by
 // ditango_check_status.
 __device__ int g_merge_check_status;
-
-struct Src {
-  const char *O;     // [Lmax][d] block of this (index, b*h): float32, or bf16 (SB)
-  const float *lse;  // [Lmax]
-  char *wbO;         // cache block to write back into, or null
-  float *wblse;
-};
-
-// Four consecutive O values of a state row (float32, or bf16 when SB).
-template <bool SB>
-__device__ __forceinline__ float4 load_o4(const char *p) {
-  if constexpr (SB) {
-    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
-    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
-                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
-  } else {
-    return __ldg(reinterpret_cast<const float4 *>(p));
-  }
-}
 
 // Raw form of four stored O values (kept packed until used).
 template <bool SB>
@@ -93,19 +72,6 @@ __device__ __forceinline__ void store_raw4(char *p, typename Raw4<SB>::T u) {
     *reinterpret_cast<float4 *>(p) = u;
 }
 
-// Store four values that came from load_o4 (exact in either format).
-template <bool SB>
-__device__ __forceinline__ void store_o4(char *p, float4 v) {
-  if constexpr (SB) {
-    uint2 u;
-    u.x = (__float_as_uint(v.x) >> 16) | (__float_as_uint(v.y) & 0xffff0000u);
-    u.y = (__float_as_uint(v.z) >> 16) | (__float_as_uint(v.w) & 0xffff0000u);
-    *reinterpret_cast<uint2 *>(p) = u;
-  } else {
-    *reinterpret_cast<float4 *>(p) = v;
-  }
-}
-
 __device__ __forceinline__ void store_out(void *out, int is_fp32, size_t off, float4 v) {
   if (is_fp32) {
     *reinterpret_cast<float4 *>(static_cast<float *>(out) + off) = v;
@@ -124,24 +90,6 @@ __device__ __forceinline__ void fma4(float4 &acc, float w, const float4 &v) {
   acc.y = fmaf(w, v.y, acc.y);
   acc.z = fmaf(w, v.z, acc.z);
   acc.w = fmaf(w, v.w, acc.w);
-}
-
-// Weights of one row: lane a holds lse of state a (l0) and a + 32 (l1);
-// returns exp(lse_a - L) for both and L = log sum_a exp(lse_a).
-__device__ __forceinline__ void lse_weights(float l0, float l1, float &w0, float &w1, float &L) {
-  float M = fmaxf(l0, l1);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const bool dead = !(M > -INFINITY);
-  const float Ms = dead ? 0.f : M;
-  const float e0 = expf(l0 - Ms), e1 = expf(l1 - Ms);
-  float S = e0 + e1;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
-  const float invS = dead ? 0.f : 1.f / S;
-  w0 = e0 * invS;
-  w1 = e1 * invS;
-  L = dead ? -INFINITY : Ms + logf(S);
 }
 
 // Merge of one block of rows (see the file comment).  Dynamic shared memory:
@@ -356,18 +304,23 @@ cache_update_kernel(DevGeom g, const signed char *__restrict__ plan,
 // (i, C) is the log-sum-exp composition of the cached states of the fine
 // units (i, c), c inside C -- no attention is recomputed.  Those fine units
 // are consecutive slots of the fine cache.  blockIdx.y = coarse slot,
-// blockIdx.z = b*h, blockIdx.x = a block of kRowsPerBlock rows; one warp
-// merges R rows at a time with d/4 lanes per row, as in the merge.  A
-// coarse slot is valid only if every fine slot it covers is; an invalid one
-// is marked and left unwritten.
+// blockIdx.z = b*h, blockIdx.x = a block of kWRows rows.  The same two
+// phases as the merge: the rows' weights (and the coarse lse) in shared
+// memory, then the fine states' rows streamed as a flat array of 4-value
+// groups into the coarse state's rows, which are contiguous too.  A coarse
+// slot is valid only if every fine slot it covers is; an invalid one is
+// marked and left unwritten.
 template <int D, bool SB>
-__global__ void __launch_bounds__(kThreads, SB ? 3 : 4)
+__global__ void __launch_bounds__(kThreads, 3)
 compose_kernel(DevGeom fine, DevGeom coarse, const char *__restrict__ fO,
                const float *__restrict__ flse, const unsigned char *__restrict__ fvalid,
                char *__restrict__ cO, float *__restrict__ clse, unsigned char *cvalid) {
-  constexpr int G4 = D / 4;                 // lanes carrying one row
+  constexpr int Q4 = D / 4;                 // 4-value groups per row
   constexpr int ES = SB ? 2 : 4;
   constexpr size_t ROWB = (size_t)D * ES;
+  constexpr int U = SB ? 4 : 2;             // groups per thread per pass
+  constexpr int SBATCH = 4;                 // states per batch of loads
+  using weights::kWRows;
   const int cslot = blockIdx.y;
   const int bh = blockIdx.z;
   int i = 0;
@@ -376,8 +329,9 @@ compose_kernel(DevGeom fine, DevGeom coarse, const char *__restrict__ fO,
   for (int t = cslot - coarse.row_start[i]; t > 0; --t) m &= m - 1;
   const int C = __ffsll((long long)m) - 1;
   const int Li = coarse.part_off[i + 1] - coarse.part_off[i];
-  const int r0 = blockIdx.x * kRowsPerBlock;
+  const int r0 = blockIdx.x * kWRows;
   if (r0 >= Li) return;
+  const int nrows = (Li - r0 < kWRows) ? Li - r0 : kWRows;
   // the fine units inside C that are active: consecutive fine slots
   int fs0 = -1, nf = 0;
   for (int c = 0; c < fine.G; ++c) {
@@ -392,56 +346,62 @@ compose_kernel(DevGeom fine, DevGeom coarse, const char *__restrict__ fO,
   if (cvalid && bh == 0 && blockIdx.x == 0) cvalid[cslot] = valid ? 1 : 0;
   if (!valid) return;   // uniform per block
 
+  extern __shared__ float sh[];             // weights [nf][kWRows]
+  __shared__ const char *s_O[kMaxP];
+  __shared__ const float *s_lse[kMaxP];
   const size_t blk = (size_t)fine.BH * fine.Lmax;
-  const size_t base = (size_t)bh * fine.Lmax;
-  const char *srcO = fO + ((size_t)fs0 * blk + base) * ROWB;   // fine slot a: + a * blk * ROWB
-  const float *srcl = flse + (size_t)fs0 * blk + base;
-  char *dstO = cO + ((size_t)cslot * blk + base) * ROWB;
-  float *dstl = clse + (size_t)cslot * blk + base;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rend = (r0 + kRowsPerBlock < Li) ? r0 + kRowsPerBlock : Li;
-  const bool act = lane < G4;
-  constexpr int R = SB ? 4 : 2;
-  for (int r = r0 + R * warp; r < rend; r += R * kWarps) {
-    float l0[R], l1[R];
+  const size_t row0 = (size_t)bh * fine.Lmax + r0;   // this block's first row in a state block
+  if (threadIdx.x < nf) {
+    s_O[threadIdx.x] = fO + ((size_t)(fs0 + threadIdx.x) * blk + row0) * ROWB;
+    s_lse[threadIdx.x] = flse + (size_t)(fs0 + threadIdx.x) * blk + row0;
+  }
+  __syncthreads();
+  char *dstO = cO + ((size_t)cslot * blk + row0) * ROWB;
+  float *dstl = clse + (size_t)cslot * blk + row0;
+
+  // ---- phase 1: weights and the coarse lse of every row
+  if (threadIdx.x < kWRows) {
+    const int t = threadIdx.x;
+    const float L = weights::row_shares(s_lse, nf, t, t < nrows, sh, t);
+    if (t < nrows) dstl[t] = L;
+  }
+  __syncthreads();
+
+  // ---- phase 2: the fine rows, weighted, into the coarse rows
+  const int n4 = nrows * Q4;
+  for (int f0 = threadIdx.x; f0 < n4; f0 += kThreads * U) {
+    float4 acc[U];
+    int row[U];
 #pragma unroll
-    for (int q = 0; q < R; ++q) {
-      const bool ok = (r + q) < rend;
-      l0[q] = (ok && lane < nf) ? __ldg(srcl + (size_t)lane * blk + r + q) : -INFINITY;
-      l1[q] = (ok && lane + 32 < nf) ? __ldg(srcl + (size_t)(lane + 32) * blk + r + q) : -INFINITY;
+    for (int u = 0; u < U; ++u) {
+      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      row[u] = (f0 + u * kThreads) / Q4;
     }
-    typename Raw4<SB>::T v[R][kBatch];
-    float w0[R], w1[R], L[R];
-    float4 acc[R];
+    for (int a0 = 0; a0 < nf; a0 += SBATCH) {
+      typename Raw4<SB>::T v[SBATCH][U];
 #pragma unroll
-    for (int q = 0; q < R; ++q) {
-      lse_weights(l0[q], l1[q], w0[q], w1[q], L[q]);
-      acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    for (int a0 = 0; a0 < nf; a0 += kBatch) {
+      for (int q = 0; q < SBATCH; ++q) {
+        const char *src = (a0 + q < nf) ? s_O[a0 + q] : nullptr;
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u)
-#pragma unroll
-        for (int q = 0; q < R; ++q) {
+        for (int u = 0; u < U; ++u) {
+          const int f = f0 + u * kThreads;
           v[q][u] = zero_raw4<SB>();
-          if (act && a0 + u < nf && (r + q) < rend)
-            v[q][u] = load_raw4<SB>(srcO + ((size_t)(a0 + u) * blk + r + q) * ROWB + lane * 4 * ES);
+          if (src != nullptr && f < n4) v[q][u] = load_raw4<SB>(src + (size_t)f * 4 * ES);
         }
+      }
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int a = a0 + u;
+      for (int q = 0; q < SBATCH; ++q) {
+        if (a0 + q >= nf) break;
+        const float *wq = sh + (a0 + q) * kWRows;
 #pragma unroll
-        for (int q = 0; q < R; ++q) {
-          const float wq = __shfl_sync(0xffffffffu, (a < 32) ? w0[q] : w1[q], a & 31);
-          if (a < nf) fma4(acc[q], wq, widen4<SB>(v[q][u]));
-        }
+        for (int u = 0; u < U; ++u)
+          if (f0 + u * kThreads < n4) fma4(acc[u], wq[row[u]], widen4<SB>(v[q][u]));
       }
     }
 #pragma unroll
-    for (int q = 0; q < R; ++q) {
-      if ((r + q) >= rend) continue;
-      if (act) store_out(dstO, SB ? 0 : 1, (size_t)(r + q) * D + lane * 4, acc[q]);
-      if (lane == 0) dstl[r + q] = L[q];
+    for (int u = 0; u < U; ++u) {
+      const int f = f0 + u * kThreads;
+      if (f < n4) store_out(dstO, SB ? 0 : 1, (size_t)f * 4, acc[u]);
     }
   }
 }
@@ -506,17 +466,27 @@ cudaError_t launch_cache_compose(const DevGeom &fine, const DevGeom &coarse, con
                                  void *coarse_O, float *coarse_lse, unsigned char *coarse_valid,
                                  int state_bf16, cudaStream_t stream) {
   if (coarse.n_active == 0) return cudaSuccess;
-  dim3 grid((coarse.Lmax + merge::kRowsPerBlock - 1) / merge::kRowsPerBlock, coarse.n_active,
-            coarse.BH);
+  dim3 grid(weights::n_row_blocks(coarse.Lmax), coarse.n_active, coarse.BH);
+  int most = 1;   // most fine units one coarse unit covers
+  for (int i = 0; i < coarse.P; ++i)
+    for (int C = 0; C < coarse.G; ++C) {
+      int n = 0;
+      for (int c = 0; c < fine.G; ++c)
+        if (fine.group_off[c] >= coarse.group_off[C] && fine.group_off[c + 1] <= coarse.group_off[C + 1] &&
+            ((fine.row_mask[i] >> c) & 1ull))
+          ++n;
+      most = n > most ? n : most;
+    }
+  const size_t smem = (size_t)most * weights::kWRows * sizeof(float);
   switch (coarse.d) {
 #define DITANGO_COMPOSE(DD)                                                                      \
   case DD:                                                                                       \
     if (state_bf16)                                                                              \
-      merge::compose_kernel<DD, true><<<grid, merge::kThreads, 0, stream>>>(                     \
+      merge::compose_kernel<DD, true><<<grid, merge::kThreads, smem, stream>>>(                  \
           fine, coarse, static_cast<const char *>(fine_O), fine_lse, fine_valid,                 \
           static_cast<char *>(coarse_O), coarse_lse, coarse_valid);                              \
     else                                                                                         \
-      merge::compose_kernel<DD, false><<<grid, merge::kThreads, 0, stream>>>(                    \
+      merge::compose_kernel<DD, false><<<grid, merge::kThreads, smem, stream>>>(                 \
           fine, coarse, static_cast<const char *>(fine_O), fine_lse, fine_valid,                 \
           static_cast<char *>(coarse_O), coarse_lse, coarse_valid);                              \
     return cudaGetLastError();
