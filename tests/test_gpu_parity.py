@@ -328,3 +328,35 @@ def test_step_captured_in_a_cuda_graph_replays_bit_identically():
         assert pa.status.item() == 0
         assert torch.equal(pa.plan, ref_plan)
         assert torch.equal(out, ref_out) and torch.equal(out_lse, ref_lse)
+
+
+@pytest.mark.parametrize("w", [configs.TINY, configs.scaled(configs.FRAME_TILE, H=3, name="frame_tile_h3"),
+                               configs.scaled(configs.LONG_VIDEO, H=2, anchor=True, name="long_video_h2")],
+                         ids=["tiny", "frame_tile_h3", "long_video_h2"])
+def test_work_counter_gives_the_fixed_order_states_and_returns_to_zero(w):
+    """Items taken from the work counter (each CTA the next one when it is
+    ready) and items dealt in a fixed stride compute the same states bit for
+    bit -- an item's arithmetic does not depend on the CTA that runs it --
+    and every launch leaves the counter at zero for the next one."""
+    Q, K, V = G.upload(w)
+    geom = dt.Geometry(w.B, w.H, w.N, w.d, w.part_off(), w.frame_off(), w.frame_mask())
+    A = OM.pair_mask(w.part_off(), w.frame_off(), w.frame_mask())
+    n, Lmax = int(A.sum()), w.Lp
+    plan = torch.zeros(w.P * w.P, dtype=torch.int8, device="cuda")
+    fresh = torch.zeros(n, dtype=torch.int32, device="cuda")
+    counts = torch.zeros(2, dtype=torch.int32, device="cuda")
+    dt.ditango_plan(geom, None, None, 0, 1.0, True, plan, fresh, counts)
+    wc = torch.zeros(2, dtype=torch.int32, device="cuda")
+    outs = []
+    for counter in (None, wc, wc):
+        O = torch.full((n, w.BH, Lmax, w.d), float("nan"), device="cuda")
+        lse = torch.full((n, w.BH, Lmax), float("nan"), device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        dt.ditango_attn_partial(geom, Q, K, V, fresh, counts, 0.0, O, lse, 0, None, st,
+                                work_counter=counter)
+        torch.cuda.synchronize()
+        assert st.item() == 0
+        assert wc.tolist() == [0, 0]
+        outs.append((O, lse))
+    for O, lse in outs[1:]:
+        assert torch.equal(O, outs[0][0]) and torch.equal(lse, outs[0][1])
