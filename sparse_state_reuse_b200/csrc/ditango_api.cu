@@ -533,7 +533,7 @@ ditango_status ditango_selftest_bounded_wait(int64_t limit_ns, int32_t *dev_stat
 // memory arena owned by someone else, a serving process whose allocator is
 // frozen after start-up, or a host that must never call cudaMalloc between
 // denoising steps.  They still pass their own inputs and outputs, but the
-// plan's scratch (the per-chunk mass sums) lives here, in a fixed device
+// plan's scratch (the mass block sums and their means) lives here, in a fixed device
 // array of this library of kNoAllocPlanScratchBytes.  Every GPU that loads
 // the library holds that array until the process exits (or until its context
 // is destroyed).
