@@ -753,10 +753,14 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int q = 0; q < 8; ++q)
           m8[q] = max3(__uint_as_float(sv[q]), __uint_as_float(sv[q + 8]), __uint_as_float(sv[q + 16]));
 #pragma unroll
-        for (int c = 24; c < BN; c += 16)
+        for (int c = 24; c + 16 <= BN; c += 16)
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             m8[q] = max3(m8[q], __uint_as_float(sv[c + q]), __uint_as_float(sv[c + q + 8]));
+        static_assert(BN % 16 == 0 && BN >= 32, "key tile: a multiple of 16 columns");
+#pragma unroll
+        for (int q = 0; q < 8; ++q)   // the last 8 columns (BN - 24 is 8 more than a multiple of 16)
+          m8[q] = fmaxf(m8[q], __uint_as_float(sv[BN - 8 + q]));
         const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
         const float mx2 = mx * sl2;
         if (t == 0) {
