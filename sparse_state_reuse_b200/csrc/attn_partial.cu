@@ -6,7 +6,8 @@
 // "Calcolo dello Stato di Gruppo"): for up to 256 query rows of partition i
 // and all keys of the active partitions of KV group c of one (b, h), the
 // state O = softmax(Q K^T * scale) V (normalised) and
-// lse = log sum exp(Q K^T * scale), by an online softmax over 128-key tiles.
+// lse = log sum exp(Q K^T * scale), by an online softmax over key tiles
+// (96 keys at d = 96, else 128).
 // Without KV groups a group is one partition and a unit is a pair (i, j).
 // A group's active partitions are walked as runs of adjacent partitions,
 // each run one contiguous key range whose last tile is masked at its end.
@@ -15,20 +16,28 @@
 //   warps 0-3  softmax warpgroup 0: rows   0..127 of the unit (Q tile 0)
 //   warps 4-7  softmax warpgroup 1: rows 128..255 of the unit (Q tile 1)
 //   warp  8    TMA producer (Q tiles, then a 2-stage K ring and V ring)
-//   warp  9    TMEM owner and MMA issuer (one thread)
-//   warps 10-11 idle
+//   warp  9    TMEM owner and MMA issuer (one thread); d = 64 and 96: the
+//              MMA issuer of Q tile 0
+//   warp  10   d = 64 and 96: the MMA issuer of Q tile 1; else idle
+//   warp  11   idle
 // Registers are rebalanced with setmaxnreg: the softmax warpgroups, which
-// hold a whole 128-column S row per thread, get kSoftmaxRegs; warpgroup 2
-// drops to kControlRegs.  2 * 128 * 216 + 128 * 72 = 384 * 168, the
-// registers the CTA is launched with; the launcher refuses to launch a build
-// whose register count differs (an unbalanced split would block forever).
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [384,384+d).
-// The bf16 probabilities P_k overwrite the first 64 columns of S_k and feed
-// the P V product straight from TMEM.  The two Q tiles ping-pong: while one
+// hold a whole S row per thread, get kSoftmaxRegs; warpgroup 2 drops to
+// kControlRegs.  2 * 128 * 216 + 128 * 72 = 384 * 168, the registers the
+// CTA is launched with; the launcher refuses to launch a build whose
+// register count differs (an unbalanced split would block forever).
+// One thread owns one query row (TMEM lane), so row max and row sum need no
+// cross-thread reduction.  O is rescaled only when a row's running maximum
+// grows by more than 2^8 (exact: O and l share the stale maximum).
+// d = 128: TMEM S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); the bf16
+// probabilities P_k overwrite the first 64 columns of S_k and feed the P V
+// product straight from TMEM.  The two Q tiles ping-pong: while one
 // warpgroup exponentiates its S tile, the tensor pipe runs the other tile's
-// P V and next Q K^T.  One thread owns one query row, so row max and row sum
-// need no cross-thread reduction.  O is rescaled only when a row's running
-// maximum grows by more than 2^8 (exact: O and l share the stale maximum).
+// P V and next Q K^T (which waits for that P V, since P lives in S).
+// d = 64 and 96 ("free S"): P_k has TMEM columns of its own (Cfg::P_COL),
+// so each softmax warp signals s_free as soon as S is in its registers and
+// the next Q K^T runs under its exponentials; before writing P again it
+// waits on p_free (the P V that read the previous P is done).  Each Q tile
+// has its own MMA warp, so neither tile waits for the other's events.
 // Work items go from the producer warp to the other roles through a 2-slot
 // ring in shared memory; with a work counter each CTA takes the next item
 // when it is ready for it (balanced whatever the items' sizes), otherwise
@@ -46,7 +55,6 @@ namespace ditango {
 namespace attn {
 
 constexpr int BM = 128;            // query rows per tile
-constexpr int BN = 128;            // keys per tile
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;   // 65536 / 384, rounded down to a multiple of 8
 constexpr int kSoftmaxRegs = 216;
@@ -56,22 +64,52 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kThreads * kLaunchR
 constexpr int kStages = 2;         // K ring and V ring depth
 constexpr float kRescaleLog2 = 8.0f;
 
+// Key tile and TMEM plan per head dimension.
+//   d = 128: 128-key tiles; S_k [128k, 128k+128), O_k [256+128k, ...); the
+//     bf16 P_k overwrites the first 64 columns of S_k, so the next Q K^T of
+//     tile k waits for its P V.
+//   d = 64 and 96 (FS, "free S"): P_k has columns of its own, so the next
+//     Q K^T of tile k is issued as soon as S_k is in the softmax registers and
+//     runs under the exponentials.  d = 96 takes 96-key tiles to fit:
+//     S0 [0,96) P0 [96,144) S1 [160,256) P1 [256,304) O0 [320,416) O1 [416,512);
+//     d = 64, 128-key tiles: S0 [0,128) P0 [128,192) S1 [192,320) P1 [320,384)
+//     O0 [384,448) O1 [448,512).  Every region starts on a multiple of 32.
 template <int D>
 struct Cfg {
+  static constexpr bool FS = (D != 128);
+  static constexpr int BN = (D == 96) ? 96 : 128;    // keys per tile
   static constexpr int NCH = (D + 63) / 64;          // 64-column chunks
-  static constexpr int CHUNK = BM * 128;             // bytes of one 128 x 64 bf16 chunk
-  static constexpr int TILE = NCH * CHUNK;
+  static constexpr int QCHUNK = BM * 128;            // bytes of one 128-row x 64-column bf16 chunk
+  static constexpr int KCHUNK = BN * 128;            // bytes of one BN-row chunk
+  static constexpr int QTILE = NCH * QCHUNK;
+  static constexpr int KTILE = NCH * KCHUNK;
   static constexpr int OFF_Q = 0;                    // Q0, Q1
-  static constexpr int OFF_K = 2 * TILE;
-  static constexpr int OFF_V = OFF_K + kStages * TILE;
-  static constexpr int OFF_EPI = OFF_V + kStages * TILE;     // 8 warps x 32 rows x 128 B
+  static constexpr int OFF_K = 2 * QTILE;
+  static constexpr int OFF_V = OFF_K + kStages * KTILE;
+  static constexpr int OFF_EPI = OFF_V + kStages * KTILE;     // 8 warps x 32 rows x 128 B
   static constexpr int EPI_BYTES = 8 * 32 * 128;
   static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
   static constexpr int BAR_BYTES = 256;
   static constexpr int USED = OFF_BAR + BAR_BYTES;
   // >= 116 KB keeps one CTA per SM (each CTA allocates all 512 TMEM columns).
   static constexpr int SMEM = (USED + 1024 > 120 * 1024 ? USED + 1024 : 120 * 1024);
+  // TMEM columns of S_k, P_k and O_k
+  __host__ __device__ static constexpr int S_COL(int k) { return !FS ? 128 * k : (D == 96 ? 160 * k : 192 * k); }
+  __host__ __device__ static constexpr int P_COL(int k) { return !FS ? 128 * k : S_COL(k) + BN; }
+  __host__ __device__ static constexpr int O_COL(int k) { return !FS ? 256 + 128 * k : (D == 96 ? 320 + 96 * k : 384 + 64 * k); }
+  static_assert(KCHUNK % 1024 == 0, "128B-swizzled tiles start on 1024-byte boundaries");
 };
+template <int D>
+constexpr bool tmem_plan_ok() {
+  using C = Cfg<D>;
+  return C::O_COL(1) + D <= 512 && C::O_COL(0) + D <= C::O_COL(1) &&
+         (C::FS ? (C::S_COL(0) + C::BN <= C::P_COL(0) && C::P_COL(0) + C::BN / 2 <= C::S_COL(1) &&
+                   C::S_COL(1) + C::BN <= C::P_COL(1) && C::P_COL(1) + C::BN / 2 <= C::O_COL(0))
+                : (C::S_COL(1) + C::BN <= C::O_COL(0))) &&
+         C::S_COL(1) % 32 == 0 && C::P_COL(0) % 32 == 0 && C::P_COL(1) % 32 == 0 &&
+         C::O_COL(0) % 32 == 0 && C::O_COL(1) % 32 == 0;
+}
+static_assert(tmem_plan_ok<64>() && tmem_plan_ok<96>() && tmem_plan_ok<128>(), "TMEM plan");
 
 struct Params {
   DevGeom g;
@@ -129,6 +167,7 @@ __device__ __forceinline__ void first_run(const DevGeom &g, unsigned long long b
 // Key tiles of unit (i, c) in order: tile t of the current run.  Only the
 // end of the current run is held; the next run is found again from the
 // geometry (kernel parameters), which keeps the softmax warps' registers.
+template <int BN>
 struct KeyCursor {
   int k0, Lk, t, jend;
   __device__ __forceinline__ void start(const DevGeom &g, int i, int c) {
@@ -182,7 +221,7 @@ __device__ __forceinline__ Item decode_item(const Params &p, const int *row_fres
 // frame mask may forbid single token pairs inside an active pair (partitions
 // that straddle frames); otherwise every unit is one key range attended by
 // all its rows.
-template <bool MR>
+template <bool MR, int BN>
 __device__ __forceinline__ UnitRange unit_at(const Params &p, int i, int f) {
   UnitRange u;
   const int unit = __ldg(p.fresh_list + f);
@@ -309,6 +348,7 @@ __device__ __forceinline__ int frame_of(const DevGeom &g, int tok) {
 // Token-level frame mask (Efficient-vDiT's frame tiles, with partitions that
 // straddle frames): in the key tile starting at token k0 (valid keys), the
 // logits of keys whose frame this row may not attend become -inf.
+template <int BN>
 __device__ __forceinline__ void mask_frames(const DevGeom &g, int k0, int valid,
                                             unsigned long long allow, uint32_t (&sv)[BN]) {
   for (int f = frame_of(g, k0); f < g.F && g.frame_off[f] < k0 + valid; ++f) {
@@ -328,6 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params p) {
   using C = Cfg<D>;
+  constexpr int BN = C::BN;
+  constexpr bool FS = C::FS;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128B-swizzled operand tiles
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -352,6 +394,9 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   auto item_full = [&](int s) { return bar + 152 + 8 * s; };
   auto item_empty = [&](int s) { return bar + 168 + 8 * s; };
   volatile int *item_slot = reinterpret_cast<volatile int *>(smem + C::OFF_BAR + 208);
+  // FS: S_k read into registers (the next Q K^T may overwrite it) / P_k V done
+  auto s_free = [&](int k) { return bar + 216 + 8 * k; };
+  auto p_free = [&](int k) { return bar + 232 + 8 * k; };
 
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + 192);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_BAR + 200);
@@ -407,24 +452,27 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     for (int i = 1; i <= p.g.P; ++i) row_fresh[i] += row_fresh[i - 1];
 
   if (threadIdx.x == 0) {
+    // FS: each of the two MMA warps releases every Q, K and V stage once
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    mbar_init(q_empty, FS ? 2 : 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(k_full(s), 1);
-      mbar_init(k_empty(s), 1);
+      mbar_init(k_empty(s), FS ? 2 : 1);
       mbar_init(v_full(s), 1);
-      mbar_init(v_empty(s), 1);
+      mbar_init(v_empty(s), FS ? 2 : 1);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(s_full(k), 1);
       mbar_init(p_full(k), 4);    // one arrival per softmax warp
       mbar_init(o_full(k), 1);
       mbar_init(o_empty(k), 4);
+      mbar_init(s_free(k), 4);    // one arrival per softmax warp
+      mbar_init(p_free(k), 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, FS ? 2 : 1);   // one commit per MMA warp
     for (int s = 0; s < 2; ++s) {
       mbar_init(item_full(s), 1);
-      mbar_init(item_empty(s), 9);   // the MMA warp and the eight softmax warps
+      mbar_init(item_empty(s), FS ? 10 : 9);   // the MMA warp(s) and the eight softmax warps
     }
 
     *abort_flag = 0;
@@ -490,19 +538,19 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         ++ic;
         if (it < 0) break;
         if (!(ok = wait_warp(q_empty, (uc & 1) ^ 1, ctl))) break;
-        const uint32_t qbytes = C::TILE * (w.rows1 > 0 ? 2 : 1);
+        const uint32_t qbytes = C::QTILE * (w.rows1 > 0 ? 2 : 1);
         if (leader) mbar_arrive_expect_tx(q_full, qbytes);
         q_armed = uc & 1;
         if (leader) {
           for (int c = 0; c < C::NCH; ++c)
-            tma_load_4d(sQ + c * C::CHUNK, &tmQ, q_full, c * 64, w.q0, w.h, w.b);
+            tma_load_4d(sQ + c * C::QCHUNK, &tmQ, q_full, c * 64, w.q0, w.h, w.b);
           if (w.rows1 > 0)
             for (int c = 0; c < C::NCH; ++c)
-              tma_load_4d(sQ + C::TILE + c * C::CHUNK, &tmQ, q_full, c * 64, w.q0 + BM, w.h, w.b);
+              tma_load_4d(sQ + C::QTILE + c * C::QCHUNK, &tmQ, q_full, c * 64, w.q0 + BM, w.h, w.b);
         }
         for (int f = w.f0; f < w.f1 && ok; ++f) {
-          const UnitRange pr = unit_at<MR>(p, w.i, f);
-          KeyCursor cur;
+          const UnitRange pr = unit_at<MR, BN>(p, w.i, f);
+          KeyCursor<BN> cur;
           if constexpr (MR) cur.start(p.g, w.i, pr.c);
           for (int t = 0; t < pr.T && ok; ++t) {
             if constexpr (MR) {
@@ -511,19 +559,19 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const int row = MR ? cur.row() : pr.k0 + t * BN;
             int s = kc % kStages;
             if (!(ok = wait_warp(k_empty(s), ((kc / kStages) & 1) ^ 1, ctl))) break;
-            if (leader) mbar_arrive_expect_tx(k_full(s), C::TILE);
+            if (leader) mbar_arrive_expect_tx(k_full(s), C::KTILE);
             k_armed = (k_armed & ~(3u << (2 * s))) | ((1u | (((kc / kStages) & 1u) << 1)) << (2 * s));
             if (leader)
               for (int c = 0; c < C::NCH; ++c)
-                tma_load_4d(sK + s * C::TILE + c * C::CHUNK, &tmK, k_full(s), c * 64, row, w.h, w.b);
+                tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tmK, k_full(s), c * 64, row, w.h, w.b);
             ++kc;
             s = vc % kStages;
             if (!(ok = wait_warp(v_empty(s), ((vc / kStages) & 1) ^ 1, ctl))) break;
-            if (leader) mbar_arrive_expect_tx(v_full(s), C::TILE);
+            if (leader) mbar_arrive_expect_tx(v_full(s), C::KTILE);
             v_armed = (v_armed & ~(3u << (2 * s))) | ((1u | (((vc / kStages) & 1u) << 1)) << (2 * s));
             if (leader)
               for (int c = 0; c < C::NCH; ++c)
-                tma_load_4d(sV + s * C::TILE + c * C::CHUNK, &tmV, v_full(s), c * 64, row, w.h, w.b);
+                tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tmV, v_full(s), c * 64, row, w.h, w.b);
             ++vc;
           }
         }
@@ -547,7 +595,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 9 || (FS && warp == 10)) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs the loop (warp-uniform control flow keeps the
     // descriptors in uniform registers); one elected lane issues every MMA
@@ -563,106 +611,192 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       // to the start-address field (all addresses stay below 256 KB, so the
       // 14-bit field never carries).
       const uint64_t dQ0 = smem_desc_sw128(sQ, 16, 1024);
-      const uint64_t dQ1 = smem_desc_sw128(sQ + C::TILE, 16, 1024);
+      const uint64_t dQ1 = smem_desc_sw128(sQ + C::QTILE, 16, 1024);
       const uint64_t dK0 = smem_desc_sw128(sK, 16, 1024);
-      const uint64_t dK1 = smem_desc_sw128(sK + C::TILE, 16, 1024);
-      const uint64_t dV0 = smem_desc_sw128(sV, C::CHUNK, 1024);
-      const uint64_t dV1 = smem_desc_sw128(sV + C::TILE, C::CHUNK, 1024);
+      const uint64_t dK1 = smem_desc_sw128(sK + C::KTILE, 16, 1024);
+      // V: MN-major; the leading offset steps from one 64-column chunk of d
+      // to the next (BN rows of 128 bytes each)
+      const uint64_t dV0 = smem_desc_sw128(sV, C::KCHUNK, 1024);
+      const uint64_t dV1 = smem_desc_sw128(sV + C::KTILE, C::KCHUNK, 1024);
       static_assert(kStages == 2, "descriptor selection assumes two stages");
       auto qk = [&](int k, int ks) {
         // S_k = Q_k K^T : K-major A and B, 16 columns of d per instruction
         const uint64_t a0 = k ? dQ1 : dQ0;
         const uint64_t b0 = ks ? dK1 : dK0;
-        const uint32_t d_tmem = tmem + k * 128;
+        const uint32_t d_tmem = tmem + C::S_COL(k);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
-          if (leader) mma_ss(d_tmem, a0 + off, b0 + off, idesc_qk, kk > 0);
+          const uint64_t offa = (uint64_t)(((kk >> 2) * C::QCHUNK + (kk & 3) * 32) >> 4);
+          const uint64_t offb = (uint64_t)(((kk >> 2) * C::KCHUNK + (kk & 3) * 32) >> 4);
+          if (leader) mma_ss(d_tmem, a0 + offa, b0 + offb, idesc_qk, kk > 0);
         }
       };
       auto pv = [&](int k, int vs, bool acc) {
         // O_k (+)= P_k V : P from TMEM (K-major), V MN-major (d contiguous)
         const uint64_t b0 = vs ? dV1 : dV0;
-        const uint32_t d_tmem = tmem + 256 + k * 128;
-        const uint32_t a_tmem = tmem + k * 128;
+        const uint32_t d_tmem = tmem + C::O_COL(k);
+        const uint32_t a_tmem = tmem + C::P_COL(k);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
           if (leader) mma_ts(d_tmem, a_tmem + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv, (acc || kk > 0));
       };
       uint32_t ic = 0;
-      while (ok) {
-        const int is = ic & 1;
-        if (!(ok = wait_warp(item_full(is), (ic >> 1) & 1, ctl))) break;
-        const int it = item_slot[is];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(item_empty(is));
-        ++ic;
-        if (it < 0) break;
-        const Item w = decode_item(p, row_fresh, it, nqt2);
-        const bool has1 = w.rows1 > 0;
-        if (!(ok = wait_warp(q_full, uc & 1, ctl))) break;
-        for (int f = w.f0; f < w.f1 && ok; ++f) {
-          const UnitRange pr = unit_at<MR>(p, w.i, f);
-          const bool last_pair = (f + 1 == w.f1);
-          int ks = kc % kStages;
-          if (!(ok = wait_warp(k_full(ks), (kc / kStages) & 1, ctl))) break;
-          tc_fence_after();
-          qk(0, ks);
-          commit_by(leader, s_full(0));
-          if (has1) {
-            qk(1, ks);
-            commit_by(leader, s_full(1));
+      if constexpr (!FS) {
+        while (ok) {
+          const int is = ic & 1;
+          if (!(ok = wait_warp(item_full(is), (ic >> 1) & 1, ctl))) break;
+          const int it = item_slot[is];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(item_empty(is));
+          ++ic;
+          if (it < 0) break;
+          const Item w = decode_item(p, row_fresh, it, nqt2);
+          const bool has1 = w.rows1 > 0;
+          if (!(ok = wait_warp(q_full, uc & 1, ctl))) break;
+          for (int f = w.f0; f < w.f1 && ok; ++f) {
+            const UnitRange pr = unit_at<MR, BN>(p, w.i, f);
+            const bool last_pair = (f + 1 == w.f1);
+            int ks = kc % kStages;
+            if (!(ok = wait_warp(k_full(ks), (kc / kStages) & 1, ctl))) break;
+            tc_fence_after();
+            qk(0, ks);
+            commit_by(leader, s_full(0));
+            if (has1) {
+              qk(1, ks);
+              commit_by(leader, s_full(1));
+            }
+            commit_by(leader, k_empty(ks));
+            ++kc;
+            if (pr.T == 1 && last_pair) commit_by(leader, q_empty);
+            for (int t = 0; t < pr.T && ok; ++t) {
+              const int vs = vc % kStages;
+              if (!(ok = wait_warp(v_full(vs), (vc / kStages) & 1, ctl))) break;
+              const bool more = (t + 1 < pr.T);
+              // ---- Q tile 0
+              if (!(ok = wait_warp(p_full(0), pc[0] & 1, ctl))) break;
+              ++pc[0];
+              if (t == 0) {
+                if (!(ok = wait_warp(o_empty(0), (oc[0] & 1) ^ 1, ctl))) break;
+                ++oc[0];
+              }
+              tc_fence_after();
+              pv(0, vs, t > 0);
+              if (!more) commit_by(leader, o_full(0));
+              const int ks2 = kc % kStages;
+              if (more) {
+                if (!(ok = wait_warp(k_full(ks2), (kc / kStages) & 1, ctl))) break;
+                tc_fence_after();
+                qk(0, ks2);
+                commit_by(leader, s_full(0));
+              }
+              // ---- Q tile 1
+              if (has1) {
+                if (!(ok = wait_warp(p_full(1), pc[1] & 1, ctl))) break;
+                ++pc[1];
+                if (t == 0) {
+                  if (!(ok = wait_warp(o_empty(1), (oc[1] & 1) ^ 1, ctl))) break;
+                  ++oc[1];
+                }
+                tc_fence_after();
+                pv(1, vs, t > 0);
+                if (!more) commit_by(leader, o_full(1));
+                if (more) {
+                  qk(1, ks2);
+                  commit_by(leader, s_full(1));
+                }
+              }
+              commit_by(leader, v_empty(vs));
+              ++vc;
+              if (more) {
+                commit_by(leader, k_empty(ks2));
+                ++kc;
+                if (t + 2 == pr.T && last_pair) commit_by(leader, q_empty);
+              }
+            }
           }
-          commit_by(leader, k_empty(ks));
+          ++uc;
+        }
+      } else {
+        // FS: one MMA warp per Q tile (warp 9: tile 0, warp 10: tile 1), each
+        // waiting in its tile's own order, so neither tile waits for the
+        // other's events.  Units and their key tiles form one stream of steps
+        // per item; at step n the Q K^T of step n + 1 is issued as soon as the
+        // softmax has read S of step n, and the P V of step n once P is
+        // written.  Each warp releases every Q, K and V stage once (the
+        // barriers count two); for an item without a second Q tile warp 10
+        // only follows the stages and releases them.
+        const int k = warp - 9;
+        uint32_t sf = 0;             // s_free completions consumed
+        while (ok) {
+          const int is = ic & 1;
+          if (!(ok = wait_warp(item_full(is), (ic >> 1) & 1, ctl))) break;
+          const int it = item_slot[is];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(item_empty(is));
+          ++ic;
+          if (it < 0) break;
+          const Item w = decode_item(p, row_fresh, it, nqt2);
+          const bool active = (k == 0) || (w.rows1 > 0);
+          int n_steps = 0;
+          for (int f = w.f0; f < w.f1; ++f) n_steps += unit_at<MR, BN>(p, w.i, f).T;
+          if (!(ok = wait_warp(q_full, uc & 1, ctl))) break;
+          ++uc;
+          if (!active) {
+            commit_by(leader, q_empty);
+            for (int n = 0; n < n_steps && ok; ++n) {
+              if (!(ok = wait_warp(k_full(kc % kStages), (kc / kStages) & 1, ctl))) break;
+              commit_by(leader, k_empty(kc % kStages));
+              ++kc;
+              if (!(ok = wait_warp(v_full(vc % kStages), (vc / kStages) & 1, ctl))) break;
+              commit_by(leader, v_empty(vc % kStages));
+              ++vc;
+            }
+            continue;
+          }
+          // Q K^T of step 0 (S_k is free: the softmax's read of the last S
+          // of the previous item was waited for)
+          if (!(ok = wait_warp(k_full(kc % kStages), (kc / kStages) & 1, ctl))) break;
+          tc_fence_after();
+          qk(k, kc % kStages);
+          commit_by(leader, s_full(k));
+          commit_by(leader, k_empty(kc % kStages));
           ++kc;
-          if (pr.T == 1 && last_pair) commit_by(leader, q_empty);
-          for (int t = 0; t < pr.T && ok; ++t) {
-            const int vs = vc % kStages;
-            if (!(ok = wait_warp(v_full(vs), (vc / kStages) & 1, ctl))) break;
-            const bool more = (t + 1 < pr.T);
-            // ---- Q tile 0
-            if (!(ok = wait_warp(p_full(0), pc[0] & 1, ctl))) break;
-            ++pc[0];
+          if (n_steps == 1) commit_by(leader, q_empty);
+          int f = w.f0, t = 0;
+          int T = unit_at<MR, BN>(p, w.i, f).T;
+          for (int n = 0; n < n_steps && ok; ++n) {
+            if (!(ok = wait_warp(s_free(k), sf & 1, ctl))) break;
+            ++sf;
+            if (n + 1 < n_steps) {
+              if (!(ok = wait_warp(k_full(kc % kStages), (kc / kStages) & 1, ctl))) break;
+              tc_fence_after();
+              qk(k, kc % kStages);
+              commit_by(leader, s_full(k));
+              commit_by(leader, k_empty(kc % kStages));
+              ++kc;
+              if (n + 2 == n_steps) commit_by(leader, q_empty);   // the item's last Q K^T
+            }
+            if (!(ok = wait_warp(v_full(vc % kStages), (vc / kStages) & 1, ctl))) break;
+            if (!(ok = wait_warp(p_full(k), pc[k] & 1, ctl))) break;
+            ++pc[k];
             if (t == 0) {
-              if (!(ok = wait_warp(o_empty(0), (oc[0] & 1) ^ 1, ctl))) break;
-              ++oc[0];
+              if (!(ok = wait_warp(o_empty(k), (oc[k] & 1) ^ 1, ctl))) break;
+              ++oc[k];
             }
             tc_fence_after();
-            pv(0, vs, t > 0);
-            if (!more) commit_by(leader, o_full(0));
-            const int ks2 = kc % kStages;
-            if (more) {
-              if (!(ok = wait_warp(k_full(ks2), (kc / kStages) & 1, ctl))) break;
-              tc_fence_after();
-              qk(0, ks2);
-              commit_by(leader, s_full(0));
-            }
-            // ---- Q tile 1
-            if (has1) {
-              if (!(ok = wait_warp(p_full(1), pc[1] & 1, ctl))) break;
-              ++pc[1];
-              if (t == 0) {
-                if (!(ok = wait_warp(o_empty(1), (oc[1] & 1) ^ 1, ctl))) break;
-                ++oc[1];
-              }
-              tc_fence_after();
-              pv(1, vs, t > 0);
-              if (!more) commit_by(leader, o_full(1));
-              if (more) {
-                qk(1, ks2);
-                commit_by(leader, s_full(1));
-              }
-            }
-            commit_by(leader, v_empty(vs));
+            pv(k, vc % kStages, t > 0);
+            commit_by(leader, p_free(k));
+            commit_by(leader, v_empty(vc % kStages));
             ++vc;
-            if (more) {
-              commit_by(leader, k_empty(ks2));
-              ++kc;
-              if (t + 2 == pr.T && last_pair) commit_by(leader, q_empty);
+            if (t + 1 == T) {
+              commit_by(leader, o_full(k));
+              t = 0;
+              if (++f < w.f1) T = unit_at<MR, BN>(p, w.i, f).T;
+            } else {
+              ++t;
             }
           }
         }
-        ++uc;
       }
       // drain: every MMA issued so far must finish before TMEM is released
       commit_by(leader, drain);
@@ -698,10 +832,12 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const int k = warp >> 2;                 // Q tile of this warpgroup
     const int r = threadIdx.x & 127;         // row within the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + k * 128;
-    const uint32_t tO = tmem + lane_base + 256 + k * 128;
+    const uint32_t tS = tmem + lane_base + C::S_COL(k);
+    const uint32_t tP = tmem + lane_base + C::P_COL(k);   // = tS unless FS
+    const uint32_t tO = tmem + lane_base + C::O_COL(k);
     const float sl2 = p.scale_log2;
     uint32_t sc = 0, ofc = 0;
+    uint32_t pst = 0;   // FS: P tiles stored so far (each one's P V completes p_free)
     bool ok = true;
     uint32_t ic = 0;
     while (ok) {
@@ -721,8 +857,8 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (p.g.token_mask) allow = p.g.frame_allow[frame_of(p.g, w.q0 + k * BM + r)];
       }
      for (int f = w.f0; f < w.f1 && ok; ++f) {
-      const UnitRange pr = unit_at<MR>(p, w.i, f);
-      KeyCursor cur;
+      const UnitRange pr = unit_at<MR, BN>(p, w.i, f);
+      KeyCursor<BN> cur;
       if constexpr (MR) cur.start(p.g, w.i, pr.c);
       float m_used = -INFINITY;   // running maximum used for exponentiation (log2 units)
       float l = 0.f;
@@ -738,6 +874,14 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
         for (int c = 0; c < BN / 16; ++c) tmem_ld16p(tS + c * 16, &sv[c * 16]);
         tc_wait_ld();
+        bool pv_done = true;   // the previous P V of this tile has completed
+        if constexpr (FS) {
+          // S is in registers: the next Q K^T may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free(k));
+          pv_done = (pst == 0);
+        }
         const int valid = MR ? cur.valid() : pr.Lk - t * BN;
         if (valid < BN) {
 #pragma unroll
@@ -768,8 +912,16 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         } else {
           const bool need = mx2 > m_used + kRescaleLog2;
           if (__any_sync(0xffffffffu, need)) {
-            // O of this row already holds every P V of earlier tiles: the
-            // commit that released S(t) covers all earlier MMAs.
+            // O of this row must hold every P V of earlier tiles: without FS
+            // the commit that released S(t) covers all earlier MMAs; with FS
+            // the last one is waited for here.
+            if constexpr (FS) {
+              if (!pv_done) {
+                if (!(ok = wait_bounded(p_free(k), (pst - 1) & 1, ctl))) break;
+                tc_fence_after();
+                pv_done = true;
+              }
+            }
             const float m_new = need ? mx2 : m_used;
             const float alpha = need ? ex2(m_used - m_new) : 1.f;   // 1, not NaN, for a row still at -inf
             l *= alpha;
@@ -785,10 +937,18 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
           }
         }
-        // P = 2^(s*scale*log2e - m), rounded to bf16 into the first 64 S columns
+        // P = 2^(s*scale*log2e - m), rounded to bf16 into P_k (the first BN/2
+        // columns of S_k unless FS)
         // (general variant) a row with no admissible key so far exponentiates against 0
         const float neg = (MR && !(m_used > -INFINITY)) ? 0.f : -m_used;
         const uint64_t sl2x2 = f2(sl2, sl2), negx2 = f2(neg, neg);
+        if constexpr (FS) {
+          // P_k is overwritten below: the P V that read it must be done
+          if (!pv_done) {
+            if (!(ok = wait_bounded(p_free(k), (pst - 1) & 1, ctl))) break;
+            tc_fence_after();
+          }
+        }
         uint64_t lsum0 = 0, lsum1 = 0;   // packed partial row sums (+0.0f bits)
 #pragma unroll
         for (int g8 = 0; g8 < BN / 16; ++g8) {
@@ -804,7 +964,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if (e & 1) lsum1 = add2(lsum1, f2(a, b)); else lsum0 = add2(lsum0, f2(a, b));
             pk[e] = pack_bf16(a, b);
           }
-          tmem_st8(tS + g8 * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+          tmem_st8(tP + g8 * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
         }
         {
           float s0, s1, s2, s3;
@@ -816,6 +976,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full(k));   // one arrival per warp
+        ++pst;
       }
       if (!ok) break;
       // ---- epilogue: O of this row into registers, release the TMEM
@@ -988,6 +1149,11 @@ cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const C
     default:
       return cudaErrorInvalidValue;
   }
+}
+
+// Keys per K/V tile of the kernel for head dimension d (the TMA box height).
+int attn_key_tile(int d) {
+  return d == 64 ? attn::Cfg<64>::BN : (d == 96 ? attn::Cfg<96>::BN : attn::Cfg<128>::BN);
 }
 
 // Read (and optionally clear) this file's check word.

@@ -18,6 +18,7 @@ cudaError_t launch_attn_partial(const DevGeom &g, const CUtensorMap &tq, const C
                                 int state_bf16, unsigned char *out_valid, float *drift_rows,
                                 int *dev_status, long long wait_limit_ns, int num_sms,
                                 int *work_counter, cudaStream_t stream);
+int attn_key_tile(int d);
 size_t plan_workspace_bytes(const DevGeom &g);
 cudaError_t launch_plan(const DevGeom &g, const float *cache_lse, const unsigned char *cache_valid,
                         int band_k, int target, int anchor, signed char *plan_out, int *fresh_list,
@@ -398,9 +399,10 @@ ditango_status ditango_attn_partial(const ditango_geom *g, const uint16_t *Q, co
   if (!(scale >= 0.f) || !std::isfinite(scale)) return DITANGO_ERR_INVALID;
   if (scale == 0.f) scale = 1.f / std::sqrt((float)dg.d);
   CUtensorMap tq, tk, tv;
-  // Q in 128-row tiles, K and V in 128-key tiles (the kernel's BM and BN)
-  if (!make_qkv_map(&tq, Q, dg, qs, 128) || !make_qkv_map(&tk, K, dg, ks, 128) ||
-      !make_qkv_map(&tv, V, dg, vs, 128))
+  // Q in 128-row tiles, K and V in the kernel's key tiles (96 keys at d = 96, else 128)
+  const unsigned bn = (unsigned)attn_key_tile(dg.d);
+  if (!make_qkv_map(&tq, Q, dg, qs, 128) || !make_qkv_map(&tk, K, dg, ks, bn) ||
+      !make_qkv_map(&tv, V, dg, vs, bn))
     return DITANGO_ERR_CUDA;
   return cuda_status(launch_attn_partial(dg, tq, tk, tv, fresh_list, counts, scale, out_O, out_lse,
                                          out_by_slot ? 1 : 0, state_bf16 ? 1 : 0, out_valid,

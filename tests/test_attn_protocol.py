@@ -37,6 +37,15 @@ Checked on every interleaving:
     complete phase.
 Planted mistakes (a dropped wait, an early release) must be caught, so that
 a checker that passes everything would fail here.
+
+The d = 64 and d = 96 kernels ("free S", fs=True below) keep P in TMEM
+columns of its own and run one MMA warp per Q tile: each softmax warp
+arrives on s_free once S is in its registers (the next Q K^T may then
+overwrite S) and waits on p_free (the P V that read its previous P is done)
+before it writes P again; each MMA warp follows its own tile, issuing the
+next Q K^T after s_free and the P V after p_full; the Q, K and V stages and
+the drain count one release per MMA warp, and for an item without a second
+Q tile the second MMA warp only follows the stages and releases them.
 """
 import random
 
@@ -81,19 +90,23 @@ class Bar:
 CONSUMERS = 1 + 2 * WARPS_PER_TILE      # the MMA warp and the eight softmax warps
 
 
-def barriers():
-    b = {"q_full": 1, "q_empty": 1, "drain": 1}
+def barriers(fs=False):
+    releases = 2 if fs else 1                 # one per MMA warp
+    b = {"q_full": 1, "q_empty": releases, "drain": releases}
     for s in range(2):
         b[f"item_full{s}"] = 1
-        b[f"item_empty{s}"] = CONSUMERS
+        b[f"item_empty{s}"] = CONSUMERS + (1 if fs else 0)
     for s in range(STAGES):
-        for n in ("k_full", "k_empty", "v_full", "v_empty"):
-            b[f"{n}{s}"] = 1
+        b[f"k_full{s}"] = b[f"v_full{s}"] = 1
+        b[f"k_empty{s}"] = b[f"v_empty{s}"] = releases
     for k in range(2):
         b[f"s_full{k}"] = 1
         b[f"p_full{k}"] = WARPS_PER_TILE      # one arrival per softmax warp
         b[f"o_full{k}"] = 1
         b[f"o_empty{k}"] = WARPS_PER_TILE
+        if fs:
+            b[f"s_free{k}"] = WARPS_PER_TILE
+            b[f"p_free{k}"] = 1
     return {n: Bar(n, c) for n, c in b.items()}
 
 
@@ -337,13 +350,167 @@ def softmax_warp(k, items, rng, rescale_p, mut):
         yield from take(ic, mut)                  # the end marker
 
 
+def mma_fs(k, items, mut):
+    """MMA warp 9 + k of the free-S kernels: Q tile k only."""
+    kc = vc = uc = 0
+    pc = oc = sf = 0
+    ok = True
+
+    def qk(ks):
+        return ("mma", {f"Q{k}", f"K{ks}"}, {f"S{k}"})
+
+    def pv(vs, acc):
+        return ("mma", {f"P{k}", f"V{vs}"} | ({f"O{k}"} if acc else set()), {f"O{k}"})
+
+    ic = 0
+    for has1, Ts in items:
+        ok = yield from take(ic, mut)
+        ic += 1
+        if not ok:
+            break
+        n_steps = sum(Ts)
+        ok = yield W("q_full", uc & 1, uc)
+        if not ok:
+            break
+        uc += 1
+        if k == 1 and not has1:
+            # no second Q tile: follow the stages and release them
+            yield ("commit", "q_empty")
+            for _ in range(n_steps):
+                ok = yield W(f"k_full{kc % STAGES}", (kc // STAGES) & 1, kc // STAGES)
+                if not ok:
+                    break
+                if mut != "fs_idle_warp_skips_release":
+                    yield ("commit", f"k_empty{kc % STAGES}")
+                kc += 1
+                ok = yield W(f"v_full{vc % STAGES}", (vc // STAGES) & 1, vc // STAGES)
+                if not ok:
+                    break
+                yield ("commit", f"v_empty{vc % STAGES}")
+                vc += 1
+            if not ok:
+                break
+            continue
+        ok = yield W(f"k_full{kc % STAGES}", (kc // STAGES) & 1, kc // STAGES)
+        if not ok:
+            break
+        yield qk(kc % STAGES)
+        yield ("commit", f"s_full{k}")
+        yield ("commit", f"k_empty{kc % STAGES}")
+        kc += 1
+        if n_steps == 1:
+            yield ("commit", "q_empty")
+        f, t, T = 0, 0, Ts[0]
+        for n in range(n_steps):
+            if mut != "fs_mma_skips_s_free":
+                ok = yield W(f"s_free{k}", sf & 1, sf)
+                if not ok:
+                    break
+            sf += 1
+            if n + 1 < n_steps:
+                ok = yield W(f"k_full{kc % STAGES}", (kc // STAGES) & 1, kc // STAGES)
+                if not ok:
+                    break
+                yield qk(kc % STAGES)
+                yield ("commit", f"s_full{k}")
+                yield ("commit", f"k_empty{kc % STAGES}")
+                kc += 1
+                if n + 2 == n_steps:
+                    yield ("commit", "q_empty")
+            ok = yield W(f"v_full{vc % STAGES}", (vc // STAGES) & 1, vc // STAGES)
+            if not ok:
+                break
+            ok = yield W(f"p_full{k}", pc & 1, pc)
+            if not ok:
+                break
+            pc += 1
+            if t == 0:
+                ok = yield W(f"o_empty{k}", (oc & 1) ^ 1, oc - 1)
+                if not ok:
+                    break
+                oc += 1
+            yield pv(vc % STAGES, t > 0)
+            yield ("commit", f"p_free{k}")
+            yield ("commit", f"v_empty{vc % STAGES}")
+            vc += 1
+            if t + 1 == T:
+                yield ("commit", f"o_full{k}")
+                t, f = 0, f + 1
+                if f < len(Ts):
+                    T = Ts[f]
+            else:
+                t += 1
+        if not ok:
+            break
+    if ok:
+        yield from take(ic, mut)                  # the end marker
+    yield ("commit", "drain")
+    yield W("drain", 0, 0, False)
+
+
+def softmax_warp_fs(k, items, rng, rescale_p, mut):
+    sc = ofc = pst = 0
+    S, P, O = f"S{k}", f"P{k}", f"O{k}"
+    ok = True
+    ic = 0
+    for has1, Ts in items:
+        ok = yield from take(ic, mut)
+        ic += 1
+        if not ok:
+            break
+        if k == 1 and not has1:
+            continue
+        for T in Ts:
+            for t in range(T):
+                ok = yield W(f"s_full{k}", sc & 1, sc)
+                if not ok:
+                    break
+                sc += 1
+                if mut == "fs_s_free_before_s_read":
+                    yield ("arrive", f"s_free{k}")
+                yield ("hold", S, "r")                 # S into registers
+                yield ("release", S)
+                if mut != "fs_s_free_before_s_read":
+                    yield ("arrive", f"s_free{k}")
+                pv_done = pst == 0 or mut == "fs_softmax_skips_p_free"
+                if t > 0 and rng.random() < rescale_p:
+                    if not pv_done:
+                        ok = yield W(f"p_free{k}", (pst - 1) & 1, pst - 1)
+                        if not ok:
+                            break
+                        pv_done = True
+                    yield ("hold", O, "w")             # O *= alpha
+                    yield ("release", O)
+                if not pv_done:
+                    ok = yield W(f"p_free{k}", (pst - 1) & 1, pst - 1)
+                    if not ok:
+                        break
+                yield ("hold", P, "w")                 # the probabilities of this tile
+                yield ("release", P)
+                yield ("arrive", f"p_full{k}")
+                pst += 1
+            if not ok:
+                break
+            ok = yield W(f"o_full{k}", ofc & 1, ofc)
+            if not ok:
+                break
+            ofc += 1
+            yield ("hold", O, "r")
+            yield ("release", O)
+            yield ("arrive", f"o_empty{k}")
+        if not ok:
+            break
+    if ok:
+        yield from take(ic, mut)                  # the end marker
+
+
 # ---------------------------------------------------------------- scheduler
 
 def conflicts(reads_a, writes_a, reads_b, writes_b):
     return bool(writes_a & (reads_b | writes_b)) or bool(reads_a & writes_b)
 
 
-def run(items, seed, rescale_p=0.5, mut=None, timeout_p=0.0, max_steps=2_000_000):
+def run(items, seed, rescale_p=0.5, mut=None, timeout_p=0.0, max_steps=2_000_000, fs=False):
     """Interleave the roles at random; raise Violation on any broken rule.
 
     timeout_p: per scheduling step, the chance that one role blocked on an
@@ -351,15 +518,23 @@ def run(items, seed, rescale_p=0.5, mut=None, timeout_p=0.0, max_steps=2_000_000
     every role blocked on an abortable wait may give up).  Returns the
     barriers and whether the run aborted."""
     rng = random.Random(seed)
-    B = barriers()
-    roles = {"producer": producer(items, mut), "mma": mma(items, mut)}
+    B = barriers(fs)
+    roles = {"producer": producer(items, mut)}
+    if fs:
+        roles["mma0"], roles["mma1"] = mma_fs(0, items, mut), mma_fs(1, items, mut)
+    else:
+        roles["mma"] = mma(items, mut)
+    sm = softmax_warp_fs if fs else softmax_warp
     for k in range(2):
         for w in range(WARPS_PER_TILE):
-            roles[f"softmax{k}.{w}"] = softmax_warp(k, items, random.Random(rng.random()),
-                                                    rescale_p, mut)
+            roles[f"softmax{k}.{w}"] = sm(k, items, random.Random(rng.random()), rescale_p, mut)
     nxt = {r: next(g, None) for r, g in roles.items()}
     loads = []                 # in flight: (region, barrier)
-    mma_q = []                 # in issue order: ("mma", reads, writes) | ("commit", barrier)
+    # in issue order, tagged with the issuing role: ("mma", reads, writes) |
+    # ("commit", barrier).  Each role's operations complete in its issue
+    # order, those of different MMA warps in any order between them; a
+    # commit arrives once every MMA its own role issued before it is done.
+    mma_q = []
     holds = {}                 # role -> {region: mode}
     aborted = False
 
@@ -371,7 +546,7 @@ def run(items, seed, rescale_p=0.5, mut=None, timeout_p=0.0, max_steps=2_000_000
             raise Violation(f"{role}: {name} completed phase {n + 1} while it waits for phase {n}")
 
     def mma_in_flight():
-        return [op for op in mma_q if op[0] == "mma"]
+        return [op for _, op in mma_q if op[0] == "mma"]
 
     def advance(role, value=None):
         try:
@@ -380,7 +555,7 @@ def run(items, seed, rescale_p=0.5, mut=None, timeout_p=0.0, max_steps=2_000_000
             nxt[role] = None
         if all(op is None for op in nxt.values()):
             # the CTA exits (TMEM is freed): nothing of it may still be in flight
-            if mma_in_flight() or any(op[0] == "commit" for op in mma_q):
+            if mma_q:
                 raise Violation("MMAs in flight when the CTA exits")
             if loads:
                 raise Violation("loads in flight when the CTA exits")
@@ -413,7 +588,10 @@ def run(items, seed, rescale_p=0.5, mut=None, timeout_p=0.0, max_steps=2_000_000
             raise Violation(f"no role can proceed: {waiting}")
         kind, x = rng.choice(choices)
         if kind == "mma":
-            op = mma_q.pop(0)
+            issuers = sorted({r for r, _ in mma_q})
+            issuer = issuers[0] if len(issuers) == 1 else rng.choice(issuers)
+            i = next(j for j, (r, _) in enumerate(mma_q) if r == issuer)
+            _, op = mma_q.pop(i)
             if op[0] == "commit":
                 B[op[1]].arrive()
             continue
@@ -452,9 +630,9 @@ def run(items, seed, rescale_p=0.5, mut=None, timeout_p=0.0, max_steps=2_000_000
                     if conflicts(reads, writes, {region} if mode == "r" else set(),
                                  {region} if mode == "w" else set()):
                         raise Violation(f"MMA on {region} while a softmax warp holds it ({mode})")
-            mma_q.append(op)
+            mma_q.append((role, op))
         elif what == "commit":
-            mma_q.append(op)
+            mma_q.append((role, op))
         elif what == "hold":
             region, mode = op[1], op[2]
             if region.startswith("ITEM"):
@@ -625,3 +803,79 @@ def test_protocol_on_a_frame_tile_cta(cta):
         B, aborted = run(items, seed, rescale_p=0.05)
         assert not aborted
         assert B["o_full0"].phase == sum(len(Ts) for _, Ts in items)
+
+
+# ------------------------------------------------ free S (d = 64 and 96)
+
+@pytest.mark.parametrize("seed", range(60))
+def test_free_s_protocol_on_random_items_and_interleavings(seed):
+    rng = random.Random(3000 + seed)
+    items = random_items(rng)
+    B, aborted = run(items, seed, rescale_p=rng.choice([0.0, 0.3, 1.0]), fs=True)
+    assert not aborted
+    n_units = sum(len(Ts) for _, Ts in items)
+    n_tiles = sum(sum(Ts) for _, Ts in items)
+    n_units1 = sum(len(Ts) for has1, Ts in items if has1)
+    n_tiles1 = sum(sum(Ts) for has1, Ts in items if has1)
+    assert B["q_full"].phase == B["q_empty"].phase == len(items)
+    assert B["item_empty0"].phase + B["item_empty1"].phase == len(items) + 1
+    assert sum(B[f"k_empty{s}"].phase for s in range(STAGES)) == n_tiles
+    assert sum(B[f"v_empty{s}"].phase for s in range(STAGES)) == n_tiles
+    for k, (tiles, units) in enumerate(((n_tiles, n_units), (n_tiles1, n_units1))):
+        assert B[f"s_full{k}"].phase == B[f"s_free{k}"].phase == tiles
+        assert B[f"p_full{k}"].phase == B[f"p_free{k}"].phase == tiles
+        assert B[f"o_full{k}"].phase == B[f"o_empty{k}"].phase == units
+    assert B["drain"].phase == 1
+
+
+@pytest.mark.parametrize("items", [
+    [(False, [1])],
+    [(True, [1])],
+    [(True, [1] * 7)],
+    [(False, [2]), (True, [1]), (False, [3, 1])],
+    [(True, [9])],
+    [(False, [4]), (False, [1]), (True, [2, 2])],   # the second MMA warp follows two items idle
+], ids=["T1_tile0", "T1_both", "units_of_one_tile", "mixed", "long_unit", "idle_items"])
+def test_free_s_protocol_edge_items(items):
+    for seed in range(20):
+        run(items, seed, fs=True)
+
+
+@pytest.mark.parametrize("mut", ["fs_s_free_before_s_read", "fs_softmax_skips_p_free",
+                                 "fs_mma_skips_s_free", "fs_idle_warp_skips_release"])
+def test_free_s_planted_mistakes_are_caught(mut):
+    item_lists = [[(True, [3, 2]), (True, [1, 4]), (False, [2])],
+                  [(True, [3]), (False, [1]), (False, [1]), (True, [2])]]
+    caught = 0
+    for items in item_lists:
+        for seed in range(40):
+            try:
+                run(items, seed, mut=mut, fs=True)
+            except Violation:
+                caught += 1
+    assert caught > 0, mut
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_free_s_stop_path_after_a_timeout(seed):
+    rng = random.Random(7000 + seed)
+    items = random_items(rng)
+    aborted_runs = 0
+    for timeout_p in (0.002, 0.02, 0.2):
+        _, aborted = run(items, seed, timeout_p=timeout_p, fs=True)
+        aborted_runs += aborted
+    assert aborted_runs > 0
+
+
+@pytest.mark.parametrize("cta", [0, 147])
+def test_free_s_protocol_on_a_frame_tile_cta(cta):
+    """The d = 96 kernel on 8 frames of 3600 tokens: 96-key tiles, 38 per
+    unit (the last one 48 keys)."""
+    F, L = 8, 3600
+    part_off = [f * L for f in range(F + 1)]
+    fresh_rows = [[L] * len({0, f - 1, f, f + 1} & set(range(F))) for f in range(F)]
+    items = cta_items(part_off, fresh_rows, 24, cta, 148, BN=96)
+    assert {T for _, Ts in items for T in Ts} == {38}
+    B, aborted = run(items, cta, rescale_p=0.05, fs=True)
+    assert not aborted
+    assert B["p_free0"].phase == sum(sum(Ts) for _, Ts in items)
