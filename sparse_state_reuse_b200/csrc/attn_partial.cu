@@ -21,10 +21,11 @@
 //   warp  10   d = 64 and 96: the MMA issuer of Q tile 1; else idle
 //   warp  11   idle
 // Registers are rebalanced with setmaxnreg: the softmax warpgroups, which
-// hold a whole S row per thread, get kSoftmaxRegs; warpgroup 2 drops to
-// kControlRegs.  2 * 128 * 216 + 128 * 72 = 384 * 168, the registers the
-// CTA is launched with; the launcher refuses to launch a build whose
-// register count differs (an unbalanced split would block forever).
+// hold a whole S row per thread, get softmax_regs; warpgroup 2 drops to
+// control_regs.  2 * 128 * 216 + 128 * 72 = 2 * 128 * 192 + 128 * 120 =
+// 384 * 168, the registers the CTA is launched with; the launcher refuses to
+// launch a build whose register count differs (an unbalanced split would
+// block forever).
 // One thread owns one query row (TMEM lane), so row max and row sum need no
 // cross-thread reduction.  O is rescaled only when a row's running maximum
 // grows by more than 2^8 (exact: O and l share the stale maximum).
@@ -57,9 +58,17 @@ namespace attn {
 constexpr int BM = 128;            // query rows per tile
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;   // 65536 / 384, rounded down to a multiple of 8
-constexpr int kSoftmaxRegs = 216;
-constexpr int kControlRegs = 72;
-static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kThreads * kLaunchRegs,
+// Registers per thread after setmaxnreg: the softmax warpgroups hold a whole
+// S row (128 columns; 96 at d = 96), the control warpgroup the producer and
+// MMA loops.  At d = 96 the two MMA warps of the free-S pipeline need more
+// than 72 (they spilled inside their loops) and the 96-column softmax rows
+// fewer than 216.
+template <int D> __host__ __device__ constexpr int softmax_regs() { return D == 96 ? 192 : 216; }
+template <int D> __host__ __device__ constexpr int control_regs() { return D == 96 ? 120 : 72; }
+template <int D> __host__ __device__ constexpr bool split_ok() {
+  return 2 * 128 * softmax_regs<D>() + 128 * control_regs<D>() == kThreads * kLaunchRegs;
+}
+static_assert(split_ok<64>() && split_ok<96>() && split_ok<128>(),
               "register split must equal the launch budget");
 constexpr int kStages = 2;         // K ring and V ring depth
 constexpr float kRescaleLog2 = 8.0f;
@@ -493,7 +502,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 8) {
-   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(control_regs<D>()));
    if (warp == 8) {
     // ------------------------------------------------------------ producer
     // Warp-uniform loop; one elected lane arms the barriers and issues TMA.
@@ -828,7 +837,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     return;
   } else {
     // ------------------------------------------------------------ softmax
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(softmax_regs<D>()));
     const int k = warp >> 2;                 // Q tile of this warpgroup
     const int r = threadIdx.x & 127;         // row within the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
