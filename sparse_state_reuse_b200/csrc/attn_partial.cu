@@ -630,8 +630,12 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       static_assert(kStages == 2, "descriptor selection assumes two stages");
       auto qk = [&](int k, int ks) {
         // S_k = Q_k K^T : K-major A and B, 16 columns of d per instruction
-        const uint64_t a0 = k ? dQ1 : dQ0;
-        const uint64_t b0 = ks ? dK1 : dK0;
+        uint64_t a0 = k ? dQ1 : dQ0;
+        uint64_t b0 = ks ? dK1 : dK0;
+        // opaque to the compiler: the per-step descriptors are formed at each
+        // use instead of all being hoisted into registers of this warp
+        asm volatile("mov.b64 %0, %0;" : "+l"(a0));
+        asm volatile("mov.b64 %0, %0;" : "+l"(b0));
         const uint32_t d_tmem = tmem + C::S_COL(k);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -642,7 +646,8 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       };
       auto pv = [&](int k, int vs, bool acc) {
         // O_k (+)= P_k V : P from TMEM (K-major), V MN-major (d contiguous)
-        const uint64_t b0 = vs ? dV1 : dV0;
+        uint64_t b0 = vs ? dV1 : dV0;
+        asm volatile("mov.b64 %0, %0;" : "+l"(b0));
         const uint32_t d_tmem = tmem + C::O_COL(k);
         const uint32_t a_tmem = tmem + C::P_COL(k);
 #pragma unroll
