@@ -22,6 +22,7 @@ import json
 import os
 import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -157,6 +158,69 @@ class ClockSampler:
         return summarise_clocks(out)
 
 
+class NvmlClockSampler:
+    """SM clock and throttle reasons read through NVML every `period` seconds
+    by a thread, between start() and stop(); reads only, changes nothing.
+    The GPU is found by its PCI bus id (the CUDA device this rank runs on,
+    whatever CUDA_VISIBLE_DEVICES maps), else by index."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown"}
+
+    def __init__(self, gpu_index, pci_bus_id=None, period=0.01, nvml=None):
+        self.idx, self.bus, self.period, self.nvml = gpu_index, pci_bus_id, period, nvml
+        self.rows, self.thread, self.halt = [], None, threading.Event()
+
+    def start(self):
+        try:
+            nv = self.nvml
+            if nv is None:
+                import pynvml as nv
+            nv.nvmlInit()
+            h = (nv.nvmlDeviceGetHandleByPciBusId(self.bus) if self.bus
+                 else nv.nvmlDeviceGetHandleByIndex(self.idx))
+            reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            clock = lambda: nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)  # noqa: E731
+            top = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except Exception:
+            return False
+        self.nv = nv
+
+        def loop():
+            while not self.halt.is_set():
+                try:
+                    self.rows.append((float(clock()), float(top), int(reasons(h))))
+                except Exception:
+                    pass
+                self.halt.wait(self.period)
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
+        return True
+
+    def stop(self):
+        if self.thread is None:
+            return None
+        self.halt.set()
+        self.thread.join(timeout=2)
+        try:
+            self.nv.nvmlShutdown()
+        except Exception:
+            pass
+        return summarise_nvml(self.rows)
+
+
+def summarise_nvml(rows):
+    """The summarise_clocks record from NVML samples (SM MHz, max SM MHz,
+    event-reason bit mask); None without samples."""
+    if not rows:
+        return None
+    reasons = sorted({name for _, _, mask in rows for bit, name in NvmlClockSampler.REASONS.items()
+                      if mask & bit})
+    return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": max(r[1] for r in rows),
+            "reasons": reasons, "samples": len(rows)}
+
+
 def summarise_clocks(csv_text):
     """Median SM clock, the highest max clock and every throttle reason seen
     Active, from nvidia-smi lines of ClockSampler.FIELDS (no header, no
@@ -255,15 +319,24 @@ def run_ours(args, w, rank, world, local_rank):
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
-    clk = ClockSampler(local_rank)
+    bus = getattr(torch.cuda.get_device_properties(dev), "pci_bus_id", None)
+    pci = (f"{getattr(torch.cuda.get_device_properties(dev), 'pci_domain_id', 0):08x}:{bus:02x}:"
+           f"{getattr(torch.cuda.get_device_properties(dev), 'pci_device_id', 0):02x}.0"
+           if bus is not None else None)
+    clk = ClockSampler(local_rank)            # nvidia-smi: the fallback record
     clk.start()
     time.sleep(0.3)
+    nv = NvmlClockSampler(local_rank, pci.encode() if pci else None)
+    stream.synchronize()
     e_start.record(stream)
+    nv_on = nv.start()                        # NVML samples span the timed region only
     for t in range(args.steps):
         one_step(t)
     e_end.record(stream)
     stream.synchronize()
-    clocks = clk.stop()
+    nv_clocks = nv.stop() if nv_on else None
+    smi_clocks = clk.stop()
+    clocks = nv_clocks or smi_clocks
     torch.cuda.synchronize()
     ms = e_start.elapsed_time(e_end)
     part_ms = float(np.mean([e_part0[t].elapsed_time(e_part1[t]) for t in range(n_ev)]))
