@@ -22,7 +22,6 @@ import json
 import os
 import subprocess
 import sys
-import threading
 import time
 
 import numpy as np
@@ -129,24 +128,30 @@ def aggregate_tflops(world, flops_per_replica, ms_per_step):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi in a process of its own (it takes nothing from this one)
+    samples the GPU every 20 ms with a timestamp; stop(t0, t1) keeps the
+    samples taken inside the timed region [t0, t1] (host wall clock), or the
+    first one after t0 when the region is shorter than the sampling period.
+    Reads only, changes nothing."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, period_ms=20):
         self.idx = gpu_index
+        self.period_ms = period_ms
         self.proc = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t0=None, t1=None):
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -155,82 +160,41 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        return summarise_clocks(out)
+        return summarise_clocks(out, t0, t1)
 
 
-class NvmlClockSampler:
-    """SM clock and throttle reasons read through NVML every `period` seconds
-    by a thread, between start() and stop(); reads only, changes nothing.
-    The GPU is found by its PCI bus id (the CUDA device this rank runs on,
-    whatever CUDA_VISIBLE_DEVICES maps), else by index."""
-    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
-               0x40: "hw_thermal_slowdown"}
-
-    def __init__(self, gpu_index, pci_bus_id=None, period=0.01, nvml=None):
-        self.idx, self.bus, self.period, self.nvml = gpu_index, pci_bus_id, period, nvml
-        self.rows, self.thread, self.halt = [], None, threading.Event()
-
-    def start(self):
-        try:
-            nv = self.nvml
-            if nv is None:
-                import pynvml as nv
-            nv.nvmlInit()
-            h = (nv.nvmlDeviceGetHandleByPciBusId(self.bus) if self.bus
-                 else nv.nvmlDeviceGetHandleByIndex(self.idx))
-            reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-                nv.nvmlDeviceGetCurrentClocksThrottleReasons
-            clock = lambda: nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)  # noqa: E731
-            top = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-        except Exception:
-            return False
-        self.nv = nv
-
-        def loop():
-            while not self.halt.is_set():
-                try:
-                    self.rows.append((float(clock()), float(top), int(reasons(h))))
-                except Exception:
-                    pass
-                self.halt.wait(self.period)
-
-        self.thread = threading.Thread(target=loop, daemon=True)
-        self.thread.start()
-        return True
-
-    def stop(self):
-        if self.thread is None:
-            return None
-        self.halt.set()
-        self.thread.join(timeout=2)
-        try:
-            self.nv.nvmlShutdown()
-        except Exception:
-            pass
-        return summarise_nvml(self.rows)
-
-
-def summarise_nvml(rows):
-    """The summarise_clocks record from NVML samples (SM MHz, max SM MHz,
-    event-reason bit mask); None without samples."""
-    if not rows:
+def _smi_time(stamp):
+    """Host epoch seconds of an nvidia-smi timestamp (local time,
+    "YYYY/MM/DD HH:MM:SS.mmm"), or None."""
+    try:
+        day, clock = stamp.split(" ")
+        whole, _, frac = clock.partition(".")
+        st = time.strptime(f"{day} {whole}", "%Y/%m/%d %H:%M:%S")
+        return time.mktime(st) + (float("0." + frac) if frac else 0.0)
+    except ValueError:
         return None
-    reasons = sorted({name for _, _, mask in rows for bit, name in NvmlClockSampler.REASONS.items()
-                      if mask & bit})
-    return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": max(r[1] for r in rows),
-            "reasons": reasons, "samples": len(rows)}
 
 
-def summarise_clocks(csv_text):
+def summarise_clocks(csv_text, t0=None, t1=None):
     """Median SM clock, the highest max clock and every throttle reason seen
     Active, from nvidia-smi lines of ClockSampler.FIELDS (no header, no
-    units); None when no line parses."""
-    sm, mx, reasons = [], 0.0, set()
-    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    units); with t0/t1, only the lines stamped inside [t0, t1], else the
+    first line after t0.  None when no line qualifies."""
+    lines = []
     for line in csv_text.strip().splitlines():
         parts = [x.strip() for x in line.split(",")]
-        if len(parts) < 9:
+        if len(parts) < 10:
             continue
+        lines.append((_smi_time(parts[0]), parts[1:]))
+    if t0 is not None and t1 is not None:
+        inside = [ln for ln in lines if ln[0] is not None and t0 <= ln[0] <= t1]
+        if not inside:
+            after = [ln for ln in lines if ln[0] is not None and ln[0] >= t0]
+            inside = after[:1]
+        lines = inside
+    sm, mx, reasons = [], 0.0, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for _, parts in lines:
         try:
             sm.append(float(parts[1]))
             mx = max(mx, float(parts[2]))
@@ -319,24 +283,18 @@ def run_ours(args, w, rank, world, local_rank):
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
-    bus = getattr(torch.cuda.get_device_properties(dev), "pci_bus_id", None)
-    pci = (f"{getattr(torch.cuda.get_device_properties(dev), 'pci_domain_id', 0):08x}:{bus:02x}:"
-           f"{getattr(torch.cuda.get_device_properties(dev), 'pci_device_id', 0):02x}.0"
-           if bus is not None else None)
-    clk = ClockSampler(local_rank)            # nvidia-smi: the fallback record
+    clk = ClockSampler(local_rank)
     clk.start()
-    time.sleep(0.3)
-    nv = NvmlClockSampler(local_rank, pci.encode() if pci else None)
+    time.sleep(0.5)                           # nvidia-smi is sampling by now
     stream.synchronize()
+    t_wall0 = time.time()
     e_start.record(stream)
-    nv_on = nv.start()                        # NVML samples span the timed region only
     for t in range(args.steps):
         one_step(t)
     e_end.record(stream)
     stream.synchronize()
-    nv_clocks = nv.stop() if nv_on else None
-    smi_clocks = clk.stop()
-    clocks = nv_clocks or smi_clocks
+    t_wall1 = time.time()
+    clocks = clk.stop(t_wall0, t_wall1)       # the samples of the timed region
     torch.cuda.synchronize()
     ms = e_start.elapsed_time(e_end)
     part_ms = float(np.mean([e_part0[t].elapsed_time(e_part1[t]) for t in range(n_ev)]))
