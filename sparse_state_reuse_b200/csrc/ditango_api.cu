@@ -425,6 +425,8 @@ ditango_status ditango_merge(const ditango_geom *g, const int8_t *plan, const vo
   if ((cache_O == nullptr) != (cache_lse == nullptr)) return DITANGO_ERR_INVALID;
   if (part_O == nullptr && cache_O == nullptr) return DITANGO_ERR_INVALID;
   if (writeback && part_O && !cache_O) return DITANGO_ERR_INVALID;
+  // the merge moves state rows in 16-byte groups
+  if ((part_O && !aligned16(part_O)) || (cache_O && !aligned16(cache_O))) return DITANGO_ERR_INVALID;
   long long osb = (long long)dg.H * dg.N * dg.d, osh = (long long)dg.N * dg.d, osn = dg.d;
   if (out_strides) {
     osb = out_strides[0];

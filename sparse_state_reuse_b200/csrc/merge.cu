@@ -12,9 +12,10 @@
 // partition).  Phase 1: one thread per row reads the row's lse of every
 // state and writes the weights to shared memory (weights.cuh, the same
 // arithmetic as the plan's mass score).  Phase 2: the block's rows of each
-// state are one contiguous run of memory, streamed as a flat array of 4-value
-// groups by all threads -- coalesced whatever d is, no idle lanes -- with
-// several states' loads of several groups in flight per thread.  Optionally
+// state are one contiguous run of memory, streamed as a flat array of 16-byte
+// groups (4 fp32 or 8 bf16 values) by all threads -- coalesced whatever d is,
+// no idle lanes -- with several states' loads of several groups in flight per
+// thread.  Optionally
 // the block also writes its sums of the weights ("mass partials"): the
 // importance w of the next step's plan, so that the plan need not read the
 // cache again.
@@ -33,43 +34,10 @@ constexpr int kWarps = kThreads / 32;
 // ditango_check_status.
 __device__ int g_merge_check_status;
 
-// Raw form of four stored O values (kept packed until used).
-template <bool SB>
-struct Raw4 {
-  using T = float4;
-};
-template <>
-struct Raw4<true> {
-  using T = uint2;
-};
-template <bool SB>
-__device__ __forceinline__ typename Raw4<SB>::T load_raw4(const char *p) {
-  if constexpr (SB)
-    return __ldg(reinterpret_cast<const uint2 *>(p));
-  else
-    return __ldg(reinterpret_cast<const float4 *>(p));
-}
-template <bool SB>
-__device__ __forceinline__ float4 widen4(typename Raw4<SB>::T u) {
-  if constexpr (SB)
-    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
-                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
-  else
-    return u;
-}
-template <bool SB>
-__device__ __forceinline__ typename Raw4<SB>::T zero_raw4() {
-  if constexpr (SB)
-    return make_uint2(0u, 0u);
-  else
-    return make_float4(0.f, 0.f, 0.f, 0.f);
-}
-template <bool SB>
-__device__ __forceinline__ void store_raw4(char *p, typename Raw4<SB>::T u) {
-  if constexpr (SB)
-    *reinterpret_cast<uint2 *>(p) = u;
-  else
-    *reinterpret_cast<float4 *>(p) = u;
+// Four bf16 values (two packed pairs, low element first) as floats.
+__device__ __forceinline__ float4 widen_bf16x4(uint32_t lo, uint32_t hi) {
+  return make_float4(__uint_as_float(lo << 16), __uint_as_float(lo & 0xffff0000u),
+                     __uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u));
 }
 
 __device__ __forceinline__ void store_out(void *out, int is_fp32, size_t off, float4 v) {
@@ -92,6 +60,70 @@ __device__ __forceinline__ void fma4(float4 &acc, float w, const float4 &v) {
   acc.w = fmaf(w, v.w, acc.w);
 }
 
+// The merge's unit of streaming: 16 bytes of one stored state row, i.e. 4
+// fp32 values or 8 bf16 values, kept packed until used.
+template <bool SB>
+struct Grp {
+  static constexpr int V = 4;               // values per group
+  using Raw = float4;
+  struct Acc { float4 a; };
+};
+template <>
+struct Grp<true> {
+  static constexpr int V = 8;
+  using Raw = uint4;
+  struct Acc { float4 a, b; };
+};
+template <bool SB>
+__device__ __forceinline__ typename Grp<SB>::Raw load_grp(const char *p) {
+  return __ldg(reinterpret_cast<const typename Grp<SB>::Raw *>(p));
+}
+template <bool SB>
+__device__ __forceinline__ typename Grp<SB>::Raw zero_grp() {
+  typename Grp<SB>::Raw r;
+  if constexpr (SB) r = make_uint4(0u, 0u, 0u, 0u); else r = make_float4(0.f, 0.f, 0.f, 0.f);
+  return r;
+}
+template <bool SB>
+__device__ __forceinline__ void store_grp(char *p, typename Grp<SB>::Raw u) {
+  *reinterpret_cast<typename Grp<SB>::Raw *>(p) = u;
+}
+template <bool SB>
+__device__ __forceinline__ void zero_acc(typename Grp<SB>::Acc &acc) {
+  acc.a = make_float4(0.f, 0.f, 0.f, 0.f);
+  if constexpr (SB) acc.b = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+template <bool SB>
+__device__ __forceinline__ void fma_grp(typename Grp<SB>::Acc &acc, float w, typename Grp<SB>::Raw u) {
+  if constexpr (SB) {
+    fma4(acc.a, w, widen_bf16x4(u.x, u.y));
+    fma4(acc.b, w, widen_bf16x4(u.z, u.w));
+  } else {
+    fma4(acc.a, w, u);
+  }
+}
+// The merged group to the output (fp32 or bf16 elements at element offset off).
+template <bool SB>
+__device__ __forceinline__ void store_out_grp(void *out, int is_fp32, size_t off,
+                                              const typename Grp<SB>::Acc &acc) {
+  if constexpr (SB) {
+    if (is_fp32) {
+      *reinterpret_cast<float4 *>(static_cast<float *>(out) + off) = acc.a;
+      *reinterpret_cast<float4 *>(static_cast<float *>(out) + off + 4) = acc.b;
+    } else {
+      uint4 u;
+      __nv_bfloat162 t;
+      t = __floats2bfloat162_rn(acc.a.x, acc.a.y); u.x = *reinterpret_cast<uint32_t *>(&t);
+      t = __floats2bfloat162_rn(acc.a.z, acc.a.w); u.y = *reinterpret_cast<uint32_t *>(&t);
+      t = __floats2bfloat162_rn(acc.b.x, acc.b.y); u.z = *reinterpret_cast<uint32_t *>(&t);
+      t = __floats2bfloat162_rn(acc.b.z, acc.b.w); u.w = *reinterpret_cast<uint32_t *>(&t);
+      *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + off) = u;
+    }
+  } else {
+    store_out(out, is_fp32, off, acc.a);
+  }
+}
+
 // Merge of one block of rows (see the file comment).  Dynamic shared memory:
 // the weights, [states][kWRows] floats.
 template <int D, bool SB>
@@ -100,10 +132,11 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
              const float *__restrict__ part_lse, char *cache_O, float *cache_lse,
              unsigned char *cache_valid, int writeback, void *out, int out_is_fp32, long long osb,
              long long osh, long long osn, float *__restrict__ out_lse, float *__restrict__ mass) {
-  constexpr int Q4 = D / 4;                 // 4-value groups per row
+  constexpr int VG = Grp<SB>::V;            // values per 16-byte group
+  constexpr int QG = D / VG;                // groups per row
   constexpr int ES = SB ? 2 : 4;            // bytes per stored O element
   constexpr size_t ROWB = (size_t)D * ES;   // bytes per state row
-  constexpr int U = SB ? 4 : 2;             // groups per thread per pass
+  constexpr int U = 2;                      // groups per thread per pass
   constexpr int SBATCH = 4;                 // states per batch of loads
   using weights::kWRows;
   const int i = blockIdx.y;
@@ -205,27 +238,27 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
     }
   }
 
-  // ---- phase 2: stream the states' rows as one flat array of 4-value groups
-  const int n4 = nrows * Q4;
+  // ---- phase 2: stream the states' rows as one flat array of 16-byte groups
+  const int ng = nrows * QG;
   const size_t obase = (size_t)b * osb + (size_t)h * osh;
-  for (int f0 = threadIdx.x; f0 < n4; f0 += kThreads * U) {
-    float4 acc[U];
+  for (int f0 = threadIdx.x; f0 < ng; f0 += kThreads * U) {
+    typename Grp<SB>::Acc acc[U];
     int row[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      row[u] = (f0 + u * kThreads) / Q4;
+      zero_acc<SB>(acc[u]);
+      row[u] = (f0 + u * kThreads) / QG;
     }
     for (int a0 = 0; a0 < n; a0 += SBATCH) {
-      typename Raw4<SB>::T v[SBATCH][U];
+      typename Grp<SB>::Raw v[SBATCH][U];
 #pragma unroll
       for (int q = 0; q < SBATCH; ++q) {
         const char *src = (a0 + q < n) ? s_O[a0 + q] : nullptr;
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int f = f0 + u * kThreads;
-          v[q][u] = zero_raw4<SB>();
-          if (src != nullptr && f < n4) v[q][u] = load_raw4<SB>(src + (size_t)f * 4 * ES);
+          v[q][u] = zero_grp<SB>();
+          if (src != nullptr && f < ng) v[q][u] = load_grp<SB>(src + (size_t)f * 16);
         }
       }
 #pragma unroll
@@ -236,9 +269,9 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int f = f0 + u * kThreads;
-          if (f < n4) {
-            fma4(acc[u], wq[row[u]], widen4<SB>(v[q][u]));
-            if (wb != nullptr) store_raw4<SB>(wb + (size_t)f * 4 * ES, v[q][u]);
+          if (f < ng) {
+            fma_grp<SB>(acc[u], wq[row[u]], v[q][u]);
+            if (wb != nullptr) store_grp<SB>(wb + (size_t)f * 16, v[q][u]);
           }
         }
       }
@@ -246,9 +279,9 @@ merge_kernel(DevGeom g, const signed char *__restrict__ plan, const char *__rest
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int f = f0 + u * kThreads;
-      if (f < n4)
-        store_out(out, out_is_fp32, obase + (size_t)(tok0 + row[u]) * osn + (f - row[u] * Q4) * 4,
-                  acc[u]);
+      if (f < ng)
+        store_out_grp<SB>(out, out_is_fp32,
+                          obase + (size_t)(tok0 + row[u]) * osn + (size_t)(f - row[u] * QG) * VG, acc[u]);
     }
   }
 }
@@ -315,10 +348,11 @@ __global__ void __launch_bounds__(kThreads, 3)
 compose_kernel(DevGeom fine, DevGeom coarse, const char *__restrict__ fO,
                const float *__restrict__ flse, const unsigned char *__restrict__ fvalid,
                char *__restrict__ cO, float *__restrict__ clse, unsigned char *cvalid) {
-  constexpr int Q4 = D / 4;                 // 4-value groups per row
+  constexpr int VG = Grp<SB>::V;            // values per 16-byte group
+  constexpr int QG = D / VG;                // groups per row
   constexpr int ES = SB ? 2 : 4;
   constexpr size_t ROWB = (size_t)D * ES;
-  constexpr int U = SB ? 4 : 2;             // groups per thread per pass
+  constexpr int U = 2;                      // groups per thread per pass
   constexpr int SBATCH = 4;                 // states per batch of loads
   using weights::kWRows;
   const int cslot = blockIdx.y;
@@ -367,26 +401,26 @@ compose_kernel(DevGeom fine, DevGeom coarse, const char *__restrict__ fO,
   }
   __syncthreads();
 
-  // ---- phase 2: the fine rows, weighted, into the coarse rows
-  const int n4 = nrows * Q4;
-  for (int f0 = threadIdx.x; f0 < n4; f0 += kThreads * U) {
-    float4 acc[U];
+  // ---- phase 2: the fine rows, weighted, into the coarse rows (16-byte groups)
+  const int ng = nrows * QG;
+  for (int f0 = threadIdx.x; f0 < ng; f0 += kThreads * U) {
+    typename Grp<SB>::Acc acc[U];
     int row[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      row[u] = (f0 + u * kThreads) / Q4;
+      zero_acc<SB>(acc[u]);
+      row[u] = (f0 + u * kThreads) / QG;
     }
     for (int a0 = 0; a0 < nf; a0 += SBATCH) {
-      typename Raw4<SB>::T v[SBATCH][U];
+      typename Grp<SB>::Raw v[SBATCH][U];
 #pragma unroll
       for (int q = 0; q < SBATCH; ++q) {
         const char *src = (a0 + q < nf) ? s_O[a0 + q] : nullptr;
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int f = f0 + u * kThreads;
-          v[q][u] = zero_raw4<SB>();
-          if (src != nullptr && f < n4) v[q][u] = load_raw4<SB>(src + (size_t)f * 4 * ES);
+          v[q][u] = zero_grp<SB>();
+          if (src != nullptr && f < ng) v[q][u] = load_grp<SB>(src + (size_t)f * 16);
         }
       }
 #pragma unroll
@@ -395,13 +429,13 @@ compose_kernel(DevGeom fine, DevGeom coarse, const char *__restrict__ fO,
         const float *wq = sh + (a0 + q) * kWRows;
 #pragma unroll
         for (int u = 0; u < U; ++u)
-          if (f0 + u * kThreads < n4) fma4(acc[u], wq[row[u]], widen4<SB>(v[q][u]));
+          if (f0 + u * kThreads < ng) fma_grp<SB>(acc[u], wq[row[u]], v[q][u]);
       }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int f = f0 + u * kThreads;
-      if (f < n4) store_out(dstO, SB ? 0 : 1, (size_t)f * 4, acc[u]);
+      if (f < ng) store_out_grp<SB>(dstO, SB ? 0 : 1, (size_t)f * VG, acc[u]);
     }
   }
 }
