@@ -370,7 +370,9 @@ def run_ours(args, w, rank, world, local_rank):
     peak_t = float(peaks.get("bf16_tflops"))          # burst figure: the conservative denominator
     peak_ts = float(peaks.get("bf16_tflops_sustained", peak_t))
     merge_gbs = mbytes / (merge_ms * 1e-3) / 1e9
-    traffic = recorded_traffic("attn_partial.cu", w.name)
+    # recorded DRAM bytes are per state format (a bf16 cache moves half the bytes)
+    tkey = w.name + (":bf16" if args.state_bf16 else "")
+    traffic = recorded_traffic("attn_partial.cu", tkey)
     res = {
         "metric": "effective attention TFLOP/s (fresh blocks only) at 1 B200; tokens/s",
         "value": round(aggregate_tflops(world, flops, ms_step), 3),
@@ -403,7 +405,7 @@ def run_ours(args, w, rank, world, local_rank):
                            "frac": round(merge_gbs / float(peaks.get("hbm_gbs")), 4),
                            "kernel_ms": round(merge_ms, 4),
                            "algorithmic_bytes_per_launch": mbytes,
-                           "traffic": recorded_traffic("merge.cu", w.name)},
+                           "traffic": recorded_traffic("merge.cu", tkey)},
         "plan": {"us": round(plan_us, 2), "launches": 1 if w.anchor else 2,
                  "note": "anchor steps: the selection alone; reuse steps: the mass score from the "
                          "previous step's merge (its block sums reduced per unit) and the selection"},
@@ -534,7 +536,8 @@ def measure_compose(w, pa, Q, K, V, dev, stream, args, peaks):
                                     + pa.state_lse.numel() * 4),
            "ms": round(ms, 4), "bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s",
            "peak": float(peaks.get("hbm_gbs")), "frac": round(gbs / float(peaks.get("hbm_gbs")), 4),
-           "algorithmic_bytes_per_launch": nbytes, "traffic": recorded_traffic("merge.cu", w.name + ":compose")}
+           "algorithmic_bytes_per_launch": nbytes,
+           "traffic": recorded_traffic("merge.cu", w.name + (":bf16" if args.state_bf16 else "") + ":compose")}
     del fine
     torch.cuda.empty_cache()
     return out
