@@ -36,8 +36,9 @@
 // P V and next Q K^T (which waits for that P V, since P lives in S).
 // d = 64 and 96 ("free S"): P_k has TMEM columns of its own (Cfg::P_COL),
 // so each softmax warp signals s_free as soon as S is in its registers and
-// the next Q K^T runs under its exponentials; before writing P again it
-// waits on p_free (the P V that read the previous P is done).  Each Q tile
+// the next Q K^T runs under its exponentials; it forms the whole P row in
+// registers and only then waits on p_free (the P V that read the previous P
+// is done, normally long before) to overwrite P_k.  Each Q tile
 // has its own MMA warp, so neither tile waits for the other's events.
 // Work items go from the producer warp to the other roles through a 2-slot
 // ring in shared memory; with a work counter each CTA takes the next item
@@ -956,29 +957,50 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // (general variant) a row with no admissible key so far exponentiates against 0
         const float neg = (MR && !(m_used > -INFINITY)) ? 0.f : -m_used;
         const uint64_t sl2x2 = f2(sl2, sl2), negx2 = f2(neg, neg);
+        uint64_t lsum0 = 0, lsum1 = 0;   // packed partial row sums (+0.0f bits)
         if constexpr (FS) {
-          // P_k is overwritten below: the P V that read it must be done
+          // The whole P row is formed in registers first.  P_k is then
+          // overwritten, once the P V that read it is done: by the end of the
+          // exponentials it normally is, so this wait no longer sits between
+          // the row maximum and the exponentials.
+          uint32_t pk[BN / 2];
+#pragma unroll
+          for (int e = 0; e < BN / 2; ++e) {
+            const int c = 2 * e;
+            float xa, xb;
+            unf2(fma2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, negx2), xa, xb);
+            const float a = (2 * (e % 8) < emu_per16<D>()) ? exp2_poly(xa) : ex2(xa);
+            const float b = (2 * (e % 8) + 1 < emu_per16<D>()) ? exp2_poly(xb) : ex2(xb);
+            if (e & 1) lsum1 = add2(lsum1, f2(a, b)); else lsum0 = add2(lsum0, f2(a, b));
+            pk[e] = pack_bf16(a, b);
+          }
           if (!pv_done) {
             if (!(ok = wait_bounded(p_free(k), (pst - 1) & 1, ctl))) break;
             tc_fence_after();
           }
-        }
-        uint64_t lsum0 = 0, lsum1 = 0;   // packed partial row sums (+0.0f bits)
 #pragma unroll
-        for (int g8 = 0; g8 < BN / 16; ++g8) {
-          // 16 probabilities -> 8 packed bf16 pairs -> TMEM columns [8*g8, 8*g8+8)
-          uint32_t pk[8];
+          for (int g8 = 0; g8 < BN / 16; ++g8)
+            tmem_st8(tP + g8 * 8, pk[g8 * 8 + 0], pk[g8 * 8 + 1], pk[g8 * 8 + 2], pk[g8 * 8 + 3],
+                     pk[g8 * 8 + 4], pk[g8 * 8 + 5], pk[g8 * 8 + 6], pk[g8 * 8 + 7]);
+        } else {
+          // P overwrites S_k: stored 16 probabilities at a time, under the
+          // exponentials
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int c = g8 * 16 + 2 * e;
-            float xa, xb;
-            unf2(fma2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, negx2), xa, xb);
-            const float a = (2 * e < emu_per16<D>()) ? exp2_poly(xa) : ex2(xa);
-            const float b = (2 * e + 1 < emu_per16<D>()) ? exp2_poly(xb) : ex2(xb);
-            if (e & 1) lsum1 = add2(lsum1, f2(a, b)); else lsum0 = add2(lsum0, f2(a, b));
-            pk[e] = pack_bf16(a, b);
+          for (int g8 = 0; g8 < BN / 16; ++g8) {
+            // 16 probabilities -> 8 packed bf16 pairs -> TMEM columns [8*g8, 8*g8+8)
+            uint32_t pk[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int c = g8 * 16 + 2 * e;
+              float xa, xb;
+              unf2(fma2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, negx2), xa, xb);
+              const float a = (2 * e < emu_per16<D>()) ? exp2_poly(xa) : ex2(xa);
+              const float b = (2 * e + 1 < emu_per16<D>()) ? exp2_poly(xb) : ex2(xb);
+              if (e & 1) lsum1 = add2(lsum1, f2(a, b)); else lsum0 = add2(lsum0, f2(a, b));
+              pk[e] = pack_bf16(a, b);
+            }
+            tmem_st8(tP + g8 * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
           }
-          tmem_st8(tP + g8 * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
         }
         {
           float s0, s1, s2, s3;

@@ -481,6 +481,8 @@ def softmax_warp_fs(k, items, rng, rescale_p, mut):
                         pv_done = True
                     yield ("hold", O, "w")             # O *= alpha
                     yield ("release", O)
+                # the P row is formed in registers (no TMEM access) before
+                # this wait; only its store touches P_k
                 if not pv_done:
                     ok = yield W(f"p_free{k}", (pst - 1) & 1, pst - 1)
                     if not ok:
